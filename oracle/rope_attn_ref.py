@@ -1,0 +1,262 @@
+"""Float64 CPU oracle for exact RoPE / LeRoPE softmax attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use it.  It shares no code with the CUDA path.
+
+What it computes, per (batch b, head h), with positions p = 0..n-1 and
+M = d/2 frequency bands:
+
+1.  theta_m = base^(-2m/d), theta_hat_m = exp(alpha_m) * theta_m.
+    ("LeRoPE: learnable RoPE frequencies", Metodologia: LeRoPE / Mecanismo
+    Central -- the effective frequency is the standard RoPE frequency rescaled
+    by a learned exponential; the standard frequencies form a geometric
+    sequence set by the base b, Declaracao do Problema.  The exponent -2m/d is
+    the standard RoPE choice; the page leaves it open.)
+2.  Band m of each query/key is rotated in its 2-D plane by the angle
+    p * theta_hat_m ("LeRoPE", Declaracao do Problema: RoPE rotates queries and
+    keys in two-dimensional frequency bands).  Band m is the pair of
+    coordinates (2m, 2m+1) ("interleaved", the default) or (m, m+M)
+    ("halfsplit"); the choice is a fixed column permutation.
+3.  S = Q~ K~^T / sqrt(d); causal: S_ij = -inf for j > i.
+4.  P = D^-1 exp(S) with D the diagonal of row sums -- the normalised softmax
+    s(x) of "RoPE attention can be trained in almost-linear time",
+    Metodologia 1 (closed-form gradient); O = P V; lse_i = log sum_j exp(S_ij).
+5.  L = 1/2 ||O - E||_F^2 and dO = O - E: the error term l(x), the difference
+    between the attention output and the target (same page, Metodologia 1).
+6.  dV = P^T dO; beta = dP = dO V^T (the error combined with the value matrix);
+    gamma = diag(s) beta - s s^T beta row by row, i.e. dS = P o (dP - rowsum(P o dP))
+    (same page, Metodologia 1 and 2, gamma_1 - gamma_2).
+7.  dQ~ = dS K~ / sqrt(d), dK~ = dS^T Q~ / sqrt(d); dQ, dK = band-wise rotation
+    by -p * theta_hat_m of dQ~, dK~ (the transpose of step 2).
+8.  dalpha_m = theta_hat_m * sum_{b,h,p} p * (<dQ~_pm, J q~_pm> + <dK~_pm, J k~_pm>),
+    J = [[0, -1], [1, 0]] (the derivative of a 2-D rotation), with alpha shared
+    by every head ("LeRoPE", Escolhas de Design Principais: one set of d/2
+    frequencies shared across all layers and heads; log-space parametrisation).
+
+A second, independent formula for dalpha -- the derivative of the real part of
+the DTFT of the offset-aggregated gradient signal ("LeRoPE", Analise Teorica)
+-- is :func:`dalpha_offset_dtft`.
+
+Everything is float64.  Inputs are the values the GPU sees (already rounded
+to the storage dtype), widened exactly.  Query rows are processed in blocks of
+full rows, so each row's softmax is the plain definition.
+"""
+import numpy as np
+
+
+# --------------------------------------------------------------------------
+# step 1-2: frequencies, angles, band rotation
+# --------------------------------------------------------------------------
+def frequencies(d, base, alpha):
+    """theta_m = base^(-2m/d) and theta_hat_m = exp(alpha_m) theta_m, m < d/2."""
+    M = d // 2
+    m = np.arange(M, dtype=np.float64)
+    theta = np.power(float(base), -2.0 * m / d)
+    theta_hat = np.exp(np.asarray(alpha, dtype=np.float64)) * theta
+    return theta, theta_hat
+
+
+def angles(n, theta_hat, offset=0):
+    """phi[p, m] = (p + offset) * theta_hat_m for positions p = 0..n-1."""
+    p = np.arange(n, dtype=np.float64) + offset
+    return p[:, None] * np.asarray(theta_hat, dtype=np.float64)[None, :]
+
+
+def band_index(d, pairing="interleaved"):
+    """Column indices (first, second) of each band's 2-D plane."""
+    M = d // 2
+    if pairing == "interleaved":
+        return np.arange(0, d, 2), np.arange(1, d, 2)
+    if pairing == "halfsplit":
+        return np.arange(M), np.arange(M, d)
+    raise ValueError(pairing)
+
+
+def rotate(x, phi, pairing="interleaved", sign=1.0):
+    """Rotate band m of row p of x ([..., n, d]) by sign * phi[p, m]."""
+    i0, i1 = band_index(x.shape[-1], pairing)
+    c, s = np.cos(phi), sign * np.sin(phi)
+    y = np.empty_like(x, dtype=np.float64)
+    x0, x1 = x[..., i0], x[..., i1]
+    y[..., i0] = c * x0 - s * x1
+    y[..., i1] = s * x0 + c * x1
+    return y
+
+
+def j_pair(x, pairing="interleaved"):
+    """J x band-wise: (x0, x1) -> (-x1, x0)."""
+    i0, i1 = band_index(x.shape[-1], pairing)
+    y = np.empty_like(x, dtype=np.float64)
+    y[..., i0] = -x[..., i1]
+    y[..., i1] = x[..., i0]
+    return y
+
+
+# --------------------------------------------------------------------------
+# steps 3-7 for one head, in blocks of full query rows
+# --------------------------------------------------------------------------
+def _scores(qt_rows, kt, rows, causal, scale):
+    s = (qt_rows @ kt.T) * scale
+    if causal:
+        cols = np.arange(kt.shape[0])
+        s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+    return s
+
+
+def _softmax_rows(s):
+    mx = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - mx)
+    z = np.sum(e, axis=1, keepdims=True)
+    return e / z, (mx + np.log(z))[:, 0]
+
+
+def head_forward(qt, kt, v, causal, rows=None, block=512):
+    """O and lse of the given query rows (default all) for rotated q~, k~ of one head."""
+    n, d = qt.shape
+    scale = 1.0 / np.sqrt(d)
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    o = np.empty((len(rows), v.shape[1]))
+    lse = np.empty(len(rows))
+    for a in range(0, len(rows), block):
+        r = rows[a:a + block]
+        p, l = _softmax_rows(_scores(qt[r], kt, r, causal, scale))
+        o[a:a + block] = p @ v
+        lse[a:a + block] = l
+    return o, lse
+
+
+def head_backward(qt, kt, v, do, causal, block=512):
+    """dQ~, dK~, dV of one head from the upstream gradient dO (= l(x))."""
+    n, d = qt.shape
+    scale = 1.0 / np.sqrt(d)
+    dqt = np.empty_like(qt)
+    dkt = np.zeros_like(kt)
+    dv = np.zeros_like(v)
+    for a in range(0, n, block):
+        r = np.arange(a, min(n, a + block))
+        p, _ = _softmax_rows(_scores(qt[r], kt, r, causal, scale))   # s(x)
+        beta = do[r] @ v.T                                           # beta(x)
+        gamma1 = p * beta                                            # diag(s) beta
+        gamma2 = p * np.sum(p * beta, axis=1, keepdims=True)         # s s^T beta
+        ds = gamma1 - gamma2                                         # gamma(x)
+        dv += p.T @ do[r]
+        dqt[r] = (ds @ kt) * scale
+        dkt += (ds.T @ qt[r]) * scale
+    return dqt, dkt, dv
+
+
+def head_matrices(qt, kt, v, do, causal):
+    """Full n x n P and dS of one head (small n only): for pins and the DTFT form."""
+    n, d = qt.shape
+    r = np.arange(n)
+    p, _ = _softmax_rows(_scores(qt, kt, r, causal, 1.0 / np.sqrt(d)))
+    beta = do @ v.T
+    ds = p * beta - p * np.sum(p * beta, axis=1, keepdims=True)
+    return p, ds
+
+
+# --------------------------------------------------------------------------
+# public API over [B, H, n, d]
+# --------------------------------------------------------------------------
+def forward(q, k, v, alpha, base, causal, pairing="interleaved", offset=0, block=512):
+    """O [B,H,n,d] and lse [B,H,n] (natural log) in float64."""
+    B, H, n, d = q.shape
+    _, th = frequencies(d, base, alpha)
+    phi = angles(n, th, offset)
+    o = np.empty((B, H, n, d))
+    lse = np.empty((B, H, n))
+    for b in range(B):
+        for h in range(H):
+            qt = rotate(q[b, h], phi, pairing)
+            kt = rotate(k[b, h], phi, pairing)
+            o[b, h], lse[b, h] = head_forward(qt, kt, v[b, h], causal, block=block)
+    return o, lse
+
+
+def loss(o, e):
+    """L = 1/2 ||O - E||_F^2 summed over every element, and dO = O - E."""
+    do = np.asarray(o, dtype=np.float64) - np.asarray(e, dtype=np.float64)
+    return 0.5 * float(np.sum(do * do)), do
+
+
+def band_torque(g, x, pairing="interleaved"):
+    """<g_pm, J x_pm> for every row p and band m: g1*x0 - g0*x1."""
+    i0, i1 = band_index(x.shape[-1], pairing)
+    return g[..., i1] * x[..., i0] - g[..., i0] * x[..., i1]
+
+
+def backward(q, k, v, do, alpha, base, causal, pairing="interleaved", offset=0, block=512,
+             return_rotated=False):
+    """dQ, dK, dV [B,H,n,d] and dalpha [d/2] in float64 for upstream gradient dO."""
+    B, H, n, d = q.shape
+    _, th = frequencies(d, base, alpha)
+    phi = angles(n, th, offset)
+    pos = np.arange(n, dtype=np.float64) + offset
+    dq = np.empty((B, H, n, d))
+    dk = np.empty((B, H, n, d))
+    dv = np.empty((B, H, n, d))
+    acc = np.zeros(d // 2)
+    extra = []
+    for b in range(B):
+        for h in range(H):
+            qt = rotate(q[b, h], phi, pairing)
+            kt = rotate(k[b, h], phi, pairing)
+            dqt, dkt, dv[b, h] = head_backward(qt, kt, v[b, h], do[b, h], causal, block)
+            dq[b, h] = rotate(dqt, phi, pairing, sign=-1.0)
+            dk[b, h] = rotate(dkt, phi, pairing, sign=-1.0)
+            tq = band_torque(dqt, qt, pairing)
+            tk = band_torque(dkt, kt, pairing)
+            acc += pos @ (tq + tk)
+            if return_rotated:
+                extra.append((qt, kt, dqt, dkt))
+    dalpha = th * acc
+    if return_rotated:
+        return dq, dk, dv, dalpha, extra
+    return dq, dk, dv, dalpha
+
+
+def forward_backward(q, k, v, e, alpha, base, causal, **kw):
+    """The whole path: O, lse, L, dO, dQ, dK, dV, dalpha."""
+    o, lse = forward(q, k, v, alpha, base, causal, **kw)
+    L, do = loss(o, e)
+    dq, dk, dv, dalpha = backward(q, k, v, do, alpha, base, causal, **kw)
+    return dict(o=o, lse=lse, L=L, do=do, dq=dq, dk=dk, dv=dv, dalpha=dalpha)
+
+
+# --------------------------------------------------------------------------
+# second formula for dalpha: derivative of the DTFT surrogate
+# --------------------------------------------------------------------------
+def dalpha_offset_dtft(q, k, v, do, alpha, base, causal, pairing="interleaved"):
+    """dalpha via the offset-aggregated gradient signal ("LeRoPE", Analise Teorica).
+
+    Band m of a row is read as the complex number z = x0 + i x1, so that a
+    rotation by psi is multiplication by exp(i psi) and the band's share of the
+    score is S_ij^(m) = Re(exp(i (i-j) theta_hat_m) z_q,i conj(z_k,j)) / sqrt(d),
+    built from the UNROTATED q, k.  With g_m(D) = sum_{i-j=D} dS_ij z_q,i
+    conj(z_k,j) / sqrt(d) (the gradient signal aggregated by offset D), the
+    surrogate P_m(theta) = Re sum_D g_m(D) exp(i D theta) is the real part of
+    the DTFT of g_m, and dL/dtheta_hat_m = P_m'(theta_hat_m); dalpha_m =
+    theta_hat_m dL/dtheta_hat_m.  Small n only (builds n x n matrices).
+    """
+    B, H, n, d = q.shape
+    _, th = frequencies(d, base, alpha)
+    phi = angles(n, th)
+    i0, i1 = band_index(d, pairing)
+    D = np.arange(n)[:, None] - np.arange(n)[None, :]
+    out = np.zeros(d // 2)
+    for b in range(B):
+        for h in range(H):
+            qt = rotate(q[b, h], phi, pairing)
+            kt = rotate(k[b, h], phi, pairing)
+            _, ds = head_matrices(qt, kt, v[b, h], do[b, h], causal)
+            zq = q[b, h][:, i0] + 1j * q[b, h][:, i1]
+            zk = k[b, h][:, i0] + 1j * k[b, h][:, i1]
+            for m in range(d // 2):
+                w = ds * np.outer(zq[:, m], np.conj(zk[:, m])) / np.sqrt(d)
+                g = np.zeros(2 * n - 1, dtype=complex)       # offsets -(n-1)..n-1
+                np.add.at(g, (D + n - 1).ravel(), w.ravel())
+                offs = np.arange(-(n - 1), n)
+                dP = np.real(np.sum(1j * offs * g * np.exp(1j * offs * th[m])))
+                out[m] += th[m] * dP
+    return out

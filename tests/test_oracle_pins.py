@@ -1,0 +1,275 @@
+"""Pins for the float64 oracle, against things other than the oracle itself.
+
+Each test names the invariant it checks (I1..I11) and the statement it rests
+on.  Between them they fail on a dropped term, a wrong sign, a wrong index or
+a transposed operand anywhere in the oracle.  CPU only.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rope_attn_naive as naive
+from oracle import rope_attn_ref as ref
+
+
+def rand_problem(seed, B, H, n, d, alpha_scale=0.4, base=10000.0, qscale=1.0):
+    rng = np.random.default_rng(seed)
+    q = qscale * rng.standard_normal((B, H, n, d))
+    k = qscale * rng.standard_normal((B, H, n, d))
+    v = rng.standard_normal((B, H, n, d))
+    e = rng.standard_normal((B, H, n, d))
+    alpha = alpha_scale * rng.standard_normal(d // 2)
+    return q, k, v, e, alpha, base
+
+
+def total_loss(q, k, v, e, alpha, base, causal, **kw):
+    o, _ = ref.forward(q, k, v, alpha, base, causal, **kw)
+    return ref.loss(o, e)[0]
+
+
+# ---------------------------------------------------------------- naive vs blocked
+@pytest.mark.parametrize("causal", [False, True])
+def test_naive_matches_blocked(causal):
+    q, k, v, e, alpha, base = rand_problem(1, 1, 2, 11, 8, base=100.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal, block=4)
+    acc = np.zeros(4)
+    Ltot = 0.0
+    for h in range(2):
+        nv = naive.head(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), e[0, h].tolist(),
+                        alpha.tolist(), base, causal)
+        for key in ("o", "dq", "dk", "dv"):
+            np.testing.assert_allclose(np.array(nv[key]), r[key][0, h], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(np.array(nv["lse"]), r["lse"][0, h], rtol=0, atol=1e-12)
+        acc += np.array(nv["dalpha"])
+        Ltot += nv["L"]
+    np.testing.assert_allclose(acc, r["dalpha"], rtol=1e-12, atol=1e-12)
+    assert abs(Ltot - r["L"]) < 1e-12 * max(1.0, abs(Ltot))
+
+
+# ---------------------------------------------------------------- I4 finite differences
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [4, 8])
+def test_I4_finite_differences(causal, d):
+    """Central differences of L (fp64, h = 1e-6) on every entry of Q, K, V and alpha."""
+    n = 6 if d == 8 else 7
+    q, k, v, e, alpha, base = rand_problem(7 + d, 1, 2, n, d, alpha_scale=0.5, base=20.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal)
+    h = 1e-6
+    for name, arr, grad in (("q", q, r["dq"]), ("k", k, r["dk"]), ("v", v, r["dv"])):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            lp = total_loss(q, k, v, e, alpha, base, causal)
+            arr[idx] = old - h
+            lm = total_loss(q, k, v, e, alpha, base, causal)
+            arr[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - grad)) / np.max(np.abs(grad))
+        assert err < 1e-7, (name, err)
+    fd = np.zeros_like(alpha)
+    for m in range(len(alpha)):
+        old = alpha[m]
+        alpha[m] = old + h
+        lp = total_loss(q, k, v, e, alpha, base, causal)
+        alpha[m] = old - h
+        lm = total_loss(q, k, v, e, alpha, base, causal)
+        alpha[m] = old
+        fd[m] = (lp - lm) / (2 * h)
+    err = np.max(np.abs(fd - r["dalpha"])) / np.max(np.abs(r["dalpha"]))
+    assert err < 1e-7, ("alpha", err)
+
+
+# ---------------------------------------------------------------- I4b autograd route
+def _torch_rope_complex(x, pos, theta_hat):
+    """Textbook complex-number RoPE: pair (2m, 2m+1) -> z, z * exp(i p theta)."""
+    z = torch.view_as_complex(x.reshape(*x.shape[:-1], -1, 2).contiguous())
+    rot = torch.polar(torch.ones_like(pos[:, None] * theta_hat[None, :]),
+                      pos[:, None] * theta_hat[None, :])
+    return torch.view_as_real(z * rot).reshape(x.shape)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_I4b_autograd_of_independent_forward(causal):
+    """A forward written with complex multiplication and torch's own softmax, differentiated
+    by autograd, gives the same dQ, dK, dV, dalpha as the oracle's hand-written backward."""
+    B, H, n, d = 2, 3, 33, 16
+    q, k, v, e, alpha, base = rand_problem(3, B, H, n, d, alpha_scale=0.7, base=500.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal, block=8)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    ta = torch.tensor(alpha, requires_grad=True)
+    m = torch.arange(d // 2, dtype=torch.float64)
+    th = torch.exp(ta) * base ** (-2.0 * m / d)
+    pos = torch.arange(n, dtype=torch.float64)
+    qr, kr = _torch_rope_complex(tq, pos, th), _torch_rope_complex(tk, pos, th)
+    s = qr @ kr.transpose(-1, -2) / math.sqrt(d)
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ tv
+    L = 0.5 * ((o - torch.tensor(e)) ** 2).sum()
+    L.backward()
+    np.testing.assert_allclose(o.detach().numpy(), r["o"], atol=1e-12)
+    assert abs(L.item() - r["L"]) < 1e-10 * abs(r["L"])
+    for g, key in ((tq.grad, "dq"), (tk.grad, "dk"), (tv.grad, "dv")):
+        np.testing.assert_allclose(g.numpy(), r[key], atol=1e-11)
+    np.testing.assert_allclose(ta.grad.numpy(), r["dalpha"], rtol=1e-10, atol=1e-11)
+
+
+# ---------------------------------------------------------------- I1 alpha = 0 is standard RoPE
+def test_I1_alpha_zero_is_textbook_rope():
+    """alpha = 0 reduces LeRoPE to standard RoPE ("LeRoPE", Escolhas de Design Principais:
+    initialisation at 0).  Textbook rotate_half RoPE over the half-split layout."""
+    n, d, base = 40, 16, 10000.0
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((n, d))
+    inv = 1.0 / (base ** (np.arange(0, d, 2) / d))
+    freqs = np.outer(np.arange(n), inv)
+    emb = np.concatenate([freqs, freqs], axis=1)
+    rot_half = np.concatenate([-x[:, d // 2:], x[:, :d // 2]], axis=1)
+    textbook = x * np.cos(emb) + rot_half * np.sin(emb)
+    _, th = ref.frequencies(d, base, np.zeros(d // 2))
+    ours = ref.rotate(x, ref.angles(n, th), pairing="halfsplit")
+    np.testing.assert_allclose(ours, textbook, atol=1e-13)
+
+
+def test_pairing_is_a_permutation():
+    """Interleaved and half-split pairings differ by a fixed column permutation: O, L and
+    dalpha agree; dQ, dK are the same numbers permuted."""
+    B, H, n, d = 1, 2, 13, 8
+    q, k, v, e, alpha, base = rand_problem(9, B, H, n, d)
+    perm = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])  # interleaved -> halfsplit
+    a = ref.forward_backward(q, k, v, e, alpha, base, True)
+    b = ref.forward_backward(q[..., perm], k[..., perm], v, e, alpha, base, True, pairing="halfsplit")
+    np.testing.assert_allclose(a["o"], b["o"], atol=1e-13)
+    np.testing.assert_allclose(a["dalpha"], b["dalpha"], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(a["dq"][..., perm], b["dq"], atol=1e-13)
+    np.testing.assert_allclose(a["dk"][..., perm], b["dk"], atol=1e-13)
+
+
+# ---------------------------------------------------------------- I2 relative position
+def test_I2_scores_depend_on_offset_only():
+    n, d = 25, 8
+    q, k, v, e, alpha, base = rand_problem(11, 1, 1, n, d, base=50.0)
+    _, th = ref.frequencies(d, base, alpha)
+    S = {}
+    for shift in (0, 1000):
+        phi = ref.angles(n, th, offset=shift)
+        S[shift] = ref.rotate(q[0, 0], phi) @ ref.rotate(k[0, 0], phi).T
+    np.testing.assert_allclose(S[1000], S[0], atol=1e-11)
+    o0, _ = ref.forward(q, k, v, alpha, base, True)
+    o1, _ = ref.forward(q, k, v, alpha, base, True, offset=1000)
+    np.testing.assert_allclose(o1, o0, atol=1e-11)
+
+
+# ---------------------------------------------------------------- I3 norms
+def test_I3_rotation_preserves_band_norms():
+    n, d = 30, 12
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((n, d))
+    _, th = ref.frequencies(d, 10000.0, rng.standard_normal(d // 2))
+    y = ref.rotate(x, ref.angles(n, th))
+    nb = lambda z: z[:, 0::2] ** 2 + z[:, 1::2] ** 2
+    np.testing.assert_allclose(nb(y), nb(x), rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(ref.rotate(y, ref.angles(n, th), sign=-1.0), x, atol=1e-14)
+
+
+# ---------------------------------------------------------------- I5 DTFT surrogate
+@pytest.mark.parametrize("causal", [False, True])
+def test_I5_dalpha_equals_dtft_surrogate_derivative(causal):
+    q, k, v, e, alpha, base = rand_problem(13, 2, 2, 17, 8, alpha_scale=0.8, base=30.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal)
+    alt = ref.dalpha_offset_dtft(q, k, v, r["do"], alpha, base, causal)
+    np.testing.assert_allclose(alt, r["dalpha"], rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- I6 global rotation
+@pytest.mark.parametrize("causal", [False, True])
+def test_I6_global_rotation_invariance(causal):
+    q, k, v, e, alpha, base = rand_problem(17, 1, 3, 21, 8, base=40.0)
+    o, _ = ref.forward(q, k, v, alpha, base, causal)
+    _, do = ref.loss(o, e)
+    *_, extra = ref.backward(q, k, v, do, alpha, base, causal, return_rotated=True)
+    for qt, kt, dqt, dkt in extra:
+        tot = ref.band_torque(dqt, qt).sum(0) + ref.band_torque(dkt, kt).sum(0)
+        scale = np.abs(ref.band_torque(dqt, qt)).sum(0)
+        assert np.all(np.abs(tot) < 1e-12 * np.maximum(scale, 1.0))
+
+
+# ---------------------------------------------------------------- I7 zero frequency
+def test_I7_zero_frequency_is_plain_attention():
+    B, H, n, d = 1, 2, 19, 8
+    q, k, v, e, _, base = rand_problem(19, B, H, n, d)
+    alpha = np.full(d // 2, -80.0)   # exp(-80) ~ 1.8e-35: no band rotates
+    o, _ = ref.forward(q, k, v, alpha, base, True)
+    sd = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v), is_causal=True).numpy()
+    np.testing.assert_allclose(o, sd, atol=1e-13)
+    # dalpha_m is linear in theta_hat_m as theta_hat_m -> 0: lowering alpha by 1 divides by e
+    _, do = ref.loss(o, e)
+    d1 = ref.backward(q, k, v, do, np.full(d // 2, -30.0), base, True)[3]
+    d2 = ref.backward(q, k, v, do, np.full(d // 2, -31.0), base, True)[3]
+    np.testing.assert_allclose(d1 / d2, np.e, rtol=1e-9)
+
+
+# ---------------------------------------------------------------- I8, I9 causal row 0, softmax rows
+def test_I8_I9_rows():
+    q, k, v, e, alpha, base = rand_problem(23, 1, 1, 15, 8)
+    o, _ = ref.forward(q, k, v, alpha, base, True)
+    assert np.array_equal(o[0, 0, 0], v[0, 0, 0])
+    _, th = ref.frequencies(8, base, alpha)
+    phi = ref.angles(15, th)
+    qt, kt = ref.rotate(q[0, 0], phi), ref.rotate(k[0, 0], phi)
+    p, ds = ref.head_matrices(qt, kt, v[0, 0], o[0, 0] - e[0, 0], True)
+    assert np.all(ds[0] == 0.0)
+    np.testing.assert_allclose(p.sum(1), 1.0, atol=1e-15)
+    np.testing.assert_allclose(ds.sum(1), 0.0, atol=1e-14)
+    assert np.all(np.triu(p, 1) == 0.0)
+
+
+# ---------------------------------------------------------------- I10 Q = 0
+@pytest.mark.parametrize("causal", [False, True])
+def test_I10_zero_queries(causal):
+    B, H, n, d = 1, 2, 12, 8
+    _, k, v, e, alpha, base = rand_problem(29, B, H, n, d)
+    q = np.zeros((B, H, n, d))
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal)
+    for h in range(H):
+        for i in range(n):
+            hi = i + 1 if causal else n
+            np.testing.assert_allclose(r["o"][0, h, i], v[0, h, :hi].mean(0), atol=1e-14)
+    assert np.max(np.abs(r["dk"])) < 1e-15
+    assert np.max(np.abs(r["dalpha"])) < 1e-14
+
+
+# ---------------------------------------------------------------- I11 d = 2 closed form
+def test_I11_single_band_closed_form():
+    """One band: S_ij = |q_i| |k_j| cos(arg q_i - arg k_j + (i - j) theta_hat) / sqrt(2)."""
+    n, theta_hat, alpha, base = 3, None, np.array([0.3]), 7.0
+    rng = np.random.default_rng(31)
+    q = rng.standard_normal((1, 1, n, 2))
+    k = rng.standard_normal((1, 1, n, 2))
+    v = rng.standard_normal((1, 1, n, 2))
+    theta_hat = math.exp(0.3) * 1.0   # m = 0: base^0 = 1
+    S = np.zeros((n, n))
+    for i in range(n):
+        for j in range(n):
+            a = math.atan2(q[0, 0, i, 1], q[0, 0, i, 0])
+            b = math.atan2(k[0, 0, j, 1], k[0, 0, j, 0])
+            S[i, j] = (np.hypot(*q[0, 0, i]) * np.hypot(*k[0, 0, j])
+                       * math.cos(a - b + (i - j) * theta_hat) / math.sqrt(2))
+    P = np.exp(S) / np.exp(S).sum(1, keepdims=True)
+    o, lse = ref.forward(q, k, v, alpha, base, False)
+    np.testing.assert_allclose(o[0, 0], P @ v[0, 0], atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], np.log(np.exp(S).sum(1)), atol=1e-14)
+
+
+# ---------------------------------------------------------------- loss special case
+def test_loss_zero_when_target_is_output():
+    q, k, v, _, alpha, base = rand_problem(37, 1, 2, 9, 8)
+    o, _ = ref.forward(q, k, v, alpha, base, False)
+    r = ref.forward_backward(q, k, v, o.copy(), alpha, base, False)
+    assert r["L"] == 0.0
+    for key in ("dq", "dk", "dv", "dalpha"):
+        assert np.max(np.abs(r[key])) == 0.0

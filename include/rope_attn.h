@@ -1,0 +1,124 @@
+/*
+ * rope_attn.h -- C ABI of librope_attn.so: exact RoPE / LeRoPE softmax attention,
+ * forward, loss and backward, on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per batch b, head h; positions p = 0..n-1; M = d/2 bands):
+ *
+ *   theta_m     = base^(-2m/d),  theta_hat_m = exp(alpha_m) * theta_m
+ *       "LeRoPE: learnable RoPE frequencies", Mecanismo Central (effective
+ *       frequency = learned exponential rescaling of the standard RoPE
+ *       frequency) and Declaracao do Problema (geometric sequence in base b).
+ *   q~_p, k~_p  = band m of q_p, k_p (coordinates 2m, 2m+1) rotated by p*theta_hat_m
+ *       same page, Declaracao do Problema (rotation in 2-D frequency bands).
+ *   O = softmax(Q~ K~^T / sqrt(d)) V, lse = log-sum-exp of each score row
+ *       "RoPE attention can be trained in almost-linear time", Metodologia 1
+ *       (normalised softmax s(x)).
+ *   L = 1/2 ||O - E||_F^2, dO = O - E
+ *       same page, Metodologia 1 (error term l(x): output minus target).
+ *   dV = P^T dO; dP = dO V^T (beta); dS = P o (dP - rowsum(dO o O)) (gamma =
+ *   diag(s) beta - s s^T beta); dQ = R(-p theta_hat) dS K~ / sqrt(d);
+ *   dK = R(-p theta_hat) dS^T Q~ / sqrt(d)
+ *       same page, Metodologia 1-2 (beta, gamma_1, gamma_2).
+ *   dalpha_m = theta_hat_m * sum_{b,h,p} p * (<dQ~_pm, J q~_pm> + <dK~_pm, J k~_pm>)
+ *       "LeRoPE", Escolhas de Design Principais (log-space parameters shared by
+ *       every head) and Analise Teorica (frequency gradient).
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  Q, K, V, O,
+ *     E, dO, dQ, dK, dV are dense row-major [B, H, n, d] in the problem dtype
+ *     (fp32 or bf16); lse is fp32 [B, H, n]; alpha and dalpha are fp32 [d/2];
+ *     L is one fp32 in device memory.  Pointers must be 16-byte aligned.
+ *   - ws / ws_bytes: caller-owned device workspace of at least
+ *     rope_attn_workspace_bytes(p) bytes, 256-byte aligned.  The library
+ *     allocates no device memory of its own and keeps nothing between calls
+ *     in it; two calls that run concurrently need two workspaces.
+ *   - stream: a cudaStream_t (0 = legacy default stream).  All calls are
+ *     asynchronous on that stream; outputs are valid once it has synchronised.
+ *   - Arguments are validated before anything is launched; a rejected call
+ *     launches nothing and returns RA_ERR_INVALID_ARG / RA_ERR_UNSUPPORTED /
+ *     RA_ERR_WORKSPACE.  A failed launch returns RA_ERR_CUDA.  Device-side
+ *     waits are bounded: a wait that expires makes the kernel record
+ *     RA_ERR_TIMEOUT in the workspace error word and return; read it with
+ *     rope_attn_device_status().  No entry point aborts or traps.
+ *   - Supported: fp32 with even d, 2 <= d <= 128 (CUDA-core path); bf16 with
+ *     d in {64, 128} (tcgen05 tensor-core path); n >= 1; B, H >= 1.
+ */
+#ifndef ROPE_ATTN_H
+#define ROPE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RA_OK = 0,
+    RA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape or flag        */
+    RA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement       */
+    RA_ERR_WORKSPACE = 3,     /* ws null, misaligned or smaller than required      */
+    RA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed       */
+    RA_ERR_TIMEOUT = 5        /* a device-side wait expired (see device_status)    */
+} ra_status;
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
+
+/* Problem description, passed by pointer to every call. */
+typedef struct {
+    int64_t B, H, n, d;  /* batch, heads, sequence length, head dimension      */
+    int32_t dtype;       /* ra_dtype of Q, K, V, O, E, dO, dQ, dK, dV          */
+    int32_t causal;      /* 1: key j is visible to query i only when j <= i     */
+    double base;         /* RoPE base b > 0 (theta_m = b^(-2m/d))               */
+} ra_problem;
+
+/* Bytes of workspace the calls below need for problem *p (0 if *p is invalid).
+ * Holds: the fp32 cos/sin table [n, d/2, 2], the rotated Q~ and K~ in the
+ * problem dtype, rowsum(dO o O) [B, H, n] fp32, per-tile dalpha partials,
+ * loss partials and the device error word. */
+size_t rope_attn_workspace_bytes(const ra_problem* p);
+
+/* Forward: o = softmax(Q~ K~^T / sqrt(d)) V and lse (natural log) from q, k, v
+ * and alpha.  Overwrites the table, Q~ and K~ regions of ws. */
+ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const void* v,
+                        const float* alpha, void* o, float* lse,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Loss: *L = 1/2 sum (o - e)^2 over all B*H*n*d elements (fixed-order, deterministic
+ * fp64 reduction, stored as fp32) and dO = o - e rounded to the dtype. */
+ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e,
+                         float* L, void* dO, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward: dq, dk, dv ([B,H,n,d], dtype) and dalpha ([d/2], fp32, summed over
+ * every batch and head) from q, k, v, the forward's o and lse, the upstream
+ * gradient dO and alpha.  Deterministic: no atomics, fixed-order reductions.
+ * Recomputes the table, Q~ and K~ in ws (it does not rely on a previous fwd). */
+ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* dO, const float* alpha,
+                        void* dq, void* dk, void* dv, float* dalpha,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads and clears the device error word in ws.
+ * Returns RA_OK, or RA_ERR_TIMEOUT if a kernel gave up on a wait since the last
+ * call (kernel id / barrier id / block id are written to info[0..2] when info
+ * is non-null). */
+ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32_t info[3]);
+
+/* Static text for a status code. */
+const char* rope_attn_status_string(ra_status s);
+
+/* ---- optional per-kernel timing (instrumentation, off by default) --------
+ * While enabled, every kernel launch made by the calls above is bracketed by
+ * CUDA events on the caller's stream.  rope_attn_timing_read synchronises
+ * those events and writes, per kernel id, the number of launches and the sum
+ * of their durations in milliseconds; it returns the number of kernel ids
+ * (at most max_ids) and clears the record. */
+void rope_attn_timing_enable(int on);
+int rope_attn_timing_read(int32_t* launches, double* total_ms, int max_ids);
+const char* rope_attn_kernel_name(int id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROPE_ATTN_H */

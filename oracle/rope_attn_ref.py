@@ -146,6 +146,32 @@ def head_backward(qt, kt, v, do, causal, block=512):
     return dqt, dkt, dv
 
 
+def head_backward_rows(qt, kt, v, do_rows, lse_rows, delta_rows, rows, causal):
+    """dQ~ of the given query rows only (row i needs its own lse_i and Delta_i)."""
+    n, d = qt.shape
+    scale = 1.0 / np.sqrt(d)
+    rows = np.asarray(rows)
+    s = _scores(qt[rows], kt, rows, causal, scale)
+    p = np.exp(s - lse_rows[:, None])                                # s(x), rows
+    beta = do_rows @ v.T
+    ds = p * beta - p * delta_rows[:, None]                          # gamma(x), rows
+    return (ds @ kt) * scale
+
+
+def head_backward_cols(qt, kt, v, do, lse, delta, cols, causal):
+    """dK~ and dV of the given key rows only; needs every query's lse and Delta."""
+    n, d = qt.shape
+    scale = 1.0 / np.sqrt(d)
+    cols = np.asarray(cols)
+    s = (qt @ kt[cols].T) * scale                                    # n x |cols|
+    if causal:
+        s = np.where(cols[None, :] > np.arange(n)[:, None], -np.inf, s)
+    p = np.exp(s - lse[:, None])
+    beta = do @ v[cols].T
+    ds = p * beta - p * delta[:, None]
+    return (ds.T @ qt) * scale, p.T @ do
+
+
 def head_matrices(qt, kt, v, do, causal):
     """Full n x n P and dS of one head (small n only): for pins and the DTFT form."""
     n, d = qt.shape

@@ -1,0 +1,167 @@
+"""ctypes binding of librope_attn.so (see include/rope_attn.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch provides device memory (outputs and workspace) and the
+current CUDA stream.  There is no fallback: if the library is missing or a
+call fails, a RuntimeError is raised.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librope_attn.so")
+
+RA_F32, RA_BF16 = 0, 1
+_DTYPE = {torch.float32: RA_F32, torch.bfloat16: RA_BF16}
+STATUS = {0: "RA_OK", 1: "RA_ERR_INVALID_ARG", 2: "RA_ERR_UNSUPPORTED", 3: "RA_ERR_WORKSPACE",
+          4: "RA_ERR_CUDA", 5: "RA_ERR_TIMEOUT"}
+
+
+class RaProblem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("n", ctypes.c_int64),
+                ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("base", ctypes.c_double)]
+
+
+class RopeAttnError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}: "
+                         f"{lib().rope_attn_status_string(code).decode()}")
+
+
+_lib = None
+
+
+def lib():
+    """Load librope_attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run python -m rope_attention_fwd_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, vp, sz = ctypes.POINTER(RaProblem), ctypes.c_void_p, ctypes.c_size_t
+        L.rope_attn_workspace_bytes.argtypes = [P]
+        L.rope_attn_workspace_bytes.restype = sz
+        L.rope_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.rope_attn_fwd.restype = ctypes.c_int
+        L.rope_attn_loss.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.rope_attn_loss.restype = ctypes.c_int
+        L.rope_attn_bwd.argtypes = [P] + [vp] * 12 + [sz, vp]
+        L.rope_attn_bwd.restype = ctypes.c_int
+        L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
+        L.rope_attn_device_status.restype = ctypes.c_int
+        L.rope_attn_status_string.argtypes = [ctypes.c_int]
+        L.rope_attn_status_string.restype = ctypes.c_char_p
+        L.rope_attn_timing_enable.argtypes = [ctypes.c_int]
+        L.rope_attn_timing_enable.restype = None
+        L.rope_attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_int32),
+                                            ctypes.POINTER(ctypes.c_double), ctypes.c_int]
+        L.rope_attn_timing_read.restype = ctypes.c_int
+        L.rope_attn_kernel_name.argtypes = [ctypes.c_int]
+        L.rope_attn_kernel_name.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def problem(B, H, n, d, dtype, causal, base):
+    if isinstance(dtype, torch.dtype):
+        dtype = _DTYPE[dtype]
+    return RaProblem(int(B), int(H), int(n), int(d), int(dtype), int(bool(causal)), float(base))
+
+
+def _problem_of(q, causal, base):
+    B, H, n, d = q.shape
+    return problem(B, H, n, d, q.dtype, causal, base)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise RopeAttnError(fn, code)
+
+
+def rope_attn_workspace_bytes(prob):
+    return int(lib().rope_attn_workspace_bytes(ctypes.byref(prob)))
+
+
+def workspace(prob, device):
+    """A fresh device workspace for `prob` (uint8 tensor)."""
+    nbytes = rope_attn_workspace_bytes(prob)
+    if nbytes == 0:
+        raise RopeAttnError("rope_attn_workspace_bytes", 1)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None):
+    """(o, lse) = softmax(Q~ K~^T / sqrt(d)) V and its row log-sum-exp."""
+    prob = _problem_of(q, causal, base)
+    B, H, n, d = q.shape
+    if ws is None:
+        ws = workspace(prob, q.device)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check("rope_attn_fwd", lib().rope_attn_fwd(
+        ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse
+
+
+def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
+    """(L, dO): L = 1/2 ||o - e||^2 (fp32 scalar tensor on device), dO = o - e."""
+    prob = _problem_of(o, causal, base)
+    if ws is None:
+        ws = workspace(prob, o.device)
+    L = torch.empty((), dtype=torch.float32, device=o.device) if L is None else L
+    dO = torch.empty_like(o) if dO is None else dO
+    _check("rope_attn_loss", lib().rope_attn_loss(
+        ctypes.byref(prob), _ptr(o), _ptr(e), _ptr(L), _ptr(dO), _ptr(ws), ws.numel(),
+        _stream(o.device)))
+    return L, dO
+
+
+def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk=None, dv=None,
+                  dalpha=None):
+    """(dq, dk, dv, dalpha) of L for upstream gradient dO."""
+    prob = _problem_of(q, causal, base)
+    if ws is None:
+        ws = workspace(prob, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dalpha = torch.empty_like(alpha) if dalpha is None else dalpha
+    _check("rope_attn_bwd", lib().rope_attn_bwd(
+        ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+        _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(),
+        _stream(q.device)))
+    return dq, dk, dv, dalpha
+
+
+def rope_attn_device_status(ws):
+    """Synchronise the current stream and return (status code, [kernel, site, block])."""
+    info = (ctypes.c_int32 * 3)()
+    code = lib().rope_attn_device_status(_ptr(ws), ws.numel(), _stream(ws.device), info)
+    return code, list(info)
+
+
+def rope_attn_timing_enable(on=True):
+    lib().rope_attn_timing_enable(1 if on else 0)
+
+
+def rope_attn_timing_read():
+    """{kernel name: (launches, total ms)} since the last read."""
+    n = 32
+    launches = (ctypes.c_int32 * n)()
+    total = (ctypes.c_double * n)()
+    k = lib().rope_attn_timing_read(launches, total, n)
+    return {lib().rope_attn_kernel_name(i).decode(): (launches[i], total[i])
+            for i in range(k) if launches[i] > 0}

@@ -1,0 +1,326 @@
+// api.cu -- host implementation of the C ABI declared in include/rope_attn.h:
+// argument validation, workspace carving, TMA tensor-map encoding, the launch
+// sequence of each call and the optional per-kernel event timing.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.h"
+#include "launch.h"
+
+using namespace ra;
+
+namespace {
+
+// ------------------------------------------------------------------ timing
+struct TimedLaunch {
+  int kid;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+bool g_timing = false;
+std::vector<TimedLaunch> g_timed;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct LaunchScope {
+  int kid;
+  cudaStream_t s;
+  cudaEvent_t start = nullptr;
+  LaunchScope(int k, cudaStream_t st) : kid(k), s(st) {
+    if (g_timing) {
+      std::lock_guard<std::mutex> g(g_timing_mu);
+      start = take_event();
+      cudaEventRecord(start, s);
+    }
+  }
+  void done() {
+    if (start) {
+      std::lock_guard<std::mutex> g(g_timing_mu);
+      cudaEvent_t stop = take_event();
+      cudaEventRecord(stop, s);
+      g_timed.push_back({kid, start, stop});
+      start = nullptr;
+    }
+  }
+};
+
+#define RA_LAUNCH(kid, stream, expr)              \
+  do {                                            \
+    LaunchScope _ls((kid), (stream));             \
+    cudaError_t _e = (expr);                      \
+    _ls.done();                                   \
+    if (_e != cudaSuccess) return RA_ERR_CUDA;    \
+  } while (0)
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void* ptr) { return ptr && (reinterpret_cast<uintptr_t>(ptr) % 16) == 0; }
+
+ra_status check_problem(const ra_problem* p) {
+  if (!p) return RA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->n < 1 || p->d < 2 || (p->d % 2) != 0) return RA_ERR_INVALID_ARG;
+  if (p->dtype != RA_F32 && p->dtype != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
+  if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
+  if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
+  if (p->d > 128) return RA_ERR_UNSUPPORTED;
+  if (p->dtype == RA_BF16 && p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) % 256) != 0) return RA_ERR_WORKSPACE;
+  if (ws_bytes < ws_layout(*p).total) return RA_ERR_WORKSPACE;
+  return RA_OK;
+}
+
+// Bound on every device-side wait: RA_WAIT_LIMIT_MS (default 2000 ms), read per call.
+uint64_t wait_limit_ns() {
+  const char* s = std::getenv("RA_WAIT_LIMIT_MS");
+  double ms = s ? std::atof(s) : 2000.0;
+  if (!(ms > 0)) ms = 2000.0;
+  return (uint64_t)(ms * 1e6);
+}
+
+// Test hook for the bounded-wait path: RA_DEBUG_STARVE_BLOCK=<cta> makes that CTA of
+// the bf16 forward skip its Q~ load, so its waits expire and it reports RA_ERR_TIMEOUT.
+int starve_block() {
+  const char* s = std::getenv("RA_DEBUG_STARVE_BLOCK");
+  return s ? std::atoi(s) : -1;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// bf16 [BH][n][d] viewed as (x = d, y = n, z = BH); box = 64 columns x `rows` rows.
+bool make_map(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)p.d, (cuuint64_t)p.n, (cuuint64_t)(p.B * p.H)};
+  const cuuint64_t strides[2] = {(cuuint64_t)p.d * 2, (cuuint64_t)p.n * p.d * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shared prefix of fwd and bwd: clear the error word, build the table, rotate Q and K.
+ra_status prepare(const ra_problem* p, const void* q, const void* k, const float* alpha,
+                  void* ws, const WsLayout& L, cudaStream_t s) {
+  if (cudaMemsetAsync(at<uint8_t>(ws, L.err), 0, 64, s) != cudaSuccess) return RA_ERR_CUDA;
+  RA_LAUNCH(K_TABLE, s, launch_table(*p, alpha, at<float2>(ws, L.table), s));
+  RA_LAUNCH(K_ROTATE, s,
+            launch_rotate(*p, q, k, at<void>(ws, L.qt), at<void>(ws, L.kt),
+                          at<float2>(ws, L.table), s));
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rope_attn_workspace_bytes(const ra_problem* p) {
+  if (check_problem(p) != RA_OK) return 0;
+  return ws_layout(*p).total;
+}
+
+const char* rope_attn_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "ok";
+    case RA_ERR_INVALID_ARG: return "invalid argument";
+    case RA_ERR_UNSUPPORTED: return "unsupported problem";
+    case RA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case RA_ERR_CUDA: return "CUDA error";
+    case RA_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const void* v,
+                        const float* alpha, void* o, float* lse, void* ws, size_t ws_bytes,
+                        void* stream) {
+  ra_status st = check_problem(p);
+  if (st != RA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(o) ||
+      !aligned16(lse))
+    return RA_ERR_INVALID_ARG;
+  if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*p);
+  if ((st = prepare(p, q, k, alpha, ws, L, s)) != RA_OK) return st;
+  if (p->dtype == RA_F32) {
+    RA_LAUNCH(K_FWD_F32, s,
+              launch_fwd_f32(*p, at<float>(ws, L.qt), at<float>(ws, L.kt), (const float*)v,
+                             (float*)o, lse, s));
+    return RA_OK;
+  }
+  Sm100Maps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!make_map(&maps.qt, at<void>(ws, L.qt), *p, 128) ||
+      !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128) || !make_map(&maps.v, v, *p, 128))
+    return RA_ERR_CUDA;
+  DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), starve_block()};
+  RA_LAUNCH(K_FWD_SM100, s, launch_fwd_sm100(*p, maps, o, lse, ctl, s));
+  return RA_OK;
+}
+
+ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e, float* Lout,
+                         void* dO, void* ws, size_t ws_bytes, void* stream) {
+  ra_status st = check_problem(p);
+  if (st != RA_OK) return st;
+  if (!aligned16(o) || !aligned16(e) || !aligned16(dO) || !Lout ||
+      (reinterpret_cast<uintptr_t>(Lout) % 4) != 0)
+    return RA_ERR_INVALID_ARG;
+  if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*p);
+  if (cudaMemsetAsync(at<uint8_t>(ws, L.err), 0, 64, s) != cudaSuccess) return RA_ERR_CUDA;
+  RA_LAUNCH(K_LOSS_PARTIAL, s, launch_loss_partial(*p, o, e, dO, at<double>(ws, L.loss_part), s));
+  RA_LAUNCH(K_LOSS_FINAL, s, launch_loss_final(at<double>(ws, L.loss_part), Lout, s));
+  return RA_OK;
+}
+
+ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* dO, const float* alpha,
+                        void* dq, void* dk, void* dv, float* dalpha, void* ws, size_t ws_bytes,
+                        void* stream) {
+  ra_status st = check_problem(p);
+  if (st != RA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dO) || !aligned16(alpha) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(dalpha))
+    return RA_ERR_INVALID_ARG;
+  if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout L = ws_layout(*p);
+  if ((st = prepare(p, q, k, alpha, ws, L, s)) != RA_OK) return st;
+  float* delta = at<float>(ws, L.delta);
+  float* dpart = at<float>(ws, L.dpart);
+  const float2* table = at<float2>(ws, L.table);
+  RA_LAUNCH(K_BWD_DELTA, s, launch_delta(*p, o, dO, delta, s));
+  if (p->dtype == RA_F32) {
+    const float* qt = at<float>(ws, L.qt);
+    const float* kt = at<float>(ws, L.kt);
+    RA_LAUNCH(K_BWD_DKDV_F32, s,
+              launch_bwd_dkdv_f32(*p, qt, kt, (const float*)v, (const float*)dO, lse, delta,
+                                  table, (float*)dk, (float*)dv, dpart, s));
+    RA_LAUNCH(K_BWD_DQ_F32, s,
+              launch_bwd_dq_f32(*p, qt, kt, (const float*)v, (const float*)dO, lse, delta, table,
+                                (float*)dq, dpart, s));
+  } else {
+    Sm100Maps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!make_map(&maps.qt, at<void>(ws, L.qt), *p, 128) ||
+        !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128) || !make_map(&maps.v, v, *p, 128) ||
+        !make_map(&maps.dO, dO, *p, 128) || !make_map(&maps.kt64, at<void>(ws, L.kt), *p, 64) ||
+        !make_map(&maps.v64, v, *p, 64))
+      return RA_ERR_CUDA;
+    DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
+    RA_LAUNCH(K_BWD_DKDV_SM100, s,
+              launch_bwd_dkdv_sm100(*p, maps, at<void>(ws, L.qt), at<void>(ws, L.kt), lse, delta,
+                                    table, dk, dv, dpart, ctl, s));
+    RA_LAUNCH(K_BWD_DQ_SM100, s,
+              launch_bwd_dq_sm100(*p, maps, at<void>(ws, L.qt), lse, delta, table, dq, dpart,
+                                  ctl, s));
+  }
+  RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
+  return RA_OK;
+}
+
+ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32_t info[3]) {
+  if (!ws || ws_bytes < 64 || (reinterpret_cast<uintptr_t>(ws) % 256) != 0)
+    return RA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word[4] = {0, 0, 0, 0};
+  // The error word is the first region of every workspace layout.
+  if (cudaMemcpyAsync(word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return RA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return RA_ERR_CUDA;
+  if (info) {
+    info[0] = (int32_t)word[1];
+    info[1] = (int32_t)word[2];
+    info[2] = (int32_t)word[3];
+  }
+  return word[0] == 0 ? RA_OK : RA_ERR_TIMEOUT;
+}
+
+void rope_attn_timing_enable(int on) {
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  g_timing = on != 0;
+}
+
+int rope_attn_timing_read(int32_t* launches, double* total_ms, int max_ids) {
+  std::vector<TimedLaunch> rec;
+  {
+    std::lock_guard<std::mutex> g(g_timing_mu);
+    rec.swap(g_timed);
+  }
+  const int nid = max_ids < K_COUNT ? max_ids : (int)K_COUNT;
+  for (int i = 0; i < nid; ++i) {
+    launches[i] = 0;
+    total_ms[i] = 0.0;
+  }
+  for (auto& r : rec) {
+    cudaEventSynchronize(r.stop);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (r.kid < nid) {
+      launches[r.kid] += 1;
+      total_ms[r.kid] += ms;
+    }
+  }
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  for (auto& r : rec) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  return nid;
+}
+
+const char* rope_attn_kernel_name(int id) {
+  static const char* names[K_COUNT] = {
+      "rope_table",       "rotate",       "fwd_f32",      "fwd_sm100",
+      "loss_partial",     "loss_final",   "bwd_delta",    "bwd_dq_f32",
+      "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final"};
+  return (id >= 0 && id < K_COUNT) ? names[id] : "unknown";
+}
+
+}  // extern "C"

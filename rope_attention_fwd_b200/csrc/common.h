@@ -1,0 +1,69 @@
+// common.h -- definitions shared by the host library and the kernels:
+// kernel ids (for timing and error reports), workspace layout, launch shapes.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/rope_attn.h"
+
+namespace ra {
+
+enum KernelId : int {
+  K_TABLE = 0,
+  K_ROTATE = 1,
+  K_FWD_F32 = 2,
+  K_FWD_SM100 = 3,
+  K_LOSS_PARTIAL = 4,
+  K_LOSS_FINAL = 5,
+  K_BWD_DELTA = 6,
+  K_BWD_DQ_F32 = 7,
+  K_BWD_DKDV_F32 = 8,
+  K_BWD_DQ_SM100 = 9,
+  K_BWD_DKDV_SM100 = 10,
+  K_DALPHA = 11,
+  K_COUNT = 12
+};
+
+// Rows per dalpha partial (one partial per band per tile of query or key rows).
+constexpr int kDalphaRows = 64;
+// Blocks of the first loss stage (fixed so the fp64 sum order never changes).
+constexpr int kLossBlocks = 1024;
+constexpr int kLossThreads = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t err;        // uint32 [8]
+  size_t loss_part;  // double [kLossBlocks]
+  size_t table;      // float2 [n][M]  (cos, sin)
+  size_t qt;         // dtype [B*H][n][d]   rotated queries
+  size_t kt;         // dtype [B*H][n][d]   rotated keys
+  size_t delta;      // float [B*H][n]      rowsum(dO o O)
+  size_t dpart;      // float [2][B*H][ceil(n/kDalphaRows)][M]
+  size_t total;
+};
+
+inline WsLayout ws_layout(const ra_problem& p) {
+  const size_t elem = p.dtype == RA_BF16 ? 2 : 4;
+  const size_t BH = (size_t)p.B * (size_t)p.H;
+  const size_t n = (size_t)p.n, d = (size_t)p.d, M = d / 2;
+  const size_t ntile = (n + kDalphaRows - 1) / kDalphaRows;
+  WsLayout w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes, 1024);
+    return at;
+  };
+  w.err = take(64);
+  w.loss_part = take(sizeof(double) * kLossBlocks);
+  w.table = take(sizeof(float) * 2 * n * M);
+  w.qt = take(elem * BH * n * d);
+  w.kt = take(elem * BH * n * d);
+  w.delta = take(sizeof(float) * BH * n);
+  w.dpart = take(sizeof(float) * 2 * BH * ntile * M);
+  w.total = off;
+  return w;
+}
+
+}  // namespace ra

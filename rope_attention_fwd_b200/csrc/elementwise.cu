@@ -1,0 +1,325 @@
+// elementwise.cu -- the HBM- and latency-bound steps of the path:
+//   * rope_table:   theta_hat_m = exp(alpha_m) base^(-2m/d), and the fp32 cos/sin of
+//                   p * theta_hat_m for every position (angle formed and reduced in fp64)
+//                   ("LeRoPE: learnable RoPE frequencies", Mecanismo Central);
+//   * rotate:       q~ = R(p theta_hat) q, k~ = R(p theta_hat) k band by band, written
+//                   once to HBM in the storage dtype and read by every attention tile
+//                   (same page, Declaracao do Problema: 2-D frequency bands);
+//   * loss:         L = 1/2 sum (O - E)^2 in two fixed-order fp64 stages, dO = O - E
+//                   ("RoPE attention can be trained in almost-linear time",
+//                   Metodologia 1: error term l(x));
+//   * delta:        Delta_i = sum_c dO_ic O_ic, the row factor of gamma_2 = s s^T beta
+//                   (same page, Metodologia 2);
+//   * dalpha final: dalpha_m = theta_hat_m * sum of the per-tile partials, fixed order,
+//                   fp64 ("LeRoPE", Escolhas de Design Principais: alpha shared by all
+//                   heads; Analise Teorica: frequency gradient).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.h"
+#include "launch.h"
+
+namespace ra {
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ double theta_hat(const float* alpha, int m, int d, double base) {
+  return exp((double)alpha[m]) * pow(base, -2.0 * (double)m / (double)d);
+}
+
+// ---------------------------------------------------------------- table
+__global__ void rope_table_kernel(const float* __restrict__ alpha, float2* __restrict__ table,
+                                  int n, int M, int d, double base) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)n * M) return;
+  const int p = (int)(idx / M), m = (int)(idx % M);
+  const double phi = (double)p * theta_hat(alpha, m, d, base);
+  double s, c;
+  sincos(phi, &s, &c);
+  table[idx] = make_float2((float)c, (float)s);
+}
+
+// ---------------------------------------------------------------- rotate
+// One thread per band pair of one row of q (blockIdx.y = 0) or k (blockIdx.y = 1).
+template <typename T>
+__global__ void rotate_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                              T* __restrict__ qt, T* __restrict__ kt,
+                              const float2* __restrict__ table, long long rows, int n, int M) {
+  const T* src = blockIdx.y == 0 ? q : k;
+  T* dst = blockIdx.y == 0 ? qt : kt;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // pair index
+  if (idx >= rows * M) return;
+  const long long row = idx / M;
+  const int m = (int)(idx % M);
+  const int p = (int)(row % n);
+  const float2 cs = table[(long long)p * M + m];
+  const float x0 = to_f(src[2 * idx]), x1 = to_f(src[2 * idx + 1]);
+  dst[2 * idx] = from_f<T>(cs.x * x0 - cs.y * x1);
+  dst[2 * idx + 1] = from_f<T>(cs.y * x0 + cs.x * x1);
+}
+
+// bf16 fast path: 4 pairs (16 bytes) per thread.
+__global__ void rotate_bf16x8_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
+                                     uint4* __restrict__ qt, uint4* __restrict__ kt,
+                                     const float2* __restrict__ table, long long rows, int n,
+                                     int M) {
+  const uint4* src = blockIdx.y == 0 ? q : k;
+  uint4* dst = blockIdx.y == 0 ? qt : kt;
+  const int vec_per_row = M / 4;  // d/8 vectors of 8 bf16
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * vec_per_row) return;
+  const long long row = idx / vec_per_row;
+  const int m0 = (int)(idx % vec_per_row) * 4;
+  const int p = (int)(row % n);
+  uint4 in = src[idx];
+  const float4* tab = reinterpret_cast<const float4*>(table + (long long)p * M + m0);
+  const float4 t01 = tab[0], t23 = tab[1];
+  const float c[4] = {t01.x, t01.z, t23.x, t23.z};
+  const float s[4] = {t01.y, t01.w, t23.y, t23.w};
+  uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
+    const float x0 = __low2float(pr), x1 = __high2float(pr);
+    pr = __floats2bfloat162_rn(c[j] * x0 - s[j] * x1, s[j] * x0 + c[j] * x1);
+    w[j] = *reinterpret_cast<uint32_t*>(&pr);
+  }
+  dst[idx] = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ---------------------------------------------------------------- loss
+template <typename T>
+__global__ void __launch_bounds__(kLossThreads)
+    loss_partial_kernel(const T* __restrict__ o, const T* __restrict__ e, T* __restrict__ dO,
+                        double* __restrict__ part, long long count) {
+  double acc = 0.0;
+  const long long stride = (long long)kLossBlocks * kLossThreads;
+  for (long long i = (long long)blockIdx.x * kLossThreads + threadIdx.x; i < count; i += stride) {
+    const float diff = to_f(o[i]) - to_f(e[i]);
+    dO[i] = from_f<T>(diff);
+    acc += (double)diff * (double)diff;
+  }
+  __shared__ double red[kLossThreads];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = kLossThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[blockIdx.x] = red[0];
+}
+
+// bf16 path with 16-byte vectors (count is a multiple of 8 for d in {64, 128}).
+__global__ void __launch_bounds__(kLossThreads)
+    loss_partial_bf16x8_kernel(const uint4* __restrict__ o, const uint4* __restrict__ e,
+                               uint4* __restrict__ dO, double* __restrict__ part,
+                               long long nvec) {
+  double acc = 0.0;
+  const long long stride = (long long)kLossBlocks * kLossThreads;
+  for (long long i = (long long)blockIdx.x * kLossThreads + threadIdx.x; i < nvec; i += stride) {
+    uint4 a = o[i], b = e[i];
+    uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w}, wr[4];
+    float sq = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&wa[j]);
+      const __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&wb[j]);
+      const float d0 = __low2float(x) - __low2float(y);
+      const float d1 = __high2float(x) - __high2float(y);
+      __nv_bfloat162 r = __floats2bfloat162_rn(d0, d1);
+      wr[j] = *reinterpret_cast<uint32_t*>(&r);
+      sq = fmaf(d0, d0, sq);
+      sq = fmaf(d1, d1, sq);
+    }
+    dO[i] = make_uint4(wr[0], wr[1], wr[2], wr[3]);
+    acc += (double)sq;
+  }
+  __shared__ double red[kLossThreads];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = kLossThreads / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[blockIdx.x] = red[0];
+}
+
+__global__ void __launch_bounds__(kLossBlocks) loss_final_kernel(const double* __restrict__ part,
+                                                                 float* __restrict__ L) {
+  __shared__ double red[kLossBlocks];
+  red[threadIdx.x] = part[threadIdx.x];
+  __syncthreads();
+  for (int w = kLossBlocks / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *L = (float)(0.5 * red[0]);
+}
+
+// ---------------------------------------------------------------- delta
+// One warp per row: Delta_row = sum_c dO[row, c] * O[row, c] in fp32.
+template <typename T>
+__global__ void delta_kernel(const T* __restrict__ o, const T* __restrict__ dO,
+                             float* __restrict__ delta, long long rows, int d) {
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int c = lane; c < d; c += 32) acc = fmaf(to_f(o[row * d + c]), to_f(dO[row * d + c]), acc);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) delta[row] = acc;
+}
+
+// bf16, d in {64, 128}: lanes load 8 bytes (4 elements) each, d/4 lanes per row.
+template <int D>
+__global__ void delta_bf16_kernel(const uint2* __restrict__ o, const uint2* __restrict__ dO,
+                                  float* __restrict__ delta, long long rows) {
+  constexpr int LPR = D / 4;           // lanes per row
+  constexpr int RPW = 32 / LPR;        // rows per warp
+  const int lane = threadIdx.x % 32;
+  const long long row =
+      ((long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32) * RPW + lane / LPR;
+  float acc = 0.f;
+  if (row < rows) {
+    const long long i = row * LPR + lane % LPR;
+    uint2 a = o[i], b = dO[i];
+    const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
+    const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
+    const __nv_bfloat162 b0 = *reinterpret_cast<__nv_bfloat162*>(&b.x);
+    const __nv_bfloat162 b1 = *reinterpret_cast<__nv_bfloat162*>(&b.y);
+    acc = __low2float(a0) * __low2float(b0);
+    acc = fmaf(__high2float(a0), __high2float(b0), acc);
+    acc = fmaf(__low2float(a1), __low2float(b1), acc);
+    acc = fmaf(__high2float(a1), __high2float(b1), acc);
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && lane % LPR == 0) delta[row] = acc;
+}
+
+// ---------------------------------------------------------------- dalpha final
+// One block per band m: fixed-order fp64 sum of the `count` partials part[i * M + m].
+__global__ void __launch_bounds__(256)
+    dalpha_final_kernel(const float* __restrict__ part, const float* __restrict__ alpha,
+                        float* __restrict__ dalpha, long long count, int M, int d, double base) {
+  const int m = blockIdx.x;
+  double acc = 0.0;
+  for (long long i = threadIdx.x; i < count; i += 256) acc += (double)part[i * M + m];
+  __shared__ double red[256];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) dalpha[m] = (float)(theta_hat(alpha, m, d, base) * red[0]);
+}
+
+// ================================================================ launchers
+cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table,
+                         cudaStream_t s) {
+  const int M = (int)(p.d / 2);
+  const long long total = p.n * M;
+  const int threads = 256;
+  rope_table_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(
+      alpha, table, (int)p.n, M, (int)p.d, p.base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate(const ra_problem& p, const void* q, const void* k, void* qt, void* kt,
+                          const float2* table, cudaStream_t s) {
+  const int M = (int)(p.d / 2);
+  const long long rows = p.B * p.H * p.n;
+  const int threads = 256;
+  if (p.dtype == RA_BF16 && M % 4 == 0) {
+    const long long total = rows * (M / 4);
+    dim3 grid((unsigned)((total + threads - 1) / threads), 2);
+    rotate_bf16x8_kernel<<<grid, threads, 0, s>>>(
+        (const uint4*)q, (const uint4*)k, (uint4*)qt, (uint4*)kt, table, rows, (int)p.n, M);
+  } else {
+    const long long total = rows * M;
+    dim3 grid((unsigned)((total + threads - 1) / threads), 2);
+    if (p.dtype == RA_BF16)
+      rotate_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(
+          (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qt,
+          (__nv_bfloat16*)kt, table, rows, (int)p.n, M);
+    else
+      rotate_kernel<float><<<grid, threads, 0, s>>>((const float*)q, (const float*)k,
+                                                    (float*)qt, (float*)kt, table, rows,
+                                                    (int)p.n, M);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loss_partial(const ra_problem& p, const void* o, const void* e, void* dO,
+                                double* part, cudaStream_t s) {
+  const long long count = p.B * p.H * p.n * p.d;
+  if (p.dtype == RA_BF16 && count % 8 == 0)
+    loss_partial_bf16x8_kernel<<<kLossBlocks, kLossThreads, 0, s>>>(
+        (const uint4*)o, (const uint4*)e, (uint4*)dO, part, count / 8);
+  else if (p.dtype == RA_BF16)
+    loss_partial_kernel<__nv_bfloat16><<<kLossBlocks, kLossThreads, 0, s>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)e, (__nv_bfloat16*)dO, part, count);
+  else
+    loss_partial_kernel<float><<<kLossBlocks, kLossThreads, 0, s>>>(
+        (const float*)o, (const float*)e, (float*)dO, part, count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loss_final(const double* part, float* L, cudaStream_t s) {
+  loss_final_kernel<<<1, kLossBlocks, 0, s>>>(part, L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, float* delta,
+                         cudaStream_t s) {
+  const long long rows = p.B * p.H * p.n;
+  const int threads = 256, warps = threads / 32;
+  if (p.dtype == RA_BF16 && (p.d == 64 || p.d == 128)) {
+    const int rpw = p.d == 64 ? 2 : 1;
+    const long long nwarps = (rows + rpw - 1) / rpw;
+    const unsigned blocks = (unsigned)((nwarps + warps - 1) / warps);
+    if (p.d == 64)
+      delta_bf16_kernel<64><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, delta,
+                                                       rows);
+    else
+      delta_bf16_kernel<128><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, delta,
+                                                        rows);
+  } else {
+    const unsigned blocks = (unsigned)((rows + warps - 1) / warps);
+    if (p.dtype == RA_BF16)
+      delta_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
+          (const __nv_bfloat16*)o, (const __nv_bfloat16*)dO, delta, rows, (int)p.d);
+    else
+      delta_kernel<float><<<blocks, threads, 0, s>>>((const float*)o, (const float*)dO, delta,
+                                                     rows, (int)p.d);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dalpha_final(const ra_problem& p, const float* part, const float* alpha,
+                                float* dalpha, cudaStream_t s) {
+  const int M = (int)(p.d / 2);
+  const long long ntile = (p.n + kDalphaRows - 1) / kDalphaRows;
+  const long long count = 2 * p.B * p.H * ntile;
+  dalpha_final_kernel<<<M, 256, 0, s>>>(part, alpha, dalpha, count, M, (int)p.d, p.base);
+  return cudaGetLastError();
+}
+
+}  // namespace ra

@@ -1,0 +1,345 @@
+// fwd_sm100.cu -- exact RoPE attention forward on B200 tensor cores (tcgen05).
+//
+// Computes, for one 128-row tile of queries of one (batch, head):
+//   S = Q~ K~^T / sqrt(d) tile by tile, the online-softmax row max and row sum,
+//   O = sum_j P_j V_j / l and lse = log sum_j exp(S_ij)
+// ("RoPE attention can be trained in almost-linear time", Metodologia 1: the
+// normalised softmax s(x) applied to the RoPE scores; Q~, K~ are the queries and
+// keys rotated band by band, "LeRoPE: learnable RoPE frequencies", Mecanismo
+// Central).  Exact: no approximation, fp32 accumulation, bf16 operands.
+//
+// CTA = 6 warps, one 128-row query tile, 1 CTA per SM:
+//   warps 0-3  softmax: thread t owns row t (= TMEM lane t) of S and O
+//   warp  4    TMA producer: Q~ once, then K~_j / V_j into a 2-stage ring
+//   warp  5    TMEM allocator + single-thread tcgen05.mma issuer
+// TMEM (512 columns): S double buffer at columns 0 and 128, O at column 256.
+// The issuer runs one tile ahead: S_{j+1} = Q~ K~_{j+1}^T is on the tensor core
+// while the softmax warps turn S_j into P_j (bf16, written to shared memory in
+// the K-major 128B-swizzled layout the MMA reads) and rescale O; then
+// O += P_j V_j.  Every wait is bounded; an expired wait records RA_ERR_TIMEOUT
+// in the workspace error word and the CTA drains its copies and MMAs and exits.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "common.h"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace ra {
+namespace {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128, BN = 128, NS = 2;
+  static constexpr int CH = D / 64;                       // 64-column chunks per row
+  static constexpr uint32_t CHUNK = 128u * 128u;          // [128 rows][128 B]
+  static constexpr uint32_t TILE = CHUNK * CH;            // [128][D] bf16
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + TILE;
+  static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
+  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // [128][128] bf16 = 2 chunks
+  static constexpr uint32_t OFF_BAR = OFF_P + 2 * CHUNK;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_O = 256;
+};
+
+enum FwdBar {
+  B_Q_FULL = 0,
+  B_K_FULL = 1,   // +stage
+  B_K_EMPTY = 3,  // +stage
+  B_V_FULL = 5,   // +stage
+  B_V_EMPTY = 7,  // +stage
+  B_S_FULL = 9,   // +buffer
+  B_S_FREE = 11,  // +buffer
+  B_P_FULL = 13,
+  B_O_DONE = 14,
+  B_DRAIN = 15,
+  B_COUNT = 16
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
+                     const __grid_constant__ CUtensorMap map_k,
+                     const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
+                     float* __restrict__ lse, int n, int BH, int causal, uint32_t* err,
+                     uint64_t wait_ns, int starve_block) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_s - raw_s);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * B_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * B_COUNT + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntq = (n + C::BM - 1) / C::BM;
+  const int tile = ntq - 1 - (int)(blockIdx.x / BH);  // heaviest causal tiles first
+  const int bh = (int)(blockIdx.x % BH);
+  const int ntk = (n + C::BN - 1) / C::BN;
+  const int nkv = causal ? min(tile + 1, ntk) : ntk;
+
+  if (threadIdx.x == 128) {
+    for (int i = 0; i < B_COUNT; ++i)
+      mbar_init(&bar[i], (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) ? 128 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      // starve_block (test hook, -1 = off): that CTA never loads Q~, so its issuer's
+      // bounded wait must expire and report RA_ERR_TIMEOUT instead of hanging.
+      const bool load_q = (int)blockIdx.x != starve_block;
+      if (load_q) {
+        mbar_arrive_expect_tx(&bar[B_Q_FULL], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &map_q, &bar[B_Q_FULL], c * 64,
+                      tile * C::BM, bh);
+      }
+      int issued_k = -1, issued_v = -1;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % C::NS;
+        const uint32_t ph = (j / C::NS) & 1;
+        if (!mbar_wait(&bar[B_K_EMPTY + s], ph ^ 1, abort_flag, err, K_FWD_SM100, 1, wait_ns))
+          break;
+        mbar_arrive_expect_tx(&bar[B_K_FULL + s], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(base + C::OFF_K + s * C::TILE + c * C::CHUNK, &map_k, &bar[B_K_FULL + s],
+                      c * 64, j * C::BN, bh);
+        issued_k = j;
+        if (!mbar_wait(&bar[B_V_EMPTY + s], ph ^ 1, abort_flag, err, K_FWD_SM100, 2, wait_ns))
+          break;
+        mbar_arrive_expect_tx(&bar[B_V_FULL + s], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(base + C::OFF_V + s * C::TILE + c * C::CHUNK, &map_v, &bar[B_V_FULL + s],
+                      c * 64, j * C::BN, bh);
+        issued_v = j;
+      }
+      if (*abort_flag) {
+        // Let every copy already in flight land before the CTA's shared memory goes away.
+        int dummy = 0;
+        if (load_q) mbar_wait(&bar[B_Q_FULL], 0, &dummy, err, K_FWD_SM100, 20, wait_ns);
+        for (int j = max(0, issued_k - C::NS + 1); j <= issued_k; ++j)
+          mbar_wait(&bar[B_K_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, K_FWD_SM100, 21,
+                    wait_ns);
+        for (int j = max(0, issued_v - C::NS + 1); j <= issued_v; ++j)
+          mbar_wait(&bar[B_V_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, K_FWD_SM100, 22,
+                    wait_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_s = base_s + C::OFF_Q, k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
+      const uint32_t p_s = base_s + C::OFF_P;
+      bool ok = mbar_wait(&bar[B_Q_FULL], 0, abort_flag, err, K_FWD_SM100, 3, wait_ns);
+      tc_fence_after();
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % C::NS, sb = j & 1;
+        if (!mbar_wait(&bar[B_K_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 4,
+                       wait_ns))
+          return false;
+        if (!mbar_wait(&bar[B_S_FREE + sb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 5,
+                       wait_ns))
+          return false;
+        tc_fence_after();
+        const uint32_t kb = k_s + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_S + sb * 128, sdesc_sw128(q_s + koff, 16, 1024),
+                      sdesc_sw128(kb + koff, 16, 1024), idS, kk > 0);
+        }
+        mma_commit(&bar[B_S_FULL + sb]);
+        mma_commit(&bar[B_K_EMPTY + s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv && !issue_s(j + 1)) break;
+        const int s = j % C::NS;
+        if (!mbar_wait(&bar[B_P_FULL], j & 1, abort_flag, err, K_FWD_SM100, 6, wait_ns)) break;
+        if (!mbar_wait(&bar[B_V_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 7,
+                       wait_ns))
+          break;
+        tc_fence_after();
+        const uint32_t vb = v_s + s * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint32_t poff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_O, sdesc_sw128(p_s + poff, 16, 1024),
+                      sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
+        }
+        mma_commit(&bar[B_O_DONE]);
+        mma_commit(&bar[B_V_EMPTY + s]);
+      }
+      // Every MMA issued above has finished once this commit arrives.
+      mma_commit(&bar[B_DRAIN]);
+      int dummy = 0;
+      mbar_wait(&bar[B_DRAIN], 0, &dummy, err, K_FWD_SM100, 23, wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int t = threadIdx.x;  // row within the tile == TMEM lane
+    const int row = tile * C::BM + t;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&bar[B_S_FULL + sb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 8,
+                     wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + C::COL_S + sb * 128 + 32 * c, r[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_wait_ld(r[c]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[c][i]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_S_FREE + sb]);
+
+      const int key0 = j * C::BN;
+      const bool need_mask = (key0 + C::BN > n) || (causal && j == tile);
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float v = x[i] * scale_log2;
+        if (need_mask) {
+          const int key = key0 + i;
+          if (key >= n || (causal && key > row)) v = -CUDART_INF_F;
+        }
+        x[i] = v;
+        mx = fmaxf(mx, v);
+      }
+      const float m_new = fmaxf(m, mx);
+      const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+      const float corr = fast_exp2(m - m_use);
+      float rs = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        x[i] = fast_exp2(x[i] - m_use);
+        rs += x[i];
+      }
+      l = l * corr + rs;
+      m = m_new;
+
+      if (j > 0 && !mbar_wait(&bar[B_O_DONE], (j - 1) & 1, abort_flag, err, K_FWD_SM100, 9,
+                              wait_ns)) {
+        ok = false;
+        break;
+      }
+      // P_j -> shared memory, K-major, 128B swizzle: row t, keys 64h .. 64h+63 in chunk h.
+      const uint32_t p_row = base_s + C::OFF_P;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* src = &x[h * 64 + u * 8];
+          st_shared_v4(p_row + h * C::CHUNK + sw128_off(t, u), pack_bf16x2(src[0], src[1]),
+                       pack_bf16x2(src[2], src[3]), pack_bf16x2(src[4], src[5]),
+                       pack_bf16x2(src[6], src[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      if (j > 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + C::COL_O + 32 * c, r);
+          tmem_wait_ld(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+          tmem_st32(lane_base + C::COL_O + 32 * c, r);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar[B_P_FULL]);
+    }
+    if (ok && mbar_wait(&bar[B_O_DONE], (nkv - 1) & 1, abort_flag, err, K_FWD_SM100, 10,
+                        wait_ns)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + C::COL_O + 32 * c, r);
+        tmem_wait_ld(r);
+        if (row < n) {
+          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * n + row) * D + 32 * c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float* f = reinterpret_cast<const float*>(&r[8 * u]);
+            dst[u] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv),
+                                pack_bf16x2(f[2] * inv, f[3] * inv),
+                                pack_bf16x2(f[4] * inv, f[5] * inv),
+                                pack_bf16x2(f[6] * inv, f[7] * inv));
+          }
+        }
+      }
+      if (row < n) lse[(size_t)bh * n + row] = (m + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
+                         const DevCtl& ctl, cudaStream_t s) {
+  using C = FwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(fwd_sm100_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int BH = (int)(p.B * p.H);
+  const long long ntq = (p.n + C::BM - 1) / C::BM;
+  fwd_sm100_kernel<D><<<(unsigned)(ntq * BH), 192, C::SMEM, s>>>(
+      maps.qt, maps.kt, maps.v, (__nv_bfloat16*)o, lse, (int)p.n, BH, p.causal, ctl.err,
+      ctl.wait_ns, ctl.starve_block);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
+                             const DevCtl& ctl, cudaStream_t s) {
+  if (p.d == 64) return launch_fwd_d<64>(p, maps, o, lse, ctl, s);
+  return launch_fwd_d<128>(p, maps, o, lse, ctl, s);
+}
+
+}  // namespace ra

@@ -1,0 +1,54 @@
+// launch.h -- host-side launchers of every kernel (defined next to the kernels).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.h"
+
+namespace ra {
+
+struct DevCtl {
+  uint32_t* err;        // workspace error word
+  uint64_t wait_ns;     // bound on every device-side wait
+  int starve_block;     // test hook: this CTA of the forward skips its Q~ load (-1 = off)
+};
+
+cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table, cudaStream_t s);
+cudaError_t launch_rotate(const ra_problem& p, const void* q, const void* k, void* qt, void* kt,
+                          const float2* table, cudaStream_t s);
+cudaError_t launch_loss_partial(const ra_problem& p, const void* o, const void* e, void* dO,
+                                double* part, cudaStream_t s);
+cudaError_t launch_loss_final(const double* part, float* L, cudaStream_t s);
+cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, float* delta,
+                         cudaStream_t s);
+cudaError_t launch_dalpha_final(const ra_problem& p, const float* part, const float* alpha,
+                                float* dalpha, cudaStream_t s);
+
+// fp32 CUDA-core attention (any even d <= 128)
+cudaError_t launch_fwd_f32(const ra_problem& p, const float* qt, const float* kt, const float* v,
+                           float* o, float* lse, cudaStream_t s);
+cudaError_t launch_bwd_dq_f32(const ra_problem& p, const float* qt, const float* kt,
+                              const float* v, const float* dO, const float* lse,
+                              const float* delta, const float2* table, float* dq, float* dpart,
+                              cudaStream_t s);
+cudaError_t launch_bwd_dkdv_f32(const ra_problem& p, const float* qt, const float* kt,
+                                const float* v, const float* dO, const float* lse,
+                                const float* delta, const float2* table, float* dk, float* dv,
+                                float* dpart, cudaStream_t s);
+
+// bf16 tcgen05 attention (d in {64, 128}); tensor maps are built by the caller.
+struct Sm100Maps {
+  CUtensorMap qt, kt, v, dO;     // boxes of 64 x 128 rows
+  CUtensorMap kt64, v64;         // boxes of 64 x 64 rows
+};
+cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
+                             const DevCtl& ctl, cudaStream_t s);
+cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps, const void* qt,
+                                  const void* kt, const float* lse, const float* delta,
+                                  const float2* table, void* dk, void* dv, float* dpart,
+                                  const DevCtl& ctl, cudaStream_t s);
+cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const void* qt,
+                                const float* lse, const float* delta, const float2* table,
+                                void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s);
+
+}  // namespace ra

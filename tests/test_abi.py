@@ -1,0 +1,103 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point the
+header declares, sizes workspaces, and rejects bad arguments before launching
+anything (none of these calls touches a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rope_attention_fwd_b200 import binding as rb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rope_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rope_attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 9
+    lib = rb.lib()
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    lib = rb.lib()
+    for code in range(6):
+        assert lib.rope_attn_status_string(code)
+    assert lib.rope_attn_status_string(0) == b"ok"
+
+
+def test_workspace_bytes():
+    p = rb.problem(2, 32, 8192, 128, rb.RA_BF16, True, 1e4)
+    nb = rb.rope_attn_workspace_bytes(p)
+    # two rotated bf16 tensors dominate: 2 * 2*32*8192*128*2 bytes
+    assert nb >= 2 * 2 * 32 * 8192 * 128 * 2
+    assert nb < 2 * 2 * 32 * 8192 * 128 * 2 * 1.1
+    assert nb % 1024 == 0
+
+
+@pytest.mark.parametrize("bad", [
+    dict(B=0), dict(H=0), dict(n=0), dict(d=3), dict(d=0), dict(dtype=7), dict(causal=2),
+    dict(base=0.0), dict(base=-1.0), dict(base=float("nan")),
+])
+def test_invalid_problem_has_no_workspace(bad):
+    args = dict(B=1, H=1, n=16, d=64, dtype=rb.RA_F32, causal=0, base=1e4)
+    args.update(bad)
+    p = rb.RaProblem(args["B"], args["H"], args["n"], args["d"], args["dtype"], args["causal"],
+                     args["base"])
+    assert rb.rope_attn_workspace_bytes(p) == 0
+
+
+@pytest.mark.parametrize("bad, code", [
+    (dict(d=96, dtype=rb.RA_BF16), 2), (dict(d=256), 2), (dict(d=32, dtype=rb.RA_BF16), 2),
+])
+def test_unsupported_problem(bad, code):
+    args = dict(B=1, H=1, n=16, d=64, dtype=rb.RA_F32, causal=0, base=1e4)
+    args.update(bad)
+    p = rb.RaProblem(args["B"], args["H"], args["n"], args["d"], args["dtype"], args["causal"],
+                     args["base"])
+    lib = rb.lib()
+    null = ctypes.c_void_p(0)
+    r = lib.rope_attn_fwd(ctypes.byref(p), null, null, null, null, null, null, null, 0, null)
+    assert r == code
+
+
+def test_null_pointers_rejected_before_launch():
+    lib = rb.lib()
+    p = rb.problem(1, 1, 16, 64, rb.RA_F32, False, 1e4)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(4096)        # aligned, never dereferenced: validation fails first
+    assert lib.rope_attn_fwd(ctypes.byref(p), null, fake, fake, fake, fake, fake, fake,
+                             1 << 20, null) == 1
+    assert lib.rope_attn_loss(ctypes.byref(p), fake, null, fake, fake, fake, 1 << 20, null) == 1
+    assert lib.rope_attn_bwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake,
+                             fake, fake, null, fake, fake, 1 << 20, null) == 1
+    misaligned = ctypes.c_void_p(4096 + 8)
+    assert lib.rope_attn_fwd(ctypes.byref(p), misaligned, fake, fake, fake, fake, fake, fake,
+                             1 << 20, null) == 1
+
+
+def test_workspace_checks_before_launch():
+    lib = rb.lib()
+    p = rb.problem(1, 1, 16, 64, rb.RA_F32, False, 1e4)
+    fake = ctypes.c_void_p(4096)
+    need = rb.rope_attn_workspace_bytes(p)
+    assert lib.rope_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake,
+                             need - 1, None) == 3
+    assert lib.rope_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake,
+                             ctypes.c_void_p(4096 + 16), need, None) == 3
+    assert lib.rope_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None,
+                             need, None) == 3
+
+
+def test_kernel_names():
+    lib = rb.lib()
+    names = {lib.rope_attn_kernel_name(i).decode() for i in range(12)}
+    assert {"fwd_sm100", "bwd_dkdv_sm100", "bwd_dq_sm100", "dalpha_final"} <= names

@@ -1,0 +1,96 @@
+"""GPU parity at sizes the oracle finishes in seconds: several tiles, ragged tails,
+n = 1, both dtypes, both head dimensions of the tensor-core path, causal and not.
+Every call goes through the C ABI; expected values come from the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import (TOL, compare, gpu_fwd, gpu_run, make, oracle_fwd, oracle_run,
+                     small_workload)
+
+pytestmark = pytest.mark.gpu
+
+F32_SHAPES = [(1, 1, 256, 64), (1, 2, 7, 8), (2, 1, 129, 64), (1, 1, 1, 64), (1, 2, 200, 128),
+              (1, 1, 65, 2), (1, 3, 96, 30)]
+BF16_N = [1, 7, 128, 129, 256, 383]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", F32_SHAPES)
+def test_f32_fwd_bwd(shape, causal):
+    wl = small_workload(*shape, "f32", causal, base=100.0, seed=sum(shape))
+    inp = make(wl)
+    compare(gpu_run(inp), oracle_run(inp), "f32")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n", BF16_N)
+def test_bf16_fwd(n, d, causal):
+    wl = small_workload(1, 2, n, d, "bf16", causal, seed=n + d)
+    inp = make(wl)
+    compare(gpu_fwd(inp), oracle_fwd(inp), "bf16", keys=("o", "lse"))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("n", BF16_N)
+def test_bf16_fwd_bwd(n, d, causal):
+    wl = small_workload(1, 2, n, d, "bf16", causal, seed=3 * n + d)
+    inp = make(wl)
+    compare(gpu_run(inp), oracle_run(inp), "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_deterministic(dtype):
+    """No atomics, fixed-order reductions: two runs agree bit for bit."""
+    wl = small_workload(2, 2, 300, 64, dtype, True, seed=11)
+    inp = make(wl)
+    a, b = gpu_run(inp), gpu_run(inp)
+    for key in ("o", "lse", "dq", "dk", "dv", "dalpha"):
+        assert np.array_equal(a[key], b[key]), key
+    assert a["L"] == b["L"]
+
+
+def test_bf16_many_heads_and_batches():
+    wl = small_workload(3, 5, 160, 64, "bf16", True, seed=5)
+    inp = make(wl)
+    compare(gpu_run(inp), oracle_run(inp), "bf16")
+
+
+def test_bf16_large_entries():
+    """Bounded-entry regime at a small size: uniform[-3, 3] entries, sharp softmax."""
+    wl = small_workload(1, 2, 300, 128, "bf16", False, base=5e5, seed=4, qkve="uniform")
+    wl = wl.with_(lo=-3.0, hi=3.0)
+    inp = make(wl)
+    compare(gpu_run(inp), oracle_run(inp), "bf16")
+
+
+def test_bf16_spread_frequencies():
+    """Near-zero-frequency bands: e^alpha spans [1e-3, 4]."""
+    wl = small_workload(1, 2, 256, 128, "bf16", True, base=5e5, seed=6)
+    wl = wl.with_(alpha="uniform", alpha_a=float(np.log(1e-3)), alpha_b=float(np.log(4.0)))
+    inp = make(wl)
+    compare(gpu_run(inp), oracle_run(inp), "bf16")
+
+
+def test_guard_bands_untouched():
+    """Outputs are written only inside their extents: NaN-filled canaries around o stay NaN."""
+    from rope_attention_fwd_b200 import binding as rb
+    wl = small_workload(1, 2, 129, 128, "bf16", True, seed=9)
+    inp = make(wl)
+    dev = "cuda"
+    q, k, v, alpha = (getattr(inp, x).to(dev) for x in ("q", "k", "v", "alpha"))
+    numel = q.numel()
+    pad = 4096
+    buf = torch.full((numel + 2 * pad,), float("nan"), dtype=torch.bfloat16, device=dev)
+    o = buf[pad:pad + numel].view_as(q)
+    lbuf = torch.full((2 * pad + 2 * 129,), float("nan"), dtype=torch.float32, device=dev)
+    lse = lbuf[pad:pad + 2 * 129].view(1, 2, 129)
+    rb.rope_attn_fwd(q, k, v, alpha, wl.base, wl.causal, o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.isnan(buf[:pad].float()).all() and torch.isnan(buf[pad + numel:].float()).all()
+    assert torch.isnan(lbuf[:pad]).all() and torch.isnan(lbuf[pad + 258:]).all()
+    assert not torch.isnan(o.float()).any()
+    np.testing.assert_array_less(np.abs(o.double().cpu().numpy() - oracle_fwd(inp)["o"]),
+                                 TOL["bf16"]["o"])

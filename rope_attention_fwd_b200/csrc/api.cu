@@ -234,8 +234,8 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
   float* delta = at<float>(ws, L.delta);
   float* dpart = at<float>(ws, L.dpart);
   const float2* table = at<float2>(ws, L.table);
-  RA_LAUNCH(K_BWD_DELTA, s, launch_delta(*p, o, dO, delta, s));
   if (p->dtype == RA_F32) {
+    RA_LAUNCH(K_BWD_DELTA, s, launch_delta(*p, o, dO, delta, s));
     const float* qt = at<float>(ws, L.qt);
     const float* kt = at<float>(ws, L.kt);
     RA_LAUNCH(K_BWD_DKDV_F32, s,
@@ -245,20 +245,22 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
               launch_bwd_dq_f32(*p, qt, kt, (const float*)v, (const float*)dO, lse, delta, table,
                                 (float*)dq, dpart, s));
   } else {
+    float* lse2 = at<float>(ws, L.lse2);
+    RA_LAUNCH(K_BWD_DELTA, s, launch_bwd_pre(*p, o, dO, lse, delta, lse2, s));
     Sm100Maps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!make_map(&maps.qt, at<void>(ws, L.qt), *p, 128) ||
-        !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128) || !make_map(&maps.v, v, *p, 128) ||
-        !make_map(&maps.dO, dO, *p, 128) || !make_map(&maps.kt64, at<void>(ws, L.kt), *p, 64) ||
-        !make_map(&maps.v64, v, *p, 64))
+    void* qt = at<void>(ws, L.qt);
+    void* kt = at<void>(ws, L.kt);
+    if (!make_map(&maps.qt, qt, *p, 128) || !make_map(&maps.kt, kt, *p, 128) ||
+        !make_map(&maps.v, v, *p, 128) || !make_map(&maps.dO, dO, *p, 128) ||
+        !make_map(&maps.qt64, qt, *p, 64) || !make_map(&maps.kt64, kt, *p, 64) ||
+        !make_map(&maps.v64, v, *p, 64) || !make_map(&maps.dO64, dO, *p, 64))
       return RA_ERR_CUDA;
     DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
     RA_LAUNCH(K_BWD_DKDV_SM100, s,
-              launch_bwd_dkdv_sm100(*p, maps, at<void>(ws, L.qt), at<void>(ws, L.kt), lse, delta,
-                                    table, dk, dv, dpart, ctl, s));
+              launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, dk, dv, dpart, ctl, s));
     RA_LAUNCH(K_BWD_DQ_SM100, s,
-              launch_bwd_dq_sm100(*p, maps, at<void>(ws, L.qt), lse, delta, table, dq, dpart,
-                                  ctl, s));
+              launch_bwd_dq_sm100(*p, maps, lse2, delta, table, dq, dpart, ctl, s));
   }
   RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;

@@ -38,10 +38,14 @@ struct WsLayout {
   size_t table;      // float2 [n][M]  (cos, sin)
   size_t qt;         // dtype [B*H][n][d]   rotated queries
   size_t kt;         // dtype [B*H][n][d]   rotated keys
-  size_t delta;      // float [B*H][n]      rowsum(dO o O)
+  size_t delta;      // float [B*H][npad]   rowsum(dO o O); 0 on rows >= n
+  size_t lse2;       // float [B*H][npad]   lse * log2(e); +inf on rows >= n
   size_t dpart;      // float [2][B*H][ceil(n/kDalphaRows)][M]
   size_t total;
 };
+
+// Rows of the padded per-row vectors (a whole number of 128-row tiles).
+inline int64_t padded_rows(int64_t n) { return (n + 127) / 128 * 128; }
 
 inline WsLayout ws_layout(const ra_problem& p) {
   const size_t elem = p.dtype == RA_BF16 ? 2 : 4;
@@ -60,7 +64,9 @@ inline WsLayout ws_layout(const ra_problem& p) {
   w.table = take(sizeof(float) * 2 * n * M);
   w.qt = take(elem * BH * n * d);
   w.kt = take(elem * BH * n * d);
-  w.delta = take(sizeof(float) * BH * n);
+  const size_t npad = (size_t)padded_rows(p.n);
+  w.delta = take(sizeof(float) * BH * npad);
+  w.lse2 = take(sizeof(float) * BH * npad);
   w.dpart = take(sizeof(float) * 2 * BH * ntile * M);
   w.total = off;
   return w;

@@ -213,6 +213,42 @@ __global__ void delta_bf16_kernel(const uint2* __restrict__ o, const uint2* __re
   if (row < rows && lane % LPR == 0) delta[row] = acc;
 }
 
+// Padded per-row vectors for the tensor-core backward, over npad = ceil(n/128)*128 rows
+// per head: deltap = rowsum(dO o O) (0 past n) and lse2p = lse * log2(e) (+inf past n,
+// so that exp2(s - lse2) vanishes on the padding rows the tiles read).
+template <int D>
+__global__ void bwd_pre_bf16_kernel(const uint2* __restrict__ o, const uint2* __restrict__ dO,
+                                    const float* __restrict__ lse, float* __restrict__ deltap,
+                                    float* __restrict__ lse2p, long long prow_count, int n,
+                                    int npad) {
+  constexpr int LPR = D / 4, RPW = 32 / LPR;
+  const int lane = threadIdx.x % 32;
+  const long long prow =
+      ((long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32) * RPW + lane / LPR;
+  const long long bh = prow / npad;
+  const int i = (int)(prow % npad);
+  const bool live = prow < prow_count && i < n;
+  float acc = 0.f;
+  if (live) {
+    const long long idx = (bh * n + i) * LPR + lane % LPR;
+    uint2 a = o[idx], b = dO[idx];
+    const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
+    const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
+    const __nv_bfloat162 b0 = *reinterpret_cast<__nv_bfloat162*>(&b.x);
+    const __nv_bfloat162 b1 = *reinterpret_cast<__nv_bfloat162*>(&b.y);
+    acc = __low2float(a0) * __low2float(b0);
+    acc = fmaf(__high2float(a0), __high2float(b0), acc);
+    acc = fmaf(__low2float(a1), __low2float(b1), acc);
+    acc = fmaf(__high2float(a1), __high2float(b1), acc);
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (prow < prow_count && lane % LPR == 0) {
+    deltap[prow] = acc;
+    lse2p[prow] = live ? lse[bh * n + i] * 1.4426950408889634f : __int_as_float(0x7f800000);
+  }
+}
+
 // ---------------------------------------------------------------- dalpha final
 // One block per band m: fixed-order fp64 sum of the `count` partials part[i * M + m].
 __global__ void __launch_bounds__(256)
@@ -310,6 +346,23 @@ cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, flo
       delta_kernel<float><<<blocks, threads, 0, s>>>((const float*)o, (const float*)dO, delta,
                                                      rows, (int)p.d);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
+                           float* deltap, float* lse2p, cudaStream_t s) {
+  const int npad = (int)padded_rows(p.n);
+  const long long prows = p.B * p.H * npad;
+  const int threads = 256, warps = threads / 32;
+  const int rpw = p.d == 64 ? 2 : 1;
+  const long long nwarps = (prows + rpw - 1) / rpw;
+  const unsigned blocks = (unsigned)((nwarps + warps - 1) / warps);
+  if (p.d == 64)
+    bwd_pre_bf16_kernel<64><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
+                                                       deltap, lse2p, prows, (int)p.n, npad);
+  else
+    bwd_pre_bf16_kernel<128><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
+                                                        deltap, lse2p, prows, (int)p.n, npad);
   return cudaGetLastError();
 }
 

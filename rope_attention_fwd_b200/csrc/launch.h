@@ -38,17 +38,20 @@ cudaError_t launch_bwd_dkdv_f32(const ra_problem& p, const float* qt, const floa
 
 // bf16 tcgen05 attention (d in {64, 128}); tensor maps are built by the caller.
 struct Sm100Maps {
-  CUtensorMap qt, kt, v, dO;     // boxes of 64 x 128 rows
-  CUtensorMap kt64, v64;         // boxes of 64 x 64 rows
+  CUtensorMap qt, kt, v, dO;         // boxes of 64 columns x 128 rows
+  CUtensorMap qt64, kt64, v64, dO64; // boxes of 64 columns x 64 rows
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
-cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps, const void* qt,
-                                  const void* kt, const float* lse, const float* delta,
-                                  const float2* table, void* dk, void* dv, float* dpart,
-                                  const DevCtl& ctl, cudaStream_t s);
-cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const void* qt,
-                                const float* lse, const float* delta, const float2* table,
-                                void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s);
+// Padded per-row vectors for the tensor-core backward: delta and lse * log2(e).
+cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
+                           float* deltap, float* lse2p, cudaStream_t s);
+cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
+                                  const float* lse2p, const float* deltap, const float2* table,
+                                  void* dk, void* dv, float* dpart, const DevCtl& ctl,
+                                  cudaStream_t s);
+cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
+                                const float* deltap, const float2* table, void* dq, float* dpart,
+                                const DevCtl& ctl, cudaStream_t s);
 
 }  // namespace ra

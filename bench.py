@@ -1,0 +1,380 @@
+"""Benchmark: RoPE/LeRoPE attention fwd + loss + bwd (incl. dalpha) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+
+One step = the whole path on one batch: rope_attn_fwd (table, rotation, tcgen05
+forward), rope_attn_loss, rope_attn_bwd (table, rotation, Delta, dK/dV, dQ, dalpha).
+Workload: 2 x 32 x 8192 x 128 bf16 causal, base 1e4, alpha ~ N(0, 0.3^2) -- the
+headline configuration.  Metric: fwd+bwd TFLOP/s with the standard count
+14 n^2 d per (batch, head), halved for causal masking.  Inputs (4 x 134 MB) exceed
+the 126 MB L2, so no flush is needed between steps.
+
+With --gpus N > 1 (under torchrun) every rank runs the same workload on its own
+batch (seeded by rank): per-GPU work is fixed (weak scaling) and the one exchange the
+method has -- the dalpha of the shared LeRoPE frequencies, summed over every head of
+every rank -- is an NCCL all-reduce of d/2 floats per step.
+
+--impl reference times the float64 CPU oracle (the only other implementation of the
+method; the pages ship no code) on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def workload(cfg):
+    from rope_attention_fwd_b200.configs import WORKLOADS
+    return WORKLOADS[cfg]
+
+
+def config_dict(wl, cfg, world):
+    return {"workload": f"config {cfg}: {wl.name}", "B": wl.B, "H": wl.H, "n": wl.n, "d": wl.d,
+            "causal": wl.causal, "base": wl.base, "global_batch": wl.B * world,
+            "seq_len": wl.n, "parallelism": f"dp{world}" if world > 1 else "single-gpu",
+            "l2": "inputs larger than L2 (4 x %.0f MB > 126 MB), no flush" %
+                  (wl.B * wl.H * wl.n * wl.d * 2 / 1e6)}
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm = float(parts[1].split()[0])
+                    mx = float(parts[2].split()[0])
+                except ValueError:
+                    continue
+                rows.append((sm, mx, parts[5:9]))
+            os.remove(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4)
+                          if r[i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- oracle timing
+def time_oracle(wl, max_seconds=30.0):
+    """Oracle fwd+loss+bwd of one (batch, head) of the workload; FLOPs by the metric's
+    count for that one head.  Returns (TFLOP/s, seconds, sample description, threads)."""
+    import numpy as np
+    import torch
+    from oracle import rope_attn_ref as ref
+    from rope_attention_fwd_b200.inputs import make_inputs
+    one = wl.with_(B=1, H=1)
+    inp = make_inputs(one)
+    q, k, v, e, al = (inp.f64(x) for x in ("q", "k", "v", "e", "alpha"))
+    t0 = time.perf_counter()
+    ref.forward_backward(q, k, v, e, al, one.base, one.causal)
+    dt = time.perf_counter() - t0
+    flops = one.flops_fwd() + one.flops_bwd()
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except AttributeError:
+        threads = os.cpu_count()
+    sample = (f"1 of {wl.B * wl.H} (batch, head) slices of the workload "
+              f"(n={wl.n}, d={wl.d}), full fwd+loss+bwd, float64 numpy")
+    return flops / dt / 1e12, dt, sample, threads
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = workload(args.config)
+    vals = []
+    for _ in range(max(0, args.warmup_ref)):
+        time_oracle(wl)
+    total = 0.0
+    for _ in range(args.steps_ref):
+        v, dt, sample, threads = time_oracle(wl)
+        vals.append(v)
+        total += dt
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": "RoPE-attn fwd+bwd TFLOP/s (bf16, incl. dalpha)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps_ref,
+            "steps_requested": args.steps,
+            "warmup": args.warmup_ref, "ms_per_step": 1e3 * total / max(1, args.steps_ref),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(wl, args.config, world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from rope_attention_fwd_b200 import binding as rb
+    from rope_attention_fwd_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    wl = workload(args.config)
+    inp = make_inputs(wl, seed=wl.seed + 7919 * rank)
+    flops_fwd, flops_bwd = wl.flops_fwd(), wl.flops_bwd()
+    flops = flops_fwd + flops_bwd
+
+    host = {x: getattr(inp, x).pin_memory() for x in ("q", "k", "v", "e", "alpha")}
+    dv_in = {x: host[x].to(dev) for x in host}
+    prob = rb.problem(wl.B, wl.H, wl.n, wl.d, dv_in["q"].dtype, wl.causal, wl.base)
+    ws = rb.workspace(prob, dev)
+    o = torch.empty_like(dv_in["q"])
+    lse = torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, device=dev)
+    L = torch.empty((), dtype=torch.float32, device=dev)
+    dO = torch.empty_like(o)
+    dq, dk, dvv = (torch.empty_like(o) for _ in range(3))
+    dalpha = torch.empty(wl.d // 2, dtype=torch.float32, device=dev)
+
+    def step(t):
+        rb.rope_attn_fwd(t["q"], t["k"], t["v"], t["alpha"], wl.base, wl.causal, ws=ws, o=o,
+                         lse=lse)
+        rb.rope_attn_loss(o, t["e"], ws=ws, L=L, dO=dO)
+        rb.rope_attn_bwd(t["q"], t["k"], t["v"], o, lse, dO, t["alpha"], wl.base, wl.causal,
+                         ws=ws, dq=dq, dk=dk, dv=dvv, dalpha=dalpha)
+        if world > 1:
+            dist.all_reduce(dalpha)  # sum over every head of every rank
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream(dev)
+    # ---------------- device-resident timing
+    for _ in range(args.warmup):
+        step(dv_in)
+    barrier()
+    code, info = rb.rope_attn_device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {rb.STATUS.get(code, code)} {info}")
+    rb.rope_attn_timing_read()
+    rb.rope_attn_timing_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(dv_in)
+        ev1.record(stream)
+        barrier()
+    rb.rope_attn_timing_enable(False)
+    kernels = rb.rope_attn_timing_read()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms)
+    clocks = clk.summary()
+    value = world * flops / (ms * 1e-3) / 1e12
+    launches = sum(c for c, _ in kernels.values())
+
+    # ---------------- end-to-end through host buffers (copies inside the timed region)
+    h2d = sum(host[x].numel() * host[x].element_size() for x in host)
+    d2h = 4 + 4 * (wl.d // 2)
+    L_host = torch.empty((), dtype=torch.float32).pin_memory()
+    da_host = torch.empty(wl.d // 2, dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, args.steps // 2)
+
+    def e2e_step():
+        t = {x: host[x].to(dev, non_blocking=True) for x in host}
+        step(t)
+        L_host.copy_(L, non_blocking=True)
+        da_host.copy_(dalpha, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps)
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---------------- roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    f = 0.5 if wl.causal else 1.0
+    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0}
+    per_kernel = {name: {"launches": c, "avg_ms": t / c, "share": t / sum(
+        tt for _, tt in kernels.values())} for name, (c, t) in kernels.items()}
+    dom = max(kernels, key=lambda k: kernels[k][1])
+    dom_avg_s = kernels[dom][1] / kernels[dom][0] * 1e-3
+    roof = None
+    if dom in alg:
+        alg_flops = alg[dom] * wl.B * wl.H * wl.n * wl.n * wl.d * f
+        achieved = alg_flops / dom_avg_s / 1e12
+        peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": f"{peak_kind} bf16 burst", "traffic": traffic_for(dom)}
+        for name in kernels:
+            if name in alg:
+                a = alg[name] * wl.B * wl.H * wl.n * wl.n * wl.d * f
+                per_kernel[name]["alg_tflops"] = a / (per_kernel[name]["avg_ms"] * 1e-3) / 1e12
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, dt, sample, threads = time_oracle(wl)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": sample + f" ({dt:.1f} s)"}
+
+    line = {
+        "metric": "RoPE-attn fwd+bwd TFLOP/s (bf16, incl. dalpha)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(wl, args.config, world),
+        "fwd_tflops_per_gpu": phase_tflops(kernels, FWD_KERNELS, flops_fwd, args.steps),
+        "bwd_tflops_per_gpu": phase_tflops(kernels, BWD_KERNELS, flops_bwd, args.steps),
+        "pct_of_nominal_bf16_peak": 100 * value / world / NOMINAL_BF16_TFLOPS,
+        "pct_of_measured_bf16_peak": 100 * value / world / peaks.get(
+            "bf16_tflops", FALLBACK["bf16_tflops"]),
+        "roofline": roof,
+        "kernels": per_kernel,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+# Kernels of each phase; the table and rotation run once in fwd and once in bwd.
+FWD_KERNELS = {"rope_table": 0.5, "rotate": 0.5, "fwd_sm100": 1.0}
+BWD_KERNELS = {"rope_table": 0.5, "rotate": 0.5, "bwd_delta": 1.0, "bwd_dkdv_sm100": 1.0,
+               "bwd_dq_sm100": 1.0, "dalpha_final": 1.0}
+
+
+def phase_tflops(kernels, share, flops, steps):
+    ms = sum(w * kernels[k][1] for k, w in share.items() if k in kernels) / steps
+    return flops / (ms * 1e-3) / 1e12 if ms > 0 else None
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "rope_attention_fwd_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return rec["bytes_per_launch"] if sha == rec["source_sha256"] else None
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=3, choices=[2, 3, 4, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be at least 3")
+    # the reference arm times a slow CPU program: bound its work per step
+    args.steps_ref = max(1, min(args.steps, 3))
+    args.warmup_ref = 0
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,14 +1,691 @@
-// bwd_sm100.cu -- placeholder until the tcgen05 backward kernels land.
+// bwd_sm100.cu -- exact RoPE attention backward on B200 tensor cores (tcgen05).
+//
+// The gradient follows "RoPE attention can be trained in almost-linear time",
+// Metodologia 1-2: with s(x) the normalised softmax P, l(x) = dO the error term and
+// beta(x) = dP = dO V^T, gamma(x) = diag(s) beta - s s^T beta is dS = P o (dP - Delta)
+// row by row, Delta_i = rowsum(dO_i o O_i).  Then dV = P^T dO, dK~ = dS^T Q~ / sqrt(d),
+// dQ~ = dS K~ / sqrt(d).  On the way out each gradient row is rotated back by -p*theta_hat
+// and its per-band torque (p - c) <dX~_pm, J x~_pm> (c = (n-1)/2) is reduced into one
+// partial per 64 rows for the LeRoPE frequency gradient ("LeRoPE: learnable RoPE
+// frequencies", Analise Teorica; alpha shared by all heads, Escolhas de Design
+// Principais).  Centring at c changes nothing in exact arithmetic: for each band the
+// Q-side and K-side torques of one head sum to zero, because rotating every query and
+// key by one common angle leaves every score unchanged.
+//
+// The torque uses the same bf16 x~ the MMAs consumed (read back from shared memory).
+// The gradients are those of the function evaluated at those bf16 operands, and with
+// the same x~ in the torque the Q/K cancellation above stays exact for that function.
+// Recomputing x~ in fp32 for the torque breaks it: on the 4x16x2048x64 causal workload
+// a CPU model of the roundings puts the dalpha error at 1.0e-2 that way, 3.8e-3 this way.
+//
+// Two kernels, no atomics (deterministic):
+//   dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
+//         time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
+//         (M = 128 keys, N = 64 queries), the softmax warps form P^T and dS^T in bf16,
+//         then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
+//         accumulated in TMEM for the whole pass.
+//   dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
+//         dP = dO V_j^T (double-buffered in TMEM), dS in bf16, dQ~ += dS K~_j.
+// Warp roles as in the forward: warps 0-3 own one TMEM lane / row each, warp 4 issues
+// TMA copies, warp 5 allocates TMEM and issues tcgen05.mma.  Every wait is bounded.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.h"
 #include "launch.h"
+#include "sm100.cuh"
+
 namespace ra {
-cudaError_t launch_bwd_dkdv_sm100(const ra_problem&, const Sm100Maps&, const void*, const void*,
-                                  const float*, const float*, const float2*, void*, void*, float*,
-                                  const DevCtl&, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void softmax_group_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
 }
-cudaError_t launch_bwd_dq_sm100(const ra_problem&, const Sm100Maps&, const void*, const float*,
-                                const float*, const float2*, void*, float*, const DevCtl&,
-                                cudaStream_t) {
-  return cudaErrorNotSupported;
+
+// Epilogue of one gradient row held in TMEM (D fp32 columns from tmem_acc, this
+// thread's lane): g = acc * scale is dX~ of position `pos`; writes R(-pos theta_hat) g as
+// bf16 to out_row (when live) and the band torques w * (g1 x0 - g0 x1) to red_row, where
+// x~ is row t of the 128B-swizzled bf16 tile at x_tile_s (chunk stride x_chunk).
+template <int D>
+__device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_tile_s,
+                                                  uint32_t x_chunk, int t,
+                                                  const float2* __restrict__ trow, float scale,
+                                                  float w, bool live,
+                                                  __nv_bfloat16* __restrict__ out_row,
+                                                  float* red_row) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tmem_acc + 32 * c, r);
+    tmem_wait_ld(r);
+    const uint32_t ch = x_tile_s + (uint32_t)((32 * c) / 64) * x_chunk;
+    const int u0 = ((32 * c) % 64) / 8;
+    uint32_t xw[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      ld_shared_v4(ch + sw128_off(t, u0 + u), xw[4 * u], xw[4 * u + 1], xw[4 * u + 2],
+                   xw[4 * u + 3]);
+    uint32_t ow[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float g0 = __uint_as_float(r[2 * k]) * scale;
+      const float g1 = __uint_as_float(r[2 * k + 1]) * scale;
+      const __nv_bfloat162 xp = *reinterpret_cast<const __nv_bfloat162*>(&xw[k]);
+      const float x0 = __low2float(xp), x1 = __high2float(xp);
+      const float2 cs = live ? trow[16 * c + k] : make_float2(1.f, 0.f);
+      ow[k] = pack_bf16x2(cs.x * g0 + cs.y * g1, cs.x * g1 - cs.y * g0);
+      red_row[16 * c + k] = live ? w * (g1 * x0 - g0 * x1) : 0.f;
+    }
+    if (live) {
+      uint4* dst = reinterpret_cast<uint4*>(out_row + 32 * c);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        dst[u] = make_uint4(ow[4 * u], ow[4 * u + 1], ow[4 * u + 2], ow[4 * u + 3]);
+    }
+  }
 }
+
+// Fixed-order per-band sums of the torques of rows 0-63 and 64-127 (red is [128][M+1]),
+// written as the partials of 64-row tiles 2*tile128 and 2*tile128+1 (when they exist).
+template <int D>
+__device__ __forceinline__ void write_dalpha_partials(const float* red, float* dpart_side_bh,
+                                                      int tile128, int ntile64, int t) {
+  constexpr int M = D / 2;
+  const int half = t / 64, m = t % 64;
+  if (m < M) {
+    const int tile64 = 2 * tile128 + half;
+    float s = 0.f;
+    for (int r = 0; r < 64; ++r) s += red[(half * 64 + r) * (M + 1) + m];
+    if (tile64 < ntile64) dpart_side_bh[(size_t)tile64 * M + m] = s;
+  }
+}
+
+// ======================================================================== dK, dV
+template <int D>
+struct DkdvCfg {
+  static constexpr int BN = 128, BQ = 64, NS = 2, CH = D / 64;
+  static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
+  static constexpr uint32_t KTILE = KCH * CH;
+  static constexpr uint32_t QCH = 64u * 128u;   // chunk of a 64-row tile
+  static constexpr uint32_t QTILE = QCH * CH;
+  static constexpr uint32_t VEC = BQ * 4;
+  static constexpr uint32_t STAGE = (2 * QTILE + 2 * VEC + 1023) / 1024 * 1024;
+  static constexpr uint32_t OFF_K = 0, OFF_V = KTILE, OFF_ST = 2 * KTILE;
+  static constexpr uint32_t OFF_P = OFF_ST + NS * STAGE;  // P^T  [128 keys][64 queries]
+  static constexpr uint32_t OFF_DS = OFF_P + KCH;         // dS^T [128 keys][64 queries]
+  static constexpr uint32_t OFF_BAR = OFF_DS + KCH;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 128, COL_DK = 128 + D;
+  static constexpr uint32_t TMEM_COLS = (128 + 2 * D) <= 256 ? 256 : 512;
+  static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
+};
+
+enum DkdvBar {
+  KB_KV_FULL = 0,
+  KB_Q_FULL = 1,   // +stage (2)
+  KB_Q_EMPTY = 3,  // +stage (2)
+  KB_S_FULL = 5,
+  KB_DP_FULL = 6,
+  KB_ST_FREE = 7,  // 128 arrivals
+  KB_DS_FULL = 8,  // 128 arrivals
+  KB_PDS_FREE = 9,
+  KB_ACC_DONE = 10,
+  KB_DRAIN = 11,
+  KB_COUNT = 12
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_kt,
+                    const __grid_constant__ CUtensorMap map_v,
+                    const __grid_constant__ CUtensorMap map_qt64,
+                    const __grid_constant__ CUtensorMap map_do64, const float* __restrict__ lse2p,
+                    const float* __restrict__ deltap, const float2* __restrict__ table,
+                    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    float* __restrict__ dpart, int n, int BH, int causal, uint32_t* err,
+                    uint64_t wait_ns) {
+  using C = DkdvCfg<D>;
+  constexpr int KID = K_BWD_DKDV_SM100;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_s - raw_s);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * KB_COUNT);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * KB_COUNT + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int jt = (int)(blockIdx.x / BH);  // key tile; low tiles carry most causal work
+  const int bh = (int)(blockIdx.x % BH);
+  const int npad = (int)((n + 127) / 128 * 128);
+  const int qstart = causal ? jt * C::BN : 0;
+  const int nq = (n - qstart + C::BQ - 1) / C::BQ;
+
+  if (threadIdx.x == 128) {
+    for (int i = 0; i < KB_COUNT; ++i)
+      mbar_init(&bar[i], (i == KB_ST_FREE || i == KB_DS_FULL) ? 128 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_kt);
+      tma_prefetch_desc(&map_v);
+      tma_prefetch_desc(&map_qt64);
+      tma_prefetch_desc(&map_do64);
+      mbar_arrive_expect_tx(&bar[KB_KV_FULL], 2 * C::KTILE);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_3d(base + C::OFF_K + c * C::KCH, &map_kt, &bar[KB_KV_FULL], c * 64, jt * C::BN,
+                    bh);
+        tma_load_3d(base + C::OFF_V + c * C::KCH, &map_v, &bar[KB_KV_FULL], c * 64, jt * C::BN,
+                    bh);
+      }
+      int issued = -1;
+      for (int it = 0; it < nq; ++it) {
+        const int s = it % C::NS;
+        if (!mbar_wait(&bar[KB_Q_EMPTY + s], ((it / C::NS) & 1) ^ 1, abort_flag, err, KID, 1,
+                       wait_ns))
+          break;
+        const int i0 = qstart + it * C::BQ;
+        uint8_t* st = base + C::OFF_ST + s * C::STAGE;
+        mbar_arrive_expect_tx(&bar[KB_Q_FULL + s], 2 * C::QTILE + 2 * C::VEC);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(st + c * C::QCH, &map_qt64, &bar[KB_Q_FULL + s], c * 64, i0, bh);
+          tma_load_3d(st + C::QTILE + c * C::QCH, &map_do64, &bar[KB_Q_FULL + s], c * 64, i0,
+                      bh);
+        }
+        bulk_load(st + 2 * C::QTILE, lse2p + (size_t)bh * npad + i0, C::VEC,
+                  &bar[KB_Q_FULL + s]);
+        bulk_load(st + 2 * C::QTILE + C::VEC, deltap + (size_t)bh * npad + i0, C::VEC,
+                  &bar[KB_Q_FULL + s]);
+        issued = it;
+      }
+      if (*abort_flag) {
+        int dummy = 0;
+        mbar_wait(&bar[KB_KV_FULL], 0, &dummy, err, KID, 20, wait_ns);
+        for (int it = max(0, issued - C::NS + 1); it <= issued; ++it)
+          mbar_wait(&bar[KB_Q_FULL + it % C::NS], (it / C::NS) & 1, &dummy, err, KID, 21,
+                    wait_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idST = idesc_bf16_f32(128, C::BQ, 0, 0);
+      constexpr uint32_t idACC = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
+      const uint32_t p_s = base_s + C::OFF_P, ds_s = base_s + C::OFF_DS;
+      bool ok = mbar_wait(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      auto issue_sdp = [&](int it) -> bool {
+        const int s = it % C::NS;
+        if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
+          return false;
+        if (!mbar_wait(&bar[KB_ST_FREE], (it & 1) ^ 1, abort_flag, err, KID, 4, wait_ns))
+          return false;
+        tc_fence_after();
+        const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
+          const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
+                      sdesc_sw128(qb + kq, 16, 1024), idST, kk > 0);
+        }
+        mma_commit(&bar[KB_S_FULL]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
+          const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
+                      sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idST, kk > 0);
+        }
+        mma_commit(&bar[KB_DP_FULL]);
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        ok = issue_sdp(0);
+      }
+      for (int it = 0; ok && it < nq; ++it) {
+        if (it + 1 < nq && !issue_sdp(it + 1)) break;
+        if (!mbar_wait(&bar[KB_DS_FULL], it & 1, abort_flag, err, KID, 5, wait_ns)) break;
+        tc_fence_after();
+        const int s = it % C::NS;
+        const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DV, sdesc_sw128(p_s + kk * 32, 16, 1024),
+                      sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idACC,
+                      (it > 0 || kk > 0));
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DK, sdesc_sw128(ds_s + kk * 32, 16, 1024),
+                      sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idACC, (it > 0 || kk > 0));
+        mma_commit(&bar[KB_PDS_FREE]);
+        mma_commit(&bar[KB_Q_EMPTY + s]);
+      }
+      if (ok) mma_commit(&bar[KB_ACC_DONE]);
+      mma_commit(&bar[KB_DRAIN]);
+      int dummy = 0;
+      mbar_wait(&bar[KB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int t = threadIdx.x;
+    const int key = jt * C::BN + t;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float scale_log2 = kLog2e / sqrtf((float)D);
+    const uint32_t p_row = base_s + C::OFF_P, ds_row = base_s + C::OFF_DS;
+    bool ok = true;
+    for (int it = 0; it < nq; ++it) {
+      const int s = it % C::NS;
+      const int i0 = qstart + it * C::BQ;
+      if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6, wait_ns) ||
+          !mbar_wait(&bar[KB_S_FULL], it & 1, abort_flag, err, KID, 7, wait_ns) ||
+          !mbar_wait(&bar[KB_DP_FULL], it & 1, abort_flag, err, KID, 8, wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[2][32], dr[2][32];
+      tmem_ld32(lane_base + C::COL_ST, sr[0]);
+      tmem_ld32(lane_base + C::COL_ST + 32, sr[1]);
+      tmem_ld32(lane_base + C::COL_DPT, dr[0]);
+      tmem_ld32(lane_base + C::COL_DPT + 32, dr[1]);
+      tmem_wait_ld(sr[0]);
+      tmem_wait_ld(sr[1]);
+      tmem_wait_ld(dr[0]);
+      tmem_wait_ld(dr[1]);
+      tc_fence_before();
+      mbar_arrive(&bar[KB_ST_FREE]);
+
+      const float4* lv = reinterpret_cast<const float4*>(base + C::OFF_ST + s * C::STAGE +
+                                                         2 * C::QTILE);
+      const float4* dvv = lv + C::BQ / 4;
+      const bool need_mask = causal && (i0 < jt * C::BN + C::BN);
+      float pv[64], dsv[64];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = lv[c4], d4 = dvv[c4];
+        const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          float p = fast_exp2(__uint_as_float(sr[c / 32][c % 32]) * scale_log2 - la[e]);
+          if (need_mask && (i0 + c < key)) p = 0.f;
+          pv[c] = p;
+          dsv[c] = p * (__uint_as_float(dr[c / 32][c % 32]) - da[e]);
+        }
+      }
+      if (it > 0 &&
+          !mbar_wait(&bar[KB_PDS_FREE], (it - 1) & 1, abort_flag, err, KID, 9, wait_ns)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        st_shared_v4(p_row + sw128_off(t, u), pack_bf16x2(pv[8 * u], pv[8 * u + 1]),
+                     pack_bf16x2(pv[8 * u + 2], pv[8 * u + 3]),
+                     pack_bf16x2(pv[8 * u + 4], pv[8 * u + 5]),
+                     pack_bf16x2(pv[8 * u + 6], pv[8 * u + 7]));
+        st_shared_v4(ds_row + sw128_off(t, u), pack_bf16x2(dsv[8 * u], dsv[8 * u + 1]),
+                     pack_bf16x2(dsv[8 * u + 2], dsv[8 * u + 3]),
+                     pack_bf16x2(dsv[8 * u + 4], dsv[8 * u + 5]),
+                     pack_bf16x2(dsv[8 * u + 6], dsv[8 * u + 7]));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[KB_DS_FULL]);
+    }
+    if (ok && mbar_wait(&bar[KB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
+      tc_fence_after();
+      const bool live = key < n;
+      // dV row
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + C::COL_DV + 32 * c, r);
+        tmem_wait_ld(r);
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)bh * n + key) * D + 32 * c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float* f = reinterpret_cast<const float*>(&r[8 * u]);
+            dst[u] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+          }
+        }
+      }
+      // dK row, its inverse rotation and the K-side torques
+      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
+      grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
+                           table + (size_t)(live ? key : 0) * (D / 2), rsqrtf((float)D),
+                           (float)key - 0.5f * (float)(n - 1), live,
+                           dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1));
+      softmax_group_sync();
+      const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
+      write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
+                               ntile64, t);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ======================================================================== dQ
+template <int D>
+struct DqCfg {
+  static constexpr int BM = 128, BK = 64, NS = 3, CH = D / 64;
+  static constexpr uint32_t QCH = 128u * 128u;  // chunk of a 128-row tile
+  static constexpr uint32_t QTILE = QCH * CH;
+  static constexpr uint32_t KCH = 64u * 128u;   // chunk of a 64-row tile
+  static constexpr uint32_t KTILE = KCH * CH;
+  static constexpr uint32_t OFF_Q = 0, OFF_DO = QTILE, OFF_ST = 2 * QTILE;
+  static constexpr uint32_t STAGE = 2 * KTILE;  // K~_j, V_j
+  static constexpr uint32_t OFF_DS = OFF_ST + NS * STAGE;  // 2 x [128 queries][64 keys]
+  static constexpr uint32_t OFF_BAR = OFF_DS + 2 * QCH;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 256;  // S, dP at +128*buffer
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
+};
+
+enum DqBar {
+  QB_Q_FULL = 0,
+  QB_KV_FULL = 1,   // +stage (3)
+  QB_KV_EMPTY = 4,  // +stage (3)
+  QB_SP_FULL = 7,   // +buffer (2)
+  QB_SP_FREE = 9,   // +buffer, 128 arrivals
+  QB_DS_FULL = 11,  // +buffer, 128 arrivals
+  QB_DS_FREE = 13,  // +buffer
+  QB_ACC_DONE = 15,
+  QB_DRAIN = 16,
+  QB_COUNT = 17
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qt,
+                  const __grid_constant__ CUtensorMap map_do,
+                  const __grid_constant__ CUtensorMap map_kt64,
+                  const __grid_constant__ CUtensorMap map_v64, const float* __restrict__ lse2p,
+                  const float* __restrict__ deltap, const float2* __restrict__ table,
+                  __nv_bfloat16* __restrict__ dq, float* __restrict__ dpart, int n, int BH,
+                  int causal, uint32_t* err, uint64_t wait_ns) {
+  using C = DqCfg<D>;
+  constexpr int KID = K_BWD_DQ_SM100;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_s - raw_s);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * QB_COUNT);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * QB_COUNT + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntq = (n + C::BM - 1) / C::BM;
+  const int qtile = ntq - 1 - (int)(blockIdx.x / BH);  // heaviest causal tiles first
+  const int bh = (int)(blockIdx.x % BH);
+  const int npad = (int)((n + 127) / 128 * 128);
+  const int kend = causal ? min(n, (qtile + 1) * C::BM) : n;
+  const int nk = (kend + C::BK - 1) / C::BK;
+
+  if (threadIdx.x == 128) {
+    for (int i = 0; i < QB_COUNT; ++i)
+      mbar_init(&bar[i], (i == QB_SP_FREE || i == QB_SP_FREE + 1 || i == QB_DS_FULL ||
+                          i == QB_DS_FULL + 1)
+                             ? 128
+                             : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_qt);
+      tma_prefetch_desc(&map_do);
+      tma_prefetch_desc(&map_kt64);
+      tma_prefetch_desc(&map_v64);
+      mbar_arrive_expect_tx(&bar[QB_Q_FULL], 2 * C::QTILE);
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_3d(base + C::OFF_Q + c * C::QCH, &map_qt, &bar[QB_Q_FULL], c * 64,
+                    qtile * C::BM, bh);
+        tma_load_3d(base + C::OFF_DO + c * C::QCH, &map_do, &bar[QB_Q_FULL], c * 64,
+                    qtile * C::BM, bh);
+      }
+      int issued = -1;
+      for (int j = 0; j < nk; ++j) {
+        const int s = j % C::NS;
+        if (!mbar_wait(&bar[QB_KV_EMPTY + s], ((j / C::NS) & 1) ^ 1, abort_flag, err, KID, 1,
+                       wait_ns))
+          break;
+        uint8_t* st = base + C::OFF_ST + s * C::STAGE;
+        mbar_arrive_expect_tx(&bar[QB_KV_FULL + s], 2 * C::KTILE);
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(st + c * C::KCH, &map_kt64, &bar[QB_KV_FULL + s], c * 64, j * C::BK, bh);
+          tma_load_3d(st + C::KTILE + c * C::KCH, &map_v64, &bar[QB_KV_FULL + s], c * 64,
+                      j * C::BK, bh);
+        }
+        issued = j;
+      }
+      if (*abort_flag) {
+        int dummy = 0;
+        mbar_wait(&bar[QB_Q_FULL], 0, &dummy, err, KID, 20, wait_ns);
+        for (int j = max(0, issued - C::NS + 1); j <= issued; ++j)
+          mbar_wait(&bar[QB_KV_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, KID, 21, wait_ns);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idSP = idesc_bf16_f32(128, C::BK, 0, 0);
+      constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_s = base_s + C::OFF_Q, do_s = base_s + C::OFF_DO;
+      const uint32_t ds_s = base_s + C::OFF_DS;
+      bool ok = mbar_wait(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      auto issue_sp = [&](int j) -> bool {
+        const int s = j % C::NS, b = j & 1;
+        if (!mbar_wait(&bar[QB_KV_FULL + s], (j / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
+          return false;
+        if (!mbar_wait(&bar[QB_SP_FREE + b], ((j >> 1) & 1) ^ 1, abort_flag, err, KID, 4,
+                       wait_ns))
+          return false;
+        tc_fence_after();
+        const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
+          const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_S + b * 128, sdesc_sw128(q_s + ka, 16, 1024),
+                      sdesc_sw128(kb + kq, 16, 1024), idSP, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
+          const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+          mma_bf16_ss(tmem + C::COL_DP + b * 128, sdesc_sw128(do_s + ka, 16, 1024),
+                      sdesc_sw128(kb + C::KTILE + kq, 16, 1024), idSP, kk > 0);
+        }
+        mma_commit(&bar[QB_SP_FULL + b]);
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        ok = issue_sp(0);
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        if (j + 1 < nk && !issue_sp(j + 1)) break;
+        const int s = j % C::NS, b = j & 1;
+        if (!mbar_wait(&bar[QB_DS_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
+          break;
+        tc_fence_after();
+        const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          mma_bf16_ss(tmem + C::COL_DQ, sdesc_sw128(ds_s + b * C::QCH + kk * 32, 16, 1024),
+                      sdesc_sw128(kb + kk * 2048, C::KCH, 1024), idDQ, (j > 0 || kk > 0));
+        mma_commit(&bar[QB_DS_FREE + b]);
+        mma_commit(&bar[QB_KV_EMPTY + s]);
+      }
+      if (ok) mma_commit(&bar[QB_ACC_DONE]);
+      mma_commit(&bar[QB_DRAIN]);
+      int dummy = 0;
+      mbar_wait(&bar[QB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int t = threadIdx.x;
+    const int row = qtile * C::BM + t;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const float scale_log2 = kLog2e / sqrtf((float)D);
+    const float lse2 = lse2p[(size_t)bh * npad + row];
+    const float dlt = deltap[(size_t)bh * npad + row];
+    bool ok = true;
+    for (int j = 0; j < nk; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&bar[QB_SP_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 6, wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[2][32], dr[2][32];
+      tmem_ld32(lane_base + C::COL_S + b * 128, sr[0]);
+      tmem_ld32(lane_base + C::COL_S + b * 128 + 32, sr[1]);
+      tmem_ld32(lane_base + C::COL_DP + b * 128, dr[0]);
+      tmem_ld32(lane_base + C::COL_DP + b * 128 + 32, dr[1]);
+      tmem_wait_ld(sr[0]);
+      tmem_wait_ld(sr[1]);
+      tmem_wait_ld(dr[0]);
+      tmem_wait_ld(dr[1]);
+      tc_fence_before();
+      mbar_arrive(&bar[QB_SP_FREE + b]);
+
+      const int key0 = j * C::BK;
+      const bool need_mask = (causal && key0 + C::BK - 1 > qtile * C::BM) || (key0 + C::BK > n);
+      float dsv[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float p = fast_exp2(__uint_as_float(sr[c / 32][c % 32]) * scale_log2 - lse2);
+        if (need_mask) {
+          const int key = key0 + c;
+          if (key >= n || (causal && key > row)) p = 0.f;
+        }
+        dsv[c] = p * (__uint_as_float(dr[c / 32][c % 32]) - dlt);
+      }
+      if (!mbar_wait(&bar[QB_DS_FREE + b], ((j >> 1) & 1) ^ 1, abort_flag, err, KID, 7,
+                     wait_ns)) {
+        ok = false;
+        break;
+      }
+      const uint32_t ds_row = base_s + C::OFF_DS + b * C::QCH;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        st_shared_v4(ds_row + sw128_off(t, u), pack_bf16x2(dsv[8 * u], dsv[8 * u + 1]),
+                     pack_bf16x2(dsv[8 * u + 2], dsv[8 * u + 3]),
+                     pack_bf16x2(dsv[8 * u + 4], dsv[8 * u + 5]),
+                     pack_bf16x2(dsv[8 * u + 6], dsv[8 * u + 7]));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bar[QB_DS_FULL + b]);
+    }
+    if (ok && mbar_wait(&bar[QB_ACC_DONE], 0, abort_flag, err, KID, 8, wait_ns)) {
+      tc_fence_after();
+      const bool live = row < n;
+      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
+      grad_row_epilogue<D>(lane_base + C::COL_DQ, base_s + C::OFF_Q, C::QCH, t,
+                           table + (size_t)(live ? row : 0) * (D / 2), rsqrtf((float)D),
+                           (float)row - 0.5f * (float)(n - 1), live,
+                           dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1));
+      softmax_group_sync();
+      const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
+      write_dalpha_partials<D>(red, dpart + ((size_t)(0 * BH + bh) * ntile64) * (D / 2), qtile,
+                               ntile64, t);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_dkdv_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
+                          const float* deltap, const float2* table, void* dk, void* dv,
+                          float* dpart, const DevCtl& ctl, cudaStream_t s) {
+  using C = DkdvCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int BH = (int)(p.B * p.H);
+  const long long ntk = (p.n + C::BN - 1) / C::BN;
+  bwd_dkdv_kernel<D><<<(unsigned)(ntk * BH), 192, C::SMEM, s>>>(
+      maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, (__nv_bfloat16*)dk,
+      (__nv_bfloat16*)dv, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
+                        const float* deltap, const float2* table, void* dq, float* dpart,
+                        const DevCtl& ctl, cudaStream_t s) {
+  using C = DqCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int BH = (int)(p.B * p.H);
+  const long long ntq = (p.n + C::BM - 1) / C::BM;
+  bwd_dq_kernel<D><<<(unsigned)(ntq * BH), 192, C::SMEM, s>>>(
+      maps.qt, maps.dO, maps.kt64, maps.v64, lse2p, deltap, table, (__nv_bfloat16*)dq, dpart,
+      (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
+                                  const float* lse2p, const float* deltap, const float2* table,
+                                  void* dk, void* dv, float* dpart, const DevCtl& ctl,
+                                  cudaStream_t s) {
+  if (p.d == 64) return launch_dkdv_d<64>(p, maps, lse2p, deltap, table, dk, dv, dpart, ctl, s);
+  return launch_dkdv_d<128>(p, maps, lse2p, deltap, table, dk, dv, dpart, ctl, s);
+}
+
+cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
+                                const float* deltap, const float2* table, void* dq, float* dpart,
+                                const DevCtl& ctl, cudaStream_t s) {
+  if (p.d == 64) return launch_dq_d<64>(p, maps, lse2p, deltap, table, dq, dpart, ctl, s);
+  return launch_dq_d<128>(p, maps, lse2p, deltap, table, dq, dpart, ctl, s);
+}
+
 }  // namespace ra

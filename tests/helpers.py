@@ -72,9 +72,29 @@ def gpu_fwd(inp, device="cuda"):
 
 
 def oracle_run(inp):
+    """Oracle results, plus `dalpha_noise`: the bf16 rounding-noise scale of dalpha.
+
+    Each weighted torque term w_p <dX~_pm, J x~_pm> of the dalpha sum is perturbed by
+    O(u) relative (u = 2^-8, bf16 unit roundoff) when x~ is rounded to bf16 for the
+    tensor cores; the perturbations have random signs, so they add in quadrature.
+    dalpha_noise = 3 u ||theta_hat * sqrt(sum of squared weighted torques)|| / ||dalpha||.
+    (A CPU model of the kernel's roundings puts the actual error at 0.14-1.7 u RSS.)
+    """
     wl = inp.wl
-    return ref.forward_backward(inp.f64("q"), inp.f64("k"), inp.f64("v"), inp.f64("e"),
-                                inp.f64("alpha"), wl.base, wl.causal)
+    q, k, v, e, al = (inp.f64(x) for x in ("q", "k", "v", "e", "alpha"))
+    o, lse = ref.forward(q, k, v, al, wl.base, wl.causal)
+    L, do = ref.loss(o, e)
+    dq, dk, dv, dalpha, extra = ref.backward(q, k, v, do, al, wl.base, wl.causal,
+                                             return_rotated=True)
+    _, th = ref.frequencies(wl.d, wl.base, al)
+    w2 = (np.arange(wl.n) - 0.5 * (wl.n - 1)) ** 2
+    rss = np.zeros(wl.d // 2)
+    for qt, kt, dqt, dkt in extra:
+        rss += w2 @ (ref.band_torque(dqt, qt) ** 2 + ref.band_torque(dkt, kt) ** 2)
+    nrm = np.linalg.norm(dalpha)
+    noise = 3 * 2.0 ** -8 * np.linalg.norm(th * np.sqrt(rss)) / nrm if nrm > 0 else 0.0
+    return dict(o=o, lse=lse, L=L, do=do, dq=dq, dk=dk, dv=dv, dalpha=dalpha,
+                dalpha_noise=float(noise))
 
 
 def oracle_fwd(inp):
@@ -84,9 +104,15 @@ def oracle_fwd(inp):
     return dict(o=o, lse=lse)
 
 
-def compare(g, r, dtype, keys=("o", "lse", "L", "dq", "dk", "dv", "dalpha")):
-    """Assert every result is inside its tolerance; return the measured errors."""
-    tol = TOL[dtype]
+def compare(g, r, dtype, keys=("o", "lse", "L", "dq", "dk", "dv", "dalpha"), small=False):
+    """Assert every result is inside its tolerance; return the measured errors.
+
+    small=True (problems far below the workload sizes, bf16 only): dalpha may also sit
+    inside the oracle's bf16 rounding-noise scale r["dalpha_noise"] (see oracle_run),
+    since with few positions the cancelling Q/K torque sums leave less signal."""
+    tol = dict(TOL[dtype])
+    if small and dtype == "bf16" and "dalpha_noise" in r:
+        tol["dalpha"] = max(tol["grad"], r["dalpha_noise"])
     errs = {}
     for key in keys:
         if key == "o":
@@ -100,7 +126,8 @@ def compare(g, r, dtype, keys=("o", "lse", "L", "dq", "dk", "dv", "dalpha")):
             assert errs[key] <= tol["L"], (key, errs[key])
         else:
             errs[key] = rel_frob(g[key], r[key])
-            assert errs[key] <= tol["grad"], (key, errs[key])
+            bound = tol.get(key, tol["grad"])
+            assert errs[key] <= bound, (key, errs[key], bound)
     return errs
 
 

@@ -169,6 +169,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     from rope_attention_fwd_b200 import binding as rb
+    from rope_attention_fwd_b200.dist import allreduce_dalpha, rank_seed
     from rope_attention_fwd_b200.inputs import make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -183,7 +184,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=dev)
     wl = workload(args.config)
-    inp = make_inputs(wl, seed=wl.seed + 7919 * rank)
+    inp = make_inputs(wl, seed=rank_seed(wl.seed, rank))
     flops_fwd, flops_bwd = wl.flops_fwd(), wl.flops_bwd()
     flops = flops_fwd + flops_bwd
 
@@ -204,8 +205,7 @@ def run_ours(args):
         rb.rope_attn_loss(o, t["e"], ws=ws, L=L, dO=dO)
         rb.rope_attn_bwd(t["q"], t["k"], t["v"], o, lse, dO, t["alpha"], wl.base, wl.causal,
                          ws=ws, dq=dq, dk=dk, dv=dvv, dalpha=dalpha)
-        if world > 1:
-            dist.all_reduce(dalpha)  # sum over every head of every rank
+        allreduce_dalpha(dalpha)  # sum over every head of every rank (no-op on one GPU)
 
     def barrier():
         if world > 1:

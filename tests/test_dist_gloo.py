@@ -1,0 +1,60 @@
+"""The multi-rank host path on CPU (gloo, world size 2): each rank draws its own batch,
+computes its dalpha (the float64 oracle stands in for the GPU kernels here), and the
+all-reduce must give the dalpha of the union of both ranks' heads."""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from rope_attention_fwd_b200.configs import Workload
+from rope_attention_fwd_b200.dist import allreduce_dalpha, rank_seed
+from rope_attention_fwd_b200.inputs import make_inputs
+
+WL = Workload("dist 1x2x24x8", 1, 2, 24, 8, "f32", True, 100.0, "normal", alpha="normal",
+              alpha_a=0.4, seed=31)
+
+
+def _dalpha(seed):
+    from oracle import rope_attn_ref as ref
+    inp = make_inputs(WL, seed=seed)
+    r = ref.forward_backward(inp.f64("q"), inp.f64("k"), inp.f64("v"), inp.f64("e"),
+                             inp.f64("alpha"), WL.base, WL.causal)
+    return r["dalpha"]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        da = torch.tensor(_dalpha(rank_seed(WL.seed, rank)), dtype=torch.float64)
+        allreduce_dalpha(da)
+        out[rank] = da.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_dalpha_allreduce_two_ranks():
+    world = 2
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    expect = sum(_dalpha(rank_seed(WL.seed, r)) for r in range(world))
+    for r in range(world):
+        np.testing.assert_allclose(res[r], expect, rtol=1e-12, atol=1e-14)
+    # the ranks' batches differ (independent heads), so each rank contributes
+    assert not np.allclose(_dalpha(rank_seed(WL.seed, 0)), _dalpha(rank_seed(WL.seed, 1)))
+
+
+def test_single_process_is_a_noop():
+    da = torch.arange(4, dtype=torch.float32)
+    assert torch.equal(allreduce_dalpha(da.clone()), da)

@@ -273,3 +273,41 @@ def test_loss_zero_when_target_is_output():
     assert r["L"] == 0.0
     for key in ("dq", "dk", "dv", "dalpha"):
         assert np.max(np.abs(r[key])) == 0.0
+
+
+# ---------------------------------------------------------------- regression fixture
+def test_oracle_regression_fixture():
+    """The oracle still produces what tests/golden/make_golden.py recorded."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "oracle_small.json")
+    g = json.load(open(path))
+    arr = lambda key: np.array(g[key], dtype=np.float64)
+    r = ref.forward_backward(arr("q"), arr("k"), arr("v"), arr("e"), arr("alpha"), g["base"],
+                             g["causal"])
+    for key in ("o", "lse", "dq", "dk", "dv", "dalpha"):
+        np.testing.assert_allclose(r[key], arr(key), rtol=1e-13, atol=1e-14)
+    assert abs(r["L"] - g["L"]) <= 1e-13 * abs(g["L"])
+
+
+# ---------------------------------------------------------------- row / column restrictions
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_and_column_restricted_backward(causal):
+    """head_backward_rows / _cols (used at full sizes on sampled rows) equal the rows of the
+    full blocked backward; Delta taken as rowsum(dO o O)."""
+    n, d = 37, 8
+    q, k, v, e, alpha, base = rand_problem(41, 1, 1, n, d, base=300.0)
+    _, th = ref.frequencies(d, base, alpha)
+    phi = ref.angles(n, th)
+    qt, kt = ref.rotate(q[0, 0], phi), ref.rotate(k[0, 0], phi)
+    o, lse = ref.head_forward(qt, kt, v[0, 0], causal)
+    do = o - e[0, 0]
+    delta = np.sum(do * o, axis=1)
+    dqt, dkt, dv = ref.head_backward(qt, kt, v[0, 0], do, causal, block=5)
+    rows = np.array([0, 3, 17, 36])
+    np.testing.assert_allclose(
+        ref.head_backward_rows(qt, kt, v[0, 0], do[rows], lse[rows], delta[rows], rows, causal),
+        dqt[rows], atol=1e-13)
+    ck, cv = ref.head_backward_cols(qt, kt, v[0, 0], do, lse, delta, rows, causal)
+    np.testing.assert_allclose(ck, dkt[rows], atol=1e-13)
+    np.testing.assert_allclose(cv, dv[rows], atol=1e-13)

@@ -107,6 +107,34 @@ ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32
 /* Static text for a status code. */
 const char* rope_attn_status_string(ra_status s);
 
+/* ---- forward without a caller workspace --------------------------------------
+ * The papers have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory at all -- a memory plan fixed before start-up, a
+ * runtime that forbids allocation after initialisation, or a host framework that owns
+ * every device byte -- and so have no workspace to hand over.
+ *
+ * Same arguments and results as rope_attn_fwd, minus ws / ws_bytes.  Its scratch (the
+ * error word, cos/sin table, Q~ and K~) lives in one static device array of
+ * RA_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  The call itself allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Limit: a problem with rope_attn_workspace_bytes(p) > RA_NOALLOC_SCRATCH_BYTES
+ *     (e.g. more than about 1.9M elements per [B,H,n,d] tensor in bf16) is rejected
+ *     with RA_ERR_UNSUPPORTED before anything is launched.
+ *   - Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture begins.  Later calls reuse the cached address.
+ *   - Sharing: every call on a device uses the same array, which keeps the last call's
+ *     contents.  Each call clears the error word and rewrites every region it reads,
+ *     but calls that overlap on the GPU (other streams, other host threads) race on
+ *     the array: issue them on one stream.
+ *   - Device-side wait timeouts are recorded in the array's own error word, which no
+ *     entry point reads back; use rope_attn_fwd with a workspace and
+ *     rope_attn_device_status when that status is needed. */
+#define RA_NOALLOC_SCRATCH_BYTES (8u << 20)
+ra_status rope_attn_fwd_noalloc(const ra_problem* p, const void* q, const void* k, const void* v,
+                                const float* alpha, void* o, float* lse, void* stream);
+
 /* ---- optional per-kernel timing (instrumentation, off by default) --------
  * While enabled, every kernel launch made by the calls above is bracketed by
  * CUDA events on the caller's stream.  rope_attn_timing_read synchronises

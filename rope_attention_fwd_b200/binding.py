@@ -51,6 +51,8 @@ def lib():
         L.rope_attn_loss.restype = ctypes.c_int
         L.rope_attn_bwd.argtypes = [P] + [vp] * 12 + [sz, vp]
         L.rope_attn_bwd.restype = ctypes.c_int
+        L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+        L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.rope_attn_device_status.restype = ctypes.c_int
         L.rope_attn_status_string.argtypes = [ctypes.c_int]
@@ -113,6 +115,19 @@ def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None):
     _check("rope_attn_fwd", lib().rope_attn_fwd(
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
         _ptr(ws), ws.numel(), _stream(q.device)))
+    return o, lse
+
+
+def rope_attn_fwd_noalloc(q, k, v, alpha, base, causal, o=None, lse=None):
+    """rope_attn_fwd without a workspace: scratch comes from the library's static
+    RA_NOALLOC_SCRATCH_BYTES device array (problems that need more are rejected)."""
+    prob = _problem_of(q, causal, base)
+    B, H, n, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check("rope_attn_fwd_noalloc", lib().rope_attn_fwd_noalloc(
+        ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
+        _stream(q.device)))
     return o, lse
 
 

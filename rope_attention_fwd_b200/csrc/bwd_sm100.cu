@@ -40,6 +40,21 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+#ifndef RA_DKDV_STAGES
+#define RA_DKDV_STAGES 3
+#endif
+#ifndef RA_BWD_PACK_ALU
+#define RA_BWD_PACK_ALU 0
+#endif
+
+__device__ __forceinline__ uint32_t pack_g(float lo, float hi) {
+#if RA_BWD_PACK_ALU
+  return pack_bf16x2_alu(lo, hi);
+#else
+  return pack_bf16x2(lo, hi);
+#endif
+}
+
 __device__ __forceinline__ void softmax_group_sync() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
@@ -105,7 +120,7 @@ __device__ __forceinline__ void write_dalpha_partials(const float* red, float* d
 // ======================================================================== dK, dV
 template <int D>
 struct DkdvCfg {
-  static constexpr int BN = 128, BQ = 64, NS = 2, CH = D / 64;
+  static constexpr int BN = 128, BQ = 64, NS = RA_DKDV_STAGES, CH = D / 64;
   static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
   static constexpr uint32_t KTILE = KCH * CH;
   static constexpr uint32_t QCH = 64u * 128u;   // chunk of a 64-row tile
@@ -124,16 +139,16 @@ struct DkdvCfg {
 
 enum DkdvBar {
   KB_KV_FULL = 0,
-  KB_Q_FULL = 1,   // +stage (2)
-  KB_Q_EMPTY = 3,  // +stage (2)
-  KB_S_FULL = 5,
-  KB_DP_FULL = 6,
-  KB_ST_FREE = 7,  // 128 arrivals
-  KB_DS_FULL = 8,  // 128 arrivals
-  KB_PDS_FREE = 9,
-  KB_ACC_DONE = 10,
-  KB_DRAIN = 11,
-  KB_COUNT = 12
+  KB_Q_FULL = 1,                        // +stage
+  KB_Q_EMPTY = 1 + RA_DKDV_STAGES,      // +stage
+  KB_S_FULL = 1 + 2 * RA_DKDV_STAGES,
+  KB_DP_FULL,
+  KB_ST_FREE,  // 128 arrivals
+  KB_DS_FULL,  // 128 arrivals
+  KB_PDS_FREE,
+  KB_ACC_DONE,
+  KB_DRAIN,
+  KB_COUNT
 };
 
 template <int D>
@@ -337,14 +352,14 @@ __global__ void __launch_bounds__(192, 1)
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        st_shared_v4(p_row + sw128_off(t, u), pack_bf16x2(pv[8 * u], pv[8 * u + 1]),
-                     pack_bf16x2(pv[8 * u + 2], pv[8 * u + 3]),
-                     pack_bf16x2(pv[8 * u + 4], pv[8 * u + 5]),
-                     pack_bf16x2(pv[8 * u + 6], pv[8 * u + 7]));
-        st_shared_v4(ds_row + sw128_off(t, u), pack_bf16x2(dsv[8 * u], dsv[8 * u + 1]),
-                     pack_bf16x2(dsv[8 * u + 2], dsv[8 * u + 3]),
-                     pack_bf16x2(dsv[8 * u + 4], dsv[8 * u + 5]),
-                     pack_bf16x2(dsv[8 * u + 6], dsv[8 * u + 7]));
+        st_shared_v4(p_row + sw128_off(t, u), pack_g(pv[8 * u], pv[8 * u + 1]),
+                     pack_g(pv[8 * u + 2], pv[8 * u + 3]),
+                     pack_g(pv[8 * u + 4], pv[8 * u + 5]),
+                     pack_g(pv[8 * u + 6], pv[8 * u + 7]));
+        st_shared_v4(ds_row + sw128_off(t, u), pack_g(dsv[8 * u], dsv[8 * u + 1]),
+                     pack_g(dsv[8 * u + 2], dsv[8 * u + 3]),
+                     pack_g(dsv[8 * u + 4], dsv[8 * u + 5]),
+                     pack_g(dsv[8 * u + 6], dsv[8 * u + 7]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -608,10 +623,10 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t ds_row = base_s + C::OFF_DS + b * C::QCH;
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        st_shared_v4(ds_row + sw128_off(t, u), pack_bf16x2(dsv[8 * u], dsv[8 * u + 1]),
-                     pack_bf16x2(dsv[8 * u + 2], dsv[8 * u + 3]),
-                     pack_bf16x2(dsv[8 * u + 4], dsv[8 * u + 5]),
-                     pack_bf16x2(dsv[8 * u + 6], dsv[8 * u + 7]));
+        st_shared_v4(ds_row + sw128_off(t, u), pack_g(dsv[8 * u], dsv[8 * u + 1]),
+                     pack_g(dsv[8 * u + 2], dsv[8 * u + 3]),
+                     pack_g(dsv[8 * u + 4], dsv[8 * u + 5]),
+                     pack_g(dsv[8 * u + 6], dsv[8 * u + 7]));
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bar[QB_DS_FULL + b]);

@@ -13,14 +13,25 @@
 //   warp  4    TMA producer: Q~ once, then K~_j / V_j into a 2-stage ring
 //   warp  5    TMEM allocator + single-thread tcgen05.mma issuer
 // TMEM (512 columns): S double buffer at columns 0 and 128, O at column 256.
-// The issuer runs one tile ahead: S_{j+1} = Q~ K~_{j+1}^T is on the tensor core
-// while the softmax warps turn S_j into P_j (bf16, written to shared memory in
-// the K-major 128B-swizzled layout the MMA reads) and rescale O; then
-// O += P_j V_j.  Every wait is bounded; an expired wait records RA_ERR_TIMEOUT
-// in the workspace error word and the CTA drains its copies and MMAs and exits.
+// Shared memory: Q~, the K~/V rings and a double-buffered P tile (bf16, K-major,
+// 128B swizzle), so P_{j+1} can be written while O += P_j V_j is still running.
+// The issuer runs one tile ahead: S_{j+1} is on the tensor core while the softmax
+// warps turn S_j into P_j.
+//
+// Online softmax with a lazy rescale: a row keeps its running max m until a tile's
+// max exceeds it by more than kRescaleTau (log2 units); until then P = 2^(s - m) may
+// reach 2^tau, which fp32 and bf16 hold exactly enough, and O and l stay consistent
+// because both are accumulated against the same m.  A rescale of O (a TMEM round trip)
+// happens only when some row of the warp needs it, which after the first tiles is rare.
+// The final O / l is identical in exact arithmetic to rescaling at every tile.
+//
+// Every wait is bounded; an expired wait records RA_ERR_TIMEOUT in the workspace error
+// word and the CTA drains its copies and MMAs and exits.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "common.h"
 #include "launch.h"
@@ -38,8 +49,9 @@ struct FwdCfg {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
-  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // [128][128] bf16 = 2 chunks
-  static constexpr uint32_t OFF_BAR = OFF_P + 2 * CHUNK;
+  static constexpr uint32_t PTILE = 2 * CHUNK;             // [128][128] bf16 = 2 chunks
+  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // 2 P buffers
+  static constexpr uint32_t OFF_BAR = OFF_P + 2 * PTILE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_O = 256;
@@ -52,11 +64,53 @@ enum FwdBar {
   B_V_FULL = 5,   // +stage
   B_V_EMPTY = 7,  // +stage
   B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer
-  B_P_FULL = 13,
-  B_O_DONE = 14,
-  B_DRAIN = 15,
-  B_COUNT = 16
+  B_S_FREE = 11,  // +buffer, 128 arrivals
+  B_P_FULL = 13,  // +buffer, 128 arrivals
+  B_P_FREE = 15,  // +buffer (PV MMA done reading it)
+  B_O_DONE = 17,
+  B_DRAIN = 18,
+  B_COUNT = 19
+};
+
+#ifndef RA_FWD_RESCALE_TAU
+#define RA_FWD_RESCALE_TAU 8.0f
+#endif
+#ifndef RA_FWD_PACK_ALU
+#define RA_FWD_PACK_ALU 0
+#endif
+#ifndef RA_FWD_POLY_EVERY
+#define RA_FWD_POLY_EVERY 0
+#endif
+constexpr float kRescaleTau = RA_FWD_RESCALE_TAU;
+
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+#if RA_FWD_PACK_ALU
+  return pack_bf16x2_alu(lo, hi);
+#else
+  return pack_bf16x2(lo, hi);
+#endif
+}
+
+template <int I>
+__device__ __forceinline__ float exp2_elem(float x) {
+#if RA_FWD_POLY_EVERY > 0
+  if constexpr (I % RA_FWD_POLY_EVERY == RA_FWD_POLY_EVERY - 1) return exp2_poly(x);
+#endif
+  return fast_exp2(x);
+}
+
+template <int I, int N>
+struct Unroll {
+  template <typename F>
+  __device__ __forceinline__ static void run(F&& f) {
+    f(std::integral_constant<int, I>{});
+    Unroll<I + 1, N>::run(f);
+  }
+};
+template <int N>
+struct Unroll<N, N> {
+  template <typename F>
+  __device__ __forceinline__ static void run(F&&) {}
 };
 
 template <int D>
@@ -84,7 +138,10 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 128) {
     for (int i = 0; i < B_COUNT; ++i)
-      mbar_init(&bar[i], (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) ? 128 : 1);
+      mbar_init(&bar[i], (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL ||
+                          i == B_P_FULL + 1)
+                             ? 128
+                             : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -175,22 +232,26 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) ok = issue_s(0);
       for (int j = 0; ok && j < nkv; ++j) {
         if (j + 1 < nkv && !issue_s(j + 1)) break;
-        const int s = j % C::NS;
-        if (!mbar_wait(&bar[B_P_FULL], j & 1, abort_flag, err, K_FWD_SM100, 6, wait_ns)) break;
+        const int s = j % C::NS, pb = j & 1;
+        if (!mbar_wait(&bar[B_P_FULL + pb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 6,
+                       wait_ns))
+          break;
         if (!mbar_wait(&bar[B_V_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 7,
                        wait_ns))
           break;
         tc_fence_after();
         const uint32_t vb = v_s + s * C::TILE;
+        const uint32_t pbase = p_s + pb * C::PTILE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint32_t poff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_O, sdesc_sw128(p_s + poff, 16, 1024),
+          mma_bf16_ss(tmem + C::COL_O, sdesc_sw128(pbase + poff, 16, 1024),
                       sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
         }
-        mma_commit(&bar[B_O_DONE]);
+        mma_commit(&bar[B_P_FREE + pb]);
         mma_commit(&bar[B_V_EMPTY + s]);
       }
+      if (ok) mma_commit(&bar[B_O_DONE]);
       // Every MMA issued above has finished once this commit arrives.
       mma_commit(&bar[B_DRAIN]);
       int dummy = 0;
@@ -202,10 +263,10 @@ __global__ void __launch_bounds__(192, 1)
     const int row = tile * C::BM + t;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    float m = -CUDART_INF_F, l = 0.f;
+    float m = -CUDART_INF_F, l = 0.f;  // running max (log2 units, scaled) and row sum
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
+      const int sb = j & 1, pb = j & 1;
       if (!mbar_wait(&bar[B_S_FULL + sb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 8,
                      wait_ns)) {
         ok = false;
@@ -228,51 +289,66 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&bar[B_S_FREE + sb]);
 
       const int key0 = j * C::BN;
-      const bool need_mask = (key0 + C::BN > n) || (causal && j == tile);
-      float mx = -CUDART_INF_F;
+      if ((key0 + C::BN > n) || (causal && j == tile)) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float v = x[i] * scale_log2;
-        if (need_mask) {
+        for (int i = 0; i < 128; ++i) {
           const int key = key0 + i;
-          if (key >= n || (causal && key > row)) v = -CUDART_INF_F;
+          if (key >= n || (causal && key > row)) x[i] = -CUDART_INF_F;
         }
-        x[i] = v;
-        mx = fmaxf(mx, v);
       }
-      const float m_new = fmaxf(m, mx);
-      const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
-      const float corr = fast_exp2(m - m_use);
-      float rs = 0.f;
+      // row max of the raw scores, 8 independent chains
+      float mp[8];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        x[i] = fast_exp2(x[i] - m_use);
-        rs += x[i];
+      for (int a = 0; a < 8; ++a) mp[a] = x[a];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], x[i]);
+      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * scale_log2;
+      // lazy rescale: move the reference max only when some row of the warp needs it
+      const bool need = mt > m + kRescaleTau;
+      const bool warp_rescale = __any_sync(0xffffffffu, need);
+      float corr = 1.f;
+      if (warp_rescale) {
+        const float m_new = fmaxf(m, mt);
+        corr = fast_exp2(m - m_new);  // 0 on the first tile (m = -inf)
+        m = m_new;
       }
-      l = l * corr + rs;
-      m = m_new;
+      const float m_use = m == -CUDART_INF_F ? 0.f : m;
+      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      Unroll<0, 128>::run([&](auto I) {
+        constexpr int i = decltype(I)::value;
+        x[i] = exp2_elem<i>(fmaf(x[i], scale_log2, -m_use));
+        sp[i & 7] += x[i];
+      });
+      l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
 
-      if (j > 0 && !mbar_wait(&bar[B_O_DONE], (j - 1) & 1, abort_flag, err, K_FWD_SM100, 9,
-                              wait_ns)) {
+      // P_j -> shared memory buffer pb once O += P_{j-2} V_{j-2} has released it
+      if (!mbar_wait(&bar[B_P_FREE + pb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 9,
+                     wait_ns)) {
         ok = false;
         break;
       }
-      // P_j -> shared memory, K-major, 128B swizzle: row t, keys 64h .. 64h+63 in chunk h.
-      const uint32_t p_row = base_s + C::OFF_P;
+      const uint32_t p_row = base_s + C::OFF_P + pb * C::PTILE;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float* src = &x[h * 64 + u * 8];
-          st_shared_v4(p_row + h * C::CHUNK + sw128_off(t, u), pack_bf16x2(src[0], src[1]),
-                       pack_bf16x2(src[2], src[3]), pack_bf16x2(src[4], src[5]),
-                       pack_bf16x2(src[6], src[7]));
+          st_shared_v4(p_row + h * C::CHUNK + sw128_off(t, u), pack_p(src[0], src[1]),
+                       pack_p(src[2], src[3]), pack_p(src[4], src[5]), pack_p(src[6], src[7]));
         }
       }
       fence_proxy_async_smem();
-      if (j > 0) {
+      if (warp_rescale && j > 0) {
+        // O must hold every P_{j'} V_{j'} with j' < j: wait for the PV MMA of step j-1
+        const int pj = j - 1;
+        if (!mbar_wait(&bar[B_P_FREE + (pj & 1)], (pj >> 1) & 1, abort_flag, err, K_FWD_SM100,
+                       11, wait_ns)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(lane_base + C::COL_O + 32 * c, r);
@@ -284,10 +360,9 @@ __global__ void __launch_bounds__(192, 1)
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&bar[B_P_FULL]);
+      mbar_arrive(&bar[B_P_FULL + pb]);
     }
-    if (ok && mbar_wait(&bar[B_O_DONE], (nkv - 1) & 1, abort_flag, err, K_FWD_SM100, 10,
-                        wait_ns)) {
+    if (ok && mbar_wait(&bar[B_O_DONE], 0, abort_flag, err, K_FWD_SM100, 10, wait_ns)) {
       tc_fence_after();
       const float inv = 1.f / l;
 #pragma unroll

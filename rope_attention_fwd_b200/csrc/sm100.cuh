@@ -18,6 +18,8 @@
 #include <cstdint>
 #include <cuda.h>
 
+#include "fastmath.cuh"
+
 namespace ra {
 
 // ------------------------------------------------------------------ error word

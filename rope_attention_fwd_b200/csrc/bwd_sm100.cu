@@ -26,8 +26,9 @@
 //         accumulated in TMEM for the whole pass.
 //   dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
 //         dP = dO V_j^T (double-buffered in TMEM), dS in bf16, dQ~ += dS K~_j.
-// Warp roles as in the forward: warps 0-3 own one TMEM lane / row each, warp 4 issues
-// TMA copies, warp 5 allocates TMEM and issues tcgen05.mma.  Every wait is bounded.
+// Warp roles: two softmax warpgroups (warps 0-7) each own every row (TMEM lane) and half
+// of the 64 streamed columns; warp 8 issues TMA copies; warp 9 allocates TMEM and issues
+// tcgen05.mma.  Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -41,11 +42,35 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 
 #ifndef RA_DKDV_STAGES
-#define RA_DKDV_STAGES 3
+#define RA_DKDV_STAGES 4
 #endif
 #ifndef RA_BWD_PACK_ALU
 #define RA_BWD_PACK_ALU 0
 #endif
+#ifndef RA_BWD_POLY_EVERY
+#define RA_BWD_POLY_EVERY 0
+#endif
+// exp2 of streamed column c: every RA_BWD_POLY_EVERY-th column on the FMA pipe (exp2_poly),
+// the others on MUFU, to split the load of the XU pipe.
+__device__ __forceinline__ float exp2_col(float x, int c) {
+#if RA_BWD_POLY_EVERY > 0
+  if (c % RA_BWD_POLY_EVERY == RA_BWD_POLY_EVERY - 1) return exp2_poly(x);
+#endif
+  return fast_exp2(x);
+}
+
+#ifndef RA_BWD_SOFT_WG
+#define RA_BWD_SOFT_WG 2
+#endif
+// Softmax warpgroups per CTA, in ping-pong: warpgroup g takes the streamed tiles
+// it = g, g + kSoftWG, ... (TMEM buffer it & 1), every row (TMEM lane) and all 64 columns
+// of its tile, so one warpgroup's TMEM round trips and barrier hand-offs overlap the
+// other's arithmetic.  The epilogue splits the D output columns between the warpgroups.
+constexpr int kSoftWG = RA_BWD_SOFT_WG;
+constexpr int kSoftThreads = 128 * kSoftWG;
+constexpr int kThreads = kSoftThreads + 64;  // + TMA producer warp + MMA warp
+constexpr int kCols = 64;                     // streamed columns per softmax thread
+constexpr int kProdWarp = 4 * kSoftWG, kMmaWarp = 4 * kSoftWG + 1;
 
 __device__ __forceinline__ uint32_t pack_g(float lo, float hi) {
 #if RA_BWD_PACK_ALU
@@ -56,7 +81,7 @@ __device__ __forceinline__ uint32_t pack_g(float lo, float hi) {
 }
 
 __device__ __forceinline__ void softmax_group_sync() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
 }
 
 // Epilogue of one gradient row held in TMEM (D fp32 columns from tmem_acc, this
@@ -69,9 +94,11 @@ __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_
                                                   const float2* __restrict__ trow, float scale,
                                                   float w, bool live,
                                                   __nv_bfloat16* __restrict__ out_row,
-                                                  float* red_row) {
+                                                  float* red_row, int half) {
+  constexpr int NC = D / 32 / kSoftWG;  // 32-column chunks of this thread
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int cc = 0; cc < NC; ++cc) {
+    const int c = half * NC + cc;
     uint32_t r[32];
     tmem_ld32(tmem_acc + 32 * c, r);
     tmem_wait_ld(r);
@@ -128,12 +155,12 @@ struct DkdvCfg {
   static constexpr uint32_t VEC = BQ * 4;
   static constexpr uint32_t STAGE = (2 * QTILE + 2 * VEC + 1023) / 1024 * 1024;
   static constexpr uint32_t OFF_K = 0, OFF_V = KTILE, OFF_ST = 2 * KTILE;
-  static constexpr uint32_t OFF_P = OFF_ST + NS * STAGE;  // P^T  [128 keys][64 queries]
-  static constexpr uint32_t OFF_DS = OFF_P + KCH;         // dS^T [128 keys][64 queries]
-  static constexpr uint32_t OFF_BAR = OFF_DS + KCH;
+  static constexpr uint32_t OFF_BAR = OFF_ST + NS * STAGE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 128, COL_DK = 128 + D;
-  static constexpr uint32_t TMEM_COLS = (128 + 2 * D) <= 256 ? 256 : 512;
+  // TMEM: two buffers of [S^T (64 fp32) | dP^T (64 fp32)] at 128 * b; P^T and dS^T are
+  // written back as bf16 over the first half of each thread's S^T / dP^T slice.
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
   static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
 };
 
@@ -141,18 +168,21 @@ enum DkdvBar {
   KB_KV_FULL = 0,
   KB_Q_FULL = 1,                        // +stage
   KB_Q_EMPTY = 1 + RA_DKDV_STAGES,      // +stage
-  KB_S_FULL = 1 + 2 * RA_DKDV_STAGES,
-  KB_DP_FULL,
-  KB_ST_FREE,  // 128 arrivals
-  KB_DS_FULL,  // 128 arrivals
-  KB_PDS_FREE,
-  KB_ACC_DONE,
+  KB_SDP_FULL = 1 + 2 * RA_DKDV_STAGES, // +buffer: S^T and dP^T of that buffer computed
+  KB_DS_FULL = KB_SDP_FULL + 2,         // +buffer: P^T, dS^T written (kSoftThreads arrivals)
+  KB_ACC_DONE = KB_DS_FULL + 2,
   KB_DRAIN,
   KB_COUNT
 };
 
+// TMEM column (relative to a buffer's S^T or dP^T base) of the bf16 pair holding streamed
+// column `c` (0..63): each softmax slice packs its kCols values at the start of its own slice.
+__device__ __forceinline__ constexpr uint32_t packed_col(int c) {
+  return (uint32_t)((c / kCols) * kCols + (c % kCols) / 2);
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap map_kt,
                     const __grid_constant__ CUtensorMap map_v,
                     const __grid_constant__ CUtensorMap map_qt64,
@@ -179,13 +209,13 @@ __global__ void __launch_bounds__(192, 1)
   const int qstart = causal ? jt * C::BN : 0;
   const int nq = (n - qstart + C::BQ - 1) / C::BQ;
 
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == kSoftThreads) {
     for (int i = 0; i < KB_COUNT; ++i)
-      mbar_init(&bar[i], (i == KB_ST_FREE || i == KB_DS_FULL) ? 128 : 1);
+      mbar_init(&bar[i], (i == KB_DS_FULL || i == KB_DS_FULL + 1) ? 128 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -194,7 +224,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&map_kt);
@@ -236,60 +266,56 @@ __global__ void __launch_bounds__(192, 1)
                     wait_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idST = idesc_bf16_f32(128, C::BQ, 0, 0);
       constexpr uint32_t idACC = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
-      const uint32_t p_s = base_s + C::OFF_P, ds_s = base_s + C::OFF_DS;
       bool ok = mbar_wait(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      // S^T / dP^T of step `it` into TMEM buffer it & 1.  That buffer last held P^T / dS^T
+      // of step it - 2, whose dV / dK MMAs were issued earlier by this thread (in order).
       auto issue_sdp = [&](int it) -> bool {
-        const int s = it % C::NS;
+        const int s = it % C::NS, b = it & 1;
         if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
           return false;
-        if (!mbar_wait(&bar[KB_ST_FREE], (it & 1) ^ 1, abort_flag, err, KID, 4, wait_ns))
-          return false;
         tc_fence_after();
         const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
+          mma_bf16_ss(tmem + b * 128 + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
                       sdesc_sw128(qb + kq, 16, 1024), idST, kk > 0);
         }
-        mma_commit(&bar[KB_S_FULL]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
+          mma_bf16_ss(tmem + b * 128 + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
                       sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idST, kk > 0);
         }
-        mma_commit(&bar[KB_DP_FULL]);
+        mma_commit(&bar[KB_SDP_FULL + b]);
         return true;
       };
-      if (ok) {
-        tc_fence_after();
-        ok = issue_sdp(0);
-      }
+      if (ok) ok = issue_sdp(0);
       for (int it = 0; ok && it < nq; ++it) {
         if (it + 1 < nq && !issue_sdp(it + 1)) break;
-        if (!mbar_wait(&bar[KB_DS_FULL], it & 1, abort_flag, err, KID, 5, wait_ns)) break;
+        const int s = it % C::NS, b = it & 1;
+        if (!mbar_wait(&bar[KB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
+          break;
         tc_fence_after();
-        const int s = it % C::NS;
         const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
+        // dV += P^T dO_i and dK~ += dS^T Q~_i with P^T, dS^T read from TMEM
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DV, sdesc_sw128(p_s + kk * 32, 16, 1024),
+          mma_bf16_ts(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
                       sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idACC,
                       (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DK, sdesc_sw128(ds_s + kk * 32, 16, 1024),
+          mma_bf16_ts(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
                       sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idACC, (it > 0 || kk > 0));
-        mma_commit(&bar[KB_PDS_FREE]);
         mma_commit(&bar[KB_Q_EMPTY + s]);
       }
       if (ok) mma_commit(&bar[KB_ACC_DONE]);
@@ -298,79 +324,71 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(&bar[KB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int t = threadIdx.x;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = threadIdx.x % 128;      // key row == TMEM lane
+    const int half = threadIdx.x / 128;   // warpgroup: takes query tiles it = half (mod kSoftWG)
+    constexpr int col0 = 0;
     const int key = jt * C::BN + t;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
-    const uint32_t p_row = base_s + C::OFF_P, ds_row = base_s + C::OFF_DS;
     bool ok = true;
-    for (int it = 0; it < nq; ++it) {
-      const int s = it % C::NS;
+    for (int it = half; it < nq; it += kSoftWG) {
+      const int s = it % C::NS, b = it & 1;
       const int i0 = qstart + it * C::BQ;
       if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6, wait_ns) ||
-          !mbar_wait(&bar[KB_S_FULL], it & 1, abort_flag, err, KID, 7, wait_ns) ||
-          !mbar_wait(&bar[KB_DP_FULL], it & 1, abort_flag, err, KID, 8, wait_ns)) {
+          !mbar_wait(&bar[KB_SDP_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 7, wait_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[2][32], dr[2][32];
-      tmem_ld32(lane_base + C::COL_ST, sr[0]);
-      tmem_ld32(lane_base + C::COL_ST + 32, sr[1]);
-      tmem_ld32(lane_base + C::COL_DPT, dr[0]);
-      tmem_ld32(lane_base + C::COL_DPT + 32, dr[1]);
-      tmem_wait_ld(sr[0]);
-      tmem_wait_ld(sr[1]);
-      tmem_wait_ld(dr[0]);
-      tmem_wait_ld(dr[1]);
-      tc_fence_before();
-      mbar_arrive(&bar[KB_ST_FREE]);
-
+      const uint32_t st_base = lane_base + b * 128 + C::COL_ST;
+      const uint32_t dpt_base = lane_base + b * 128 + C::COL_DPT;
       const float4* lv = reinterpret_cast<const float4*>(base + C::OFF_ST + s * C::STAGE +
                                                          2 * C::QTILE);
       const float4* dvv = lv + C::BQ / 4;
       const bool need_mask = causal && (i0 < jt * C::BN + C::BN);
-      float pv[64], dsv[64];
+      // 32 columns at a time: load S^T, dP^T; P^T, dS^T back as bf16 over the first 16
+      // columns of each half (packed_col order), all before this warpgroup's arrival
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l4 = lv[c4], d4 = dvv[c4];
-        const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(st_base + 32 * h, sr);
+        tmem_ld32(dpt_base + 32 * h, dr);
+        tmem_wait_ld(sr);
+        tmem_wait_ld(dr);
+        uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;
-          float p = fast_exp2(__uint_as_float(sr[c / 32][c % 32]) * scale_log2 - la[e]);
-          if (need_mask && (i0 + c < key)) p = 0.f;
-          pv[c] = p;
-          dsv[c] = p * (__uint_as_float(dr[c / 32][c % 32]) - da[e]);
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = lv[8 * h + c4], d4 = dvv[8 * h + c4];
+          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;  // column within this half
+            float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - la[e], 32 * h + c);
+            if (need_mask && (i0 + 32 * h + c < key)) p = 0.f;
+            pv[e] = p;
+            dsv[e] = p * (__uint_as_float(dr[c]) - da[e]);
+          }
+          pw[2 * c4] = pack_g(pv[0], pv[1]);
+          pw[2 * c4 + 1] = pack_g(pv[2], pv[3]);
+          dw[2 * c4] = pack_g(dsv[0], dsv[1]);
+          dw[2 * c4 + 1] = pack_g(dsv[2], dsv[3]);
         }
+        tmem_st16(st_base + packed_col(32 * h), pw);
+        tmem_st16(dpt_base + packed_col(32 * h), dw);
       }
-      if (it > 0 &&
-          !mbar_wait(&bar[KB_PDS_FREE], (it - 1) & 1, abort_flag, err, KID, 9, wait_ns)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        st_shared_v4(p_row + sw128_off(t, u), pack_g(pv[8 * u], pv[8 * u + 1]),
-                     pack_g(pv[8 * u + 2], pv[8 * u + 3]),
-                     pack_g(pv[8 * u + 4], pv[8 * u + 5]),
-                     pack_g(pv[8 * u + 6], pv[8 * u + 7]));
-        st_shared_v4(ds_row + sw128_off(t, u), pack_g(dsv[8 * u], dsv[8 * u + 1]),
-                     pack_g(dsv[8 * u + 2], dsv[8 * u + 3]),
-                     pack_g(dsv[8 * u + 4], dsv[8 * u + 5]),
-                     pack_g(dsv[8 * u + 6], dsv[8 * u + 7]));
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar[KB_DS_FULL]);
+      mbar_arrive(&bar[KB_DS_FULL + b]);
     }
     if (ok && mbar_wait(&bar[KB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
       tc_fence_after();
       const bool live = key < n;
-      // dV row
+      // dV row (this thread's D / kSoftWG columns)
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int cc = 0; cc < D / 32 / kSoftWG; ++cc) {
+        const int c = half * (D / 32 / kSoftWG) + cc;
         uint32_t r[32];
         tmem_ld32(lane_base + C::COL_DV + 32 * c, r);
         tmem_wait_ld(r);
@@ -389,55 +407,60 @@ __global__ void __launch_bounds__(192, 1)
       grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
                            table + (size_t)(live ? key : 0) * (D / 2), rsqrtf((float)D),
                            (float)key - 0.5f * (float)(n - 1), live,
-                           dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1));
+                           dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
+                           half);
       softmax_group_sync();
       const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
-                               ntile64, t);
+      if (threadIdx.x < 128)
+        write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
+                                 ntile64, t);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
 // ======================================================================== dQ
+#ifndef RA_DQ_STAGES
+#define RA_DQ_STAGES 4
+#endif
+
 template <int D>
 struct DqCfg {
-  static constexpr int BM = 128, BK = 64, NS = 3, CH = D / 64;
+  static constexpr int BM = 128, BK = 64, NS = RA_DQ_STAGES, CH = D / 64;
   static constexpr uint32_t QCH = 128u * 128u;  // chunk of a 128-row tile
   static constexpr uint32_t QTILE = QCH * CH;
   static constexpr uint32_t KCH = 64u * 128u;   // chunk of a 64-row tile
   static constexpr uint32_t KTILE = KCH * CH;
   static constexpr uint32_t OFF_Q = 0, OFF_DO = QTILE, OFF_ST = 2 * QTILE;
   static constexpr uint32_t STAGE = 2 * KTILE;  // K~_j, V_j
-  static constexpr uint32_t OFF_DS = OFF_ST + NS * STAGE;  // 2 x [128 queries][64 keys]
-  static constexpr uint32_t OFF_BAR = OFF_DS + 2 * QCH;
+  static constexpr uint32_t OFF_BAR = OFF_ST + NS * STAGE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 256;  // S, dP at +128*buffer
+  // TMEM: two buffers of [S (64 fp32) | dP (64 fp32)] at 128 * b, dS written back as bf16
+  // over the start of each thread's S slice; dQ~ accumulator at 256.
+  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
 };
 
 enum DqBar {
   QB_Q_FULL = 0,
-  QB_KV_FULL = 1,   // +stage (3)
-  QB_KV_EMPTY = 4,  // +stage (3)
-  QB_SP_FULL = 7,   // +buffer (2)
-  QB_SP_FREE = 9,   // +buffer, 128 arrivals
-  QB_DS_FULL = 11,  // +buffer, 128 arrivals
-  QB_DS_FREE = 13,  // +buffer
-  QB_ACC_DONE = 15,
-  QB_DRAIN = 16,
-  QB_COUNT = 17
+  QB_KV_FULL = 1,                      // +stage
+  QB_KV_EMPTY = 1 + RA_DQ_STAGES,      // +stage
+  QB_SP_FULL = 1 + 2 * RA_DQ_STAGES,   // +buffer
+  QB_DS_FULL = QB_SP_FULL + 2,         // +buffer, kSoftThreads arrivals
+  QB_ACC_DONE = QB_DS_FULL + 2,
+  QB_DRAIN,
+  QB_COUNT
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap map_qt,
                   const __grid_constant__ CUtensorMap map_do,
                   const __grid_constant__ CUtensorMap map_kt64,
@@ -464,16 +487,13 @@ __global__ void __launch_bounds__(192, 1)
   const int kend = causal ? min(n, (qtile + 1) * C::BM) : n;
   const int nk = (kend + C::BK - 1) / C::BK;
 
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == kSoftThreads) {
     for (int i = 0; i < QB_COUNT; ++i)
-      mbar_init(&bar[i], (i == QB_SP_FREE || i == QB_SP_FREE + 1 || i == QB_DS_FULL ||
-                          i == QB_DS_FULL + 1)
-                             ? 128
-                             : 1);
+      mbar_init(&bar[i], (i == QB_DS_FULL || i == QB_DS_FULL + 1) ? 128 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -482,7 +502,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&map_qt);
@@ -518,20 +538,18 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait(&bar[QB_KV_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, KID, 21, wait_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idSP = idesc_bf16_f32(128, C::BK, 0, 0);
       constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_s = base_s + C::OFF_Q, do_s = base_s + C::OFF_DO;
-      const uint32_t ds_s = base_s + C::OFF_DS;
       bool ok = mbar_wait(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      // S / dP of key tile j into TMEM buffer j & 1, which last held dS of tile j - 2;
+      // the dQ MMA that read it was issued earlier by this thread (in-order execution).
       auto issue_sp = [&](int j) -> bool {
         const int s = j % C::NS, b = j & 1;
         if (!mbar_wait(&bar[QB_KV_FULL + s], (j / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
-          return false;
-        if (!mbar_wait(&bar[QB_SP_FREE + b], ((j >> 1) & 1) ^ 1, abort_flag, err, KID, 4,
-                       wait_ns))
           return false;
         tc_fence_after();
         const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
@@ -552,10 +570,7 @@ __global__ void __launch_bounds__(192, 1)
         mma_commit(&bar[QB_SP_FULL + b]);
         return true;
       };
-      if (ok) {
-        tc_fence_after();
-        ok = issue_sp(0);
-      }
+      if (ok) ok = issue_sp(0);
       for (int j = 0; ok && j < nk; ++j) {
         if (j + 1 < nk && !issue_sp(j + 1)) break;
         const int s = j % C::NS, b = j & 1;
@@ -563,11 +578,11 @@ __global__ void __launch_bounds__(192, 1)
           break;
         tc_fence_after();
         const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
+        // dQ~ += dS K~_j with dS read from TMEM
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_bf16_ss(tmem + C::COL_DQ, sdesc_sw128(ds_s + b * C::QCH + kk * 32, 16, 1024),
+          mma_bf16_ts(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
                       sdesc_sw128(kb + kk * 2048, C::KCH, 1024), idDQ, (j > 0 || kk > 0));
-        mma_commit(&bar[QB_DS_FREE + b]);
         mma_commit(&bar[QB_KV_EMPTY + s]);
       }
       if (ok) mma_commit(&bar[QB_ACC_DONE]);
@@ -576,58 +591,53 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(&bar[QB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int t = threadIdx.x;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = threadIdx.x % 128;      // query row == TMEM lane
+    const int half = threadIdx.x / 128;   // warpgroup: takes key tiles j = half (mod kSoftWG)
+    constexpr int col0 = 0;
     const int row = qtile * C::BM + t;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
     const float lse2 = lse2p[(size_t)bh * npad + row];
     const float dlt = deltap[(size_t)bh * npad + row];
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = half; j < nk; j += kSoftWG) {
       const int b = j & 1;
       if (!mbar_wait(&bar[QB_SP_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 6, wait_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[2][32], dr[2][32];
-      tmem_ld32(lane_base + C::COL_S + b * 128, sr[0]);
-      tmem_ld32(lane_base + C::COL_S + b * 128 + 32, sr[1]);
-      tmem_ld32(lane_base + C::COL_DP + b * 128, dr[0]);
-      tmem_ld32(lane_base + C::COL_DP + b * 128 + 32, dr[1]);
-      tmem_wait_ld(sr[0]);
-      tmem_wait_ld(sr[1]);
-      tmem_wait_ld(dr[0]);
-      tmem_wait_ld(dr[1]);
-      tc_fence_before();
-      mbar_arrive(&bar[QB_SP_FREE + b]);
-
+      const uint32_t s_base = lane_base + C::COL_S + b * 128;
+      const uint32_t dp_base = lane_base + C::COL_DP + b * 128;
       const int key0 = j * C::BK;
       const bool need_mask = (causal && key0 + C::BK - 1 > qtile * C::BM) || (key0 + C::BK > n);
-      float dsv[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float p = fast_exp2(__uint_as_float(sr[c / 32][c % 32]) * scale_log2 - lse2);
-        if (need_mask) {
-          const int key = key0 + c;
-          if (key >= n || (causal && key > row)) p = 0.f;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(s_base + 32 * h, sr);
+        tmem_ld32(dp_base + 32 * h, dr);
+        tmem_wait_ld(sr);
+        tmem_wait_ld(dr);
+        uint32_t dw[16];
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) {
+          float dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = 2 * c2 + e;  // column within this half
+            float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - lse2, 32 * h + c);
+            if (need_mask) {
+              const int key = key0 + 32 * h + c;
+              if (key >= n || (causal && key > row)) p = 0.f;
+            }
+            dsv[e] = p * (__uint_as_float(dr[c]) - dlt);
+          }
+          dw[c2] = pack_g(dsv[0], dsv[1]);
         }
-        dsv[c] = p * (__uint_as_float(dr[c / 32][c % 32]) - dlt);
+        tmem_st16(s_base + packed_col(32 * h), dw);
       }
-      if (!mbar_wait(&bar[QB_DS_FREE + b], ((j >> 1) & 1) ^ 1, abort_flag, err, KID, 7,
-                     wait_ns)) {
-        ok = false;
-        break;
-      }
-      const uint32_t ds_row = base_s + C::OFF_DS + b * C::QCH;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        st_shared_v4(ds_row + sw128_off(t, u), pack_g(dsv[8 * u], dsv[8 * u + 1]),
-                     pack_g(dsv[8 * u + 2], dsv[8 * u + 3]),
-                     pack_g(dsv[8 * u + 4], dsv[8 * u + 5]),
-                     pack_g(dsv[8 * u + 6], dsv[8 * u + 7]));
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar[QB_DS_FULL + b]);
     }
@@ -638,17 +648,19 @@ __global__ void __launch_bounds__(192, 1)
       grad_row_epilogue<D>(lane_base + C::COL_DQ, base_s + C::OFF_Q, C::QCH, t,
                            table + (size_t)(live ? row : 0) * (D / 2), rsqrtf((float)D),
                            (float)row - 0.5f * (float)(n - 1), live,
-                           dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1));
+                           dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1),
+                           half);
       softmax_group_sync();
       const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      write_dalpha_partials<D>(red, dpart + ((size_t)(0 * BH + bh) * ntile64) * (D / 2), qtile,
-                               ntile64, t);
+      if (threadIdx.x < 128)
+        write_dalpha_partials<D>(red, dpart + ((size_t)(0 * BH + bh) * ntile64) * (D / 2),
+                                 qtile, ntile64, t);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -664,7 +676,7 @@ cudaError_t launch_dkdv_d(const ra_problem& p, const Sm100Maps& maps, const floa
   if (e != cudaSuccess) return e;
   const int BH = (int)(p.B * p.H);
   const long long ntk = (p.n + C::BN - 1) / C::BN;
-  bwd_dkdv_kernel<D><<<(unsigned)(ntk * BH), 192, C::SMEM, s>>>(
+  bwd_dkdv_kernel<D><<<(unsigned)(ntk * BH), kThreads, C::SMEM, s>>>(
       maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, (__nv_bfloat16*)dk,
       (__nv_bfloat16*)dv, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
   return cudaGetLastError();
@@ -680,7 +692,7 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
   if (e != cudaSuccess) return e;
   const int BH = (int)(p.B * p.H);
   const long long ntq = (p.n + C::BM - 1) / C::BM;
-  bwd_dq_kernel<D><<<(unsigned)(ntq * BH), 192, C::SMEM, s>>>(
+  bwd_dq_kernel<D><<<(unsigned)(ntq * BH), kThreads, C::SMEM, s>>>(
       maps.qt, maps.dO, maps.kt64, maps.v64, lse2p, deltap, table, (__nv_bfloat16*)dq, dpart,
       (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
   return cudaGetLastError();

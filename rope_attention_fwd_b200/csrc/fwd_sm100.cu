@@ -40,9 +40,14 @@
 namespace ra {
 namespace {
 
+#ifndef RA_FWD_P_TMEM
+#define RA_FWD_P_TMEM 1
+#endif
+
 template <int D>
 struct FwdCfg {
-  static constexpr int BM = 128, BN = 128, NS = 2;
+  // P in TMEM frees the shared-memory P buffers for a third K~/V stage.
+  static constexpr int BM = 128, BN = 128, NS = RA_FWD_P_TMEM ? 3 : 2;
   static constexpr int CH = D / 64;                       // 64-column chunks per row
   static constexpr uint32_t CHUNK = 128u * 128u;          // [128 rows][128 B]
   static constexpr uint32_t TILE = CHUNK * CH;            // [128][D] bf16
@@ -50,8 +55,8 @@ struct FwdCfg {
   static constexpr uint32_t OFF_K = OFF_Q + TILE;
   static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
   static constexpr uint32_t PTILE = 2 * CHUNK;             // [128][128] bf16 = 2 chunks
-  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // 2 P buffers
-  static constexpr uint32_t OFF_BAR = OFF_P + 2 * PTILE;
+  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // 2 P buffers (P in smem only)
+  static constexpr uint32_t OFF_BAR = OFF_P + (RA_FWD_P_TMEM ? 0 : 2 * PTILE);
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_O = 256;
@@ -59,17 +64,17 @@ struct FwdCfg {
 
 enum FwdBar {
   B_Q_FULL = 0,
-  B_K_FULL = 1,   // +stage
-  B_K_EMPTY = 3,  // +stage
-  B_V_FULL = 5,   // +stage
-  B_V_EMPTY = 7,  // +stage
-  B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer, 128 arrivals
-  B_P_FULL = 13,  // +buffer, 128 arrivals
-  B_P_FREE = 15,  // +buffer (PV MMA done reading it)
-  B_O_DONE = 17,
-  B_DRAIN = 18,
-  B_COUNT = 19
+  B_K_FULL = 1,   // +stage (3)
+  B_K_EMPTY = 4,  // +stage (3)
+  B_V_FULL = 7,   // +stage (3)
+  B_V_EMPTY = 10, // +stage (3)
+  B_S_FULL = 13,  // +buffer
+  B_S_FREE = 15,  // +buffer, 128 arrivals
+  B_P_FULL = 17,  // +buffer, 128 arrivals
+  B_P_FREE = 19,  // +buffer: the PV MMA of that buffer's P has completed
+  B_O_DONE = 21,
+  B_DRAIN = 22,
+  B_COUNT = 23
 };
 
 #ifndef RA_FWD_RESCALE_TAU
@@ -241,6 +246,15 @@ __global__ void __launch_bounds__(192, 1)
           break;
         tc_fence_after();
         const uint32_t vb = v_s + s * C::TILE;
+#if RA_FWD_P_TMEM
+        // P_j (bf16, two per column) sits over S_j in TMEM buffer pb; the S MMA that next
+        // overwrites that buffer is issued after this one, and tcgen05.mma ops from one
+        // thread execute in issue order.
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_bf16_ts(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
+                      sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
+#else
         const uint32_t pbase = p_s + pb * C::PTILE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
@@ -248,6 +262,7 @@ __global__ void __launch_bounds__(192, 1)
           mma_bf16_ss(tmem + C::COL_O, sdesc_sw128(pbase + poff, 16, 1024),
                       sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
         }
+#endif
         mma_commit(&bar[B_P_FREE + pb]);
         mma_commit(&bar[B_V_EMPTY + s]);
       }
@@ -322,6 +337,18 @@ __global__ void __launch_bounds__(192, 1)
       });
       l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
 
+#if RA_FWD_P_TMEM
+      // P_j -> TMEM over S_j (this thread's lane, 64 columns of bf16 pairs).  The PV MMA
+      // that read this buffer two tiles ago completed before S_j did.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = pack_p(x[64 * h + 2 * i], x[64 * h + 2 * i + 1]);
+        tmem_st32(lane_base + C::COL_S + sb * 128 + 32 * h, w);
+      }
+      tmem_wait_st();
+#else
       // P_j -> shared memory buffer pb once O += P_{j-2} V_{j-2} has released it
       if (!mbar_wait(&bar[B_P_FREE + pb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 9,
                      wait_ns)) {
@@ -339,6 +366,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       fence_proxy_async_smem();
+#endif
       if (warp_rescale && j > 0) {
         // O must hold every P_{j'} V_{j'} with j' < j: wait for the PV MMA of step j-1
         const int pj = j - 1;

@@ -42,6 +42,13 @@
  *     rope_attn_device_status().  No entry point aborts or traps.
  *   - Supported: fp32 with even d, 2 <= d <= 128 (CUDA-core path); bf16 with
  *     d in {64, 128} (tcgen05 tensor-core path); n >= 1; B, H >= 1.
+ *   - Precision of the bf16 path: the rotated Q~, K~ feed the score products
+ *     S = Q~ K~^T as fp16 (11-bit significand, 8x finer than bf16: sharp softmaxes
+ *     amplify score rounding), P, V and dO stay bf16, dS is fp16 with a power-of-two
+ *     scale derived on the device from max_i |dO_i| * max_j |v_j|; every product
+ *     accumulates in fp32.  Rotated entries must stay within fp16 range
+ *     (|q|, |k| below about 46000); a larger one is clamped and reported as
+ *     RA_ERR_RANGE by rope_attn_device_status.
  */
 #ifndef ROPE_ATTN_H
 #define ROPE_ATTN_H
@@ -59,7 +66,9 @@ typedef enum {
     RA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement       */
     RA_ERR_WORKSPACE = 3,     /* ws null, misaligned or smaller than required      */
     RA_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed       */
-    RA_ERR_TIMEOUT = 5        /* a device-side wait expired (see device_status)    */
+    RA_ERR_TIMEOUT = 5,       /* a device-side wait expired (see device_status)    */
+    RA_ERR_RANGE = 6          /* an input exceeds the fp16 range of the bf16 path's
+                                 score operands (see device_status)                */
 } ra_status;
 
 typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
@@ -99,9 +108,10 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
                         void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the device error word in ws.
- * Returns RA_OK, or RA_ERR_TIMEOUT if a kernel gave up on a wait since the last
- * call (kernel id / barrier id / block id are written to info[0..2] when info
- * is non-null). */
+ * Returns RA_OK; RA_ERR_TIMEOUT if a kernel gave up on a wait during the most recent
+ * call on ws (kernel id / wait site / block id are written to info[0..2] when info is
+ * non-null); or RA_ERR_RANGE if a rotated query or key entry exceeded the fp16 range
+ * of the bf16 path's score operands. */
 ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32_t info[3]);
 
 /* Static text for a status code. */

@@ -128,15 +128,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [BH][n][d] viewed as (x = d, y = n, z = BH); box = 64 columns x `rows` rows.
-bool make_map(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows) {
+// 16-bit [BH][n][d] tensor (bf16 inputs, or the fp16 rotated Q~ / K~ when fp16 is set)
+// viewed as (x = d, y = n, z = BH); box = 64 columns x `rows` rows.
+bool make_map(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows,
+              bool fp16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)p.d, (cuuint64_t)p.n, (cuuint64_t)(p.B * p.H)};
   const cuuint64_t strides[2] = {(cuuint64_t)p.d * 2, (cuuint64_t)p.n * p.d * 2};
   const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  return fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -148,7 +151,7 @@ ra_status prepare(const ra_problem* p, const void* q, const void* k, const float
   RA_LAUNCH(K_TABLE, s, launch_table(*p, alpha, at<float2>(ws, L.table), s));
   RA_LAUNCH(K_ROTATE, s,
             launch_rotate(*p, q, k, at<void>(ws, L.qt), at<void>(ws, L.kt),
-                          at<float2>(ws, L.table), s));
+                          at<float2>(ws, L.table), at<uint32_t>(ws, L.err), s));
   return RA_OK;
 }
 
@@ -169,6 +172,7 @@ const char* rope_attn_status_string(ra_status s) {
     case RA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case RA_ERR_CUDA: return "CUDA error";
     case RA_ERR_TIMEOUT: return "device-side wait timed out";
+    case RA_ERR_RANGE: return "input entry beyond the fp16 range of the score operands";
   }
   return "unknown status";
 }
@@ -193,8 +197,8 @@ ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const
   }
   Sm100Maps maps;
   std::memset(&maps, 0, sizeof(maps));
-  if (!make_map(&maps.qt, at<void>(ws, L.qt), *p, 128) ||
-      !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128) || !make_map(&maps.v, v, *p, 128))
+  if (!make_map(&maps.qt, at<void>(ws, L.qt), *p, 128, true) ||
+      !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128, true) || !make_map(&maps.v, v, *p, 128))
     return RA_ERR_CUDA;
   DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), starve_block()};
   RA_LAUNCH(K_FWD_SM100, s, launch_fwd_sm100(*p, maps, o, lse, ctl, s));
@@ -246,21 +250,23 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
                                 (float*)dq, dpart, s));
   } else {
     float* lse2 = at<float>(ws, L.lse2);
-    RA_LAUNCH(K_BWD_DELTA, s, launch_bwd_pre(*p, o, dO, lse, delta, lse2, s));
+    uint32_t* stats = at<uint32_t>(ws, L.err) + 8;  // zeroed with the error word in prepare()
+    RA_LAUNCH(K_BWD_DELTA, s, launch_bwd_pre(*p, o, dO, lse, delta, lse2, stats, s));
+    RA_LAUNCH(K_BWD_DELTA, s, launch_vnorm_max(*p, v, stats + 1, s));
     Sm100Maps maps;
     std::memset(&maps, 0, sizeof(maps));
     void* qt = at<void>(ws, L.qt);
     void* kt = at<void>(ws, L.kt);
-    if (!make_map(&maps.qt, qt, *p, 128) || !make_map(&maps.kt, kt, *p, 128) ||
+    if (!make_map(&maps.qt, qt, *p, 128, true) || !make_map(&maps.kt, kt, *p, 128, true) ||
         !make_map(&maps.v, v, *p, 128) || !make_map(&maps.dO, dO, *p, 128) ||
-        !make_map(&maps.qt64, qt, *p, 64) || !make_map(&maps.kt64, kt, *p, 64) ||
+        !make_map(&maps.qt64, qt, *p, 64, true) || !make_map(&maps.kt64, kt, *p, 64, true) ||
         !make_map(&maps.v64, v, *p, 64) || !make_map(&maps.dO64, dO, *p, 64))
       return RA_ERR_CUDA;
     DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
     RA_LAUNCH(K_BWD_DKDV_SM100, s,
-              launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, dk, dv, dpart, ctl, s));
+              launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl, s));
     RA_LAUNCH(K_BWD_DQ_SM100, s,
-              launch_bwd_dq_sm100(*p, maps, lse2, delta, table, dq, dpart, ctl, s));
+              launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
   }
   RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;
@@ -281,7 +287,8 @@ ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32
     info[1] = (int32_t)word[2];
     info[2] = (int32_t)word[3];
   }
-  return word[0] == 0 ? RA_OK : RA_ERR_TIMEOUT;
+  if (word[0] == 0) return RA_OK;
+  return word[0] == (uint32_t)RA_ERR_RANGE ? RA_ERR_RANGE : RA_ERR_TIMEOUT;
 }
 
 void rope_attn_timing_enable(int on) {

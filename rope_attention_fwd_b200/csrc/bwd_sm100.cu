@@ -12,11 +12,20 @@
 // Q-side and K-side torques of one head sum to zero, because rotating every query and
 // key by one common angle leaves every score unchanged.
 //
-// The torque uses the same bf16 x~ the MMAs consumed (read back from shared memory).
-// The gradients are those of the function evaluated at those bf16 operands, and with
-// the same x~ in the torque the Q/K cancellation above stays exact for that function.
+// Operand types: S = Q~ K~^T from fp16 Q~, K~ (the rotation kernel writes them in fp16:
+// a sharp softmax amplifies score rounding, and fp16 rounds 8x finer than bf16); dP from
+// bf16 dO, V; P (for dV) in bf16; dS in fp16, because its MMAs pair it with the fp16
+// Q~ / K~.  dS is multiplied by a power of two s before the conversion so that it sits
+// well inside the fp16 range: |dS_ij| <= P_ij |dO_i| (|v_j| + max_j |v_j|) <= 2 D V with
+// D = max_i |dO_i|, V = max_j |v_j| (measured on the device), s = 2^floor(log2(2^14 / 2DV));
+// the epilogues divide s back out.
+//
+// The torque uses the same fp16 x~ the MMAs consumed (read back from shared memory).
+// The gradients are those of the function evaluated at those operands, and with the
+// same x~ in the torque the Q/K cancellation above stays exact for that function.
 // Recomputing x~ in fp32 for the torque breaks it: on the 4x16x2048x64 causal workload
-// a CPU model of the roundings puts the dalpha error at 1.0e-2 that way, 3.8e-3 this way.
+// a CPU model of the roundings (bf16 operands) puts the dalpha error at 1.0e-2 that way,
+// 3.8e-3 this way.
 //
 // Two kernels, no atomics (deterministic):
 //   dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
@@ -30,6 +39,7 @@
 // of the 64 streamed columns; warp 8 issues TMA copies; warp 9 allocates TMEM and issues
 // tcgen05.mma.  Every wait is bounded.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.h"
@@ -84,10 +94,19 @@ __device__ __forceinline__ void softmax_group_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
 }
 
+// Power-of-two scale for dS in fp16 from stats = {max_i |dO_i|, max_j |v_j|} (fp32 bits):
+// 2 * D * V * s <= 2^14, with s in [2^-60, 2^60] (s = 1 when dO or V is all zero).
+__device__ __forceinline__ float ds_scale(const uint32_t* __restrict__ stats) {
+  const float bound = 2.f * __uint_as_float(stats[0]) * __uint_as_float(stats[1]);
+  if (!(bound > 0.f) || !(bound < 3.0e38f)) return 1.f;
+  const float e = fminf(fmaxf(floorf(log2f(16384.f / bound)), -60.f), 60.f);
+  return exp2f(e);
+}
+
 // Epilogue of one gradient row held in TMEM (D fp32 columns from tmem_acc, this
 // thread's lane): g = acc * scale is dX~ of position `pos`; writes R(-pos theta_hat) g as
 // bf16 to out_row (when live) and the band torques w * (g1 x0 - g0 x1) to red_row, where
-// x~ is row t of the 128B-swizzled bf16 tile at x_tile_s (chunk stride x_chunk).
+// x~ is row t of the 128B-swizzled fp16 tile at x_tile_s (chunk stride x_chunk).
 template <int D>
 __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_tile_s,
                                                   uint32_t x_chunk, int t,
@@ -114,7 +133,7 @@ __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_
     for (int k = 0; k < 16; ++k) {
       const float g0 = __uint_as_float(r[2 * k]) * scale;
       const float g1 = __uint_as_float(r[2 * k + 1]) * scale;
-      const __nv_bfloat162 xp = *reinterpret_cast<const __nv_bfloat162*>(&xw[k]);
+      const __half2 xp = *reinterpret_cast<const __half2*>(&xw[k]);
       const float x0 = __low2float(xp), x1 = __high2float(xp);
       const float2 cs = live ? trow[16 * c + k] : make_float2(1.f, 0.f);
       ow[k] = pack_bf16x2(cs.x * g0 + cs.y * g1, cs.x * g1 - cs.y * g0);
@@ -188,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap map_qt64,
                     const __grid_constant__ CUtensorMap map_do64, const float* __restrict__ lse2p,
                     const float* __restrict__ deltap, const float2* __restrict__ table,
-                    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                    const uint32_t* __restrict__ stats, __nv_bfloat16* __restrict__ dk,
+                    __nv_bfloat16* __restrict__ dv,
                     float* __restrict__ dpart, int n, int BH, int causal, uint32_t* err,
                     uint64_t wait_ns) {
   using C = DkdvCfg<D>;
@@ -269,8 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idST = idesc_bf16_f32(128, C::BQ, 0, 0);
-      constexpr uint32_t idACC = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idST = idesc_f16_f32(128, C::BQ, 0, 0);   // fp16 K~ Q~^T
+      constexpr uint32_t idDPT = idesc_bf16_f32(128, C::BQ, 0, 0);  // bf16 V dO^T
+      constexpr uint32_t idDV = idesc_bf16_f32(128, D, 0, 1);       // bf16 P^T dO
+      constexpr uint32_t idDK = idesc_f16_f32(128, D, 0, 1);        // fp16 dS^T Q~
       const uint32_t k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
       bool ok = mbar_wait(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
       // S^T / dP^T of step `it` into TMEM buffer it & 1.  That buffer last held P^T / dS^T
@@ -293,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
           mma_bf16_ss(tmem + b * 128 + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
-                      sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idST, kk > 0);
+                      sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idDPT, kk > 0);
         }
         mma_commit(&bar[KB_SDP_FULL + b]);
         return true;
@@ -310,12 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           mma_bf16_ts(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
-                      sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idACC,
+                      sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idDV,
                       (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           mma_bf16_ts(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
-                      sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idACC, (it > 0 || kk > 0));
+                      sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idDK, (it > 0 || kk > 0));
         mma_commit(&bar[KB_Q_EMPTY + s]);
       }
       if (ok) mma_commit(&bar[KB_ACC_DONE]);
@@ -327,10 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax warpgroups
     const int t = threadIdx.x % 128;      // key row == TMEM lane
     const int half = threadIdx.x / 128;   // warpgroup: takes query tiles it = half (mod kSoftWG)
-    constexpr int col0 = 0;
     const int key = jt * C::BN + t;
     const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
+    const float dss = ds_scale(stats);
     bool ok = true;
     for (int it = half; it < nq; it += kSoftWG) {
       const int s = it % C::NS, b = it & 1;
@@ -368,12 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - la[e], 32 * h + c);
             if (need_mask && (i0 + 32 * h + c < key)) p = 0.f;
             pv[e] = p;
-            dsv[e] = p * (__uint_as_float(dr[c]) - da[e]);
+            dsv[e] = p * (__uint_as_float(dr[c]) - da[e]) * dss;
           }
           pw[2 * c4] = pack_g(pv[0], pv[1]);
           pw[2 * c4 + 1] = pack_g(pv[2], pv[3]);
-          dw[2 * c4] = pack_g(dsv[0], dsv[1]);
-          dw[2 * c4 + 1] = pack_g(dsv[2], dsv[3]);
+          dw[2 * c4] = pack_f16x2_sat(dsv[0], dsv[1]);
+          dw[2 * c4 + 1] = pack_f16x2_sat(dsv[2], dsv[3]);
         }
         tmem_st16(st_base + packed_col(32 * h), pw);
         tmem_st16(dpt_base + packed_col(32 * h), dw);
@@ -405,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dK row, its inverse rotation and the K-side torques
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);
       grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
-                           table + (size_t)(live ? key : 0) * (D / 2), rsqrtf((float)D),
+                           table + (size_t)(live ? key : 0) * (D / 2), rsqrtf((float)D) / dss,
                            (float)key - 0.5f * (float)(n - 1), live,
                            dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
                            half);
@@ -466,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap map_kt64,
                   const __grid_constant__ CUtensorMap map_v64, const float* __restrict__ lse2p,
                   const float* __restrict__ deltap, const float2* __restrict__ table,
-                  __nv_bfloat16* __restrict__ dq, float* __restrict__ dpart, int n, int BH,
+                  const uint32_t* __restrict__ stats, __nv_bfloat16* __restrict__ dq,
+                  float* __restrict__ dpart, int n, int BH,
                   int causal, uint32_t* err, uint64_t wait_ns) {
   using C = DqCfg<D>;
   constexpr int KID = K_BWD_DQ_SM100;
@@ -541,8 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idSP = idesc_bf16_f32(128, C::BK, 0, 0);
-      constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idS = idesc_f16_f32(128, C::BK, 0, 0);    // fp16 Q~ K~^T
+      constexpr uint32_t idDP = idesc_bf16_f32(128, C::BK, 0, 0);  // bf16 dO V^T
+      constexpr uint32_t idDQ = idesc_f16_f32(128, D, 0, 1);       // fp16 dS K~
       const uint32_t q_s = base_s + C::OFF_Q, do_s = base_s + C::OFF_DO;
       bool ok = mbar_wait(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
       // S / dP of key tile j into TMEM buffer j & 1, which last held dS of tile j - 2;
@@ -558,14 +582,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
           mma_bf16_ss(tmem + C::COL_S + b * 128, sdesc_sw128(q_s + ka, 16, 1024),
-                      sdesc_sw128(kb + kq, 16, 1024), idSP, kk > 0);
+                      sdesc_sw128(kb + kq, 16, 1024), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
           mma_bf16_ss(tmem + C::COL_DP + b * 128, sdesc_sw128(do_s + ka, 16, 1024),
-                      sdesc_sw128(kb + C::KTILE + kq, 16, 1024), idSP, kk > 0);
+                      sdesc_sw128(kb + C::KTILE + kq, 16, 1024), idDP, kk > 0);
         }
         mma_commit(&bar[QB_SP_FULL + b]);
         return true;
@@ -594,12 +618,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax warpgroups
     const int t = threadIdx.x % 128;      // query row == TMEM lane
     const int half = threadIdx.x / 128;   // warpgroup: takes key tiles j = half (mod kSoftWG)
-    constexpr int col0 = 0;
     const int row = qtile * C::BM + t;
     const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
     const float lse2 = lse2p[(size_t)bh * npad + row];
     const float dlt = deltap[(size_t)bh * npad + row];
+    const float dss = ds_scale(stats);
     bool ok = true;
     for (int j = half; j < nk; j += kSoftWG) {
       const int b = j & 1;
@@ -631,9 +655,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int key = key0 + 32 * h + c;
               if (key >= n || (causal && key > row)) p = 0.f;
             }
-            dsv[e] = p * (__uint_as_float(dr[c]) - dlt);
+            dsv[e] = p * (__uint_as_float(dr[c]) - dlt) * dss;
           }
-          dw[c2] = pack_g(dsv[0], dsv[1]);
+          dw[c2] = pack_f16x2_sat(dsv[0], dsv[1]);
         }
         tmem_st16(s_base + packed_col(32 * h), dw);
       }
@@ -646,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool live = row < n;
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);
       grad_row_epilogue<D>(lane_base + C::COL_DQ, base_s + C::OFF_Q, C::QCH, t,
-                           table + (size_t)(live ? row : 0) * (D / 2), rsqrtf((float)D),
+                           table + (size_t)(live ? row : 0) * (D / 2), rsqrtf((float)D) / dss,
                            (float)row - 0.5f * (float)(n - 1), live,
                            dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1),
                            half);
@@ -668,8 +692,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D>
 cudaError_t launch_dkdv_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                          const float* deltap, const float2* table, void* dk, void* dv,
-                          float* dpart, const DevCtl& ctl, cudaStream_t s) {
+                          const float* deltap, const float2* table, const uint32_t* stats,
+                          void* dk, void* dv, float* dpart, const DevCtl& ctl, cudaStream_t s) {
   using C = DkdvCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -677,15 +701,15 @@ cudaError_t launch_dkdv_d(const ra_problem& p, const Sm100Maps& maps, const floa
   const int BH = (int)(p.B * p.H);
   const long long ntk = (p.n + C::BN - 1) / C::BN;
   bwd_dkdv_kernel<D><<<(unsigned)(ntk * BH), kThreads, C::SMEM, s>>>(
-      maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, (__nv_bfloat16*)dk,
+      maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, stats, (__nv_bfloat16*)dk,
       (__nv_bfloat16*)dv, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                        const float* deltap, const float2* table, void* dq, float* dpart,
-                        const DevCtl& ctl, cudaStream_t s) {
+                        const float* deltap, const float2* table, const uint32_t* stats, void* dq,
+                        float* dpart, const DevCtl& ctl, cudaStream_t s) {
   using C = DqCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -693,7 +717,8 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
   const int BH = (int)(p.B * p.H);
   const long long ntq = (p.n + C::BM - 1) / C::BM;
   bwd_dq_kernel<D><<<(unsigned)(ntq * BH), kThreads, C::SMEM, s>>>(
-      maps.qt, maps.dO, maps.kt64, maps.v64, lse2p, deltap, table, (__nv_bfloat16*)dq, dpart,
+      maps.qt, maps.dO, maps.kt64, maps.v64, lse2p, deltap, table, stats, (__nv_bfloat16*)dq,
+      dpart,
       (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
   return cudaGetLastError();
 }
@@ -702,17 +727,18 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
 
 cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,
-                                  void* dk, void* dv, float* dpart, const DevCtl& ctl,
-                                  cudaStream_t s) {
-  if (p.d == 64) return launch_dkdv_d<64>(p, maps, lse2p, deltap, table, dk, dv, dpart, ctl, s);
-  return launch_dkdv_d<128>(p, maps, lse2p, deltap, table, dk, dv, dpart, ctl, s);
+                                  const uint32_t* stats, void* dk, void* dv, float* dpart,
+                                  const DevCtl& ctl, cudaStream_t s) {
+  if (p.d == 64)
+    return launch_dkdv_d<64>(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
+  return launch_dkdv_d<128>(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
 }
 
 cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                                const float* deltap, const float2* table, void* dq, float* dpart,
-                                const DevCtl& ctl, cudaStream_t s) {
-  if (p.d == 64) return launch_dq_d<64>(p, maps, lse2p, deltap, table, dq, dpart, ctl, s);
-  return launch_dq_d<128>(p, maps, lse2p, deltap, table, dq, dpart, ctl, s);
+                                const float* deltap, const float2* table, const uint32_t* stats,
+                                void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s) {
+  if (p.d == 64) return launch_dq_d<64>(p, maps, lse2p, deltap, table, stats, dq, dpart, ctl, s);
+  return launch_dq_d<128>(p, maps, lse2p, deltap, table, stats, dq, dpart, ctl, s);
 }
 
 }  // namespace ra

@@ -33,7 +33,7 @@ constexpr int kLossThreads = 256;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t err;        // uint32 [8]
+  size_t err;        // uint32 [16]: [0..3] status word, [8] max |dO_i|, [9] max |v_j| (fp32 bits)
   size_t loss_part;  // double [kLossBlocks]
   size_t table;      // float2 [n][M]  (cos, sin)
   size_t qt;         // dtype [B*H][n][d]   rotated queries

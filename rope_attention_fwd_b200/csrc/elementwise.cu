@@ -14,6 +14,7 @@
 //                   fp64 ("LeRoPE", Escolhas de Design Principais: alpha shared by all
 //                   heads; Analise Teorica: frequency gradient).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "common.h"
@@ -73,11 +74,13 @@ __global__ void rotate_kernel(const T* __restrict__ q, const T* __restrict__ k,
   dst[2 * idx + 1] = from_f<T>(cs.y * x0 + cs.x * x1);
 }
 
-// bf16 fast path: 4 pairs (16 bytes) per thread.
+// bf16 inputs: 4 pairs (16 bytes) per thread; the rotated rows are written as fp16, the
+// score-operand type of the tensor-core path (11-bit significand).  An entry beyond the
+// fp16 range is clamped (satfinite) and reported as status 6 (RA_ERR_RANGE) in err[0].
 __global__ void rotate_bf16x8_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                      uint4* __restrict__ qt, uint4* __restrict__ kt,
                                      const float2* __restrict__ table, long long rows, int n,
-                                     int M) {
+                                     int M, uint32_t* __restrict__ err) {
   const uint4* src = blockIdx.y == 0 ? q : k;
   uint4* dst = blockIdx.y == 0 ? qt : kt;
   const int vec_per_row = M / 4;  // d/8 vectors of 8 bf16
@@ -92,14 +95,19 @@ __global__ void rotate_bf16x8_kernel(const uint4* __restrict__ q, const uint4* _
   const float c[4] = {t01.x, t01.z, t23.x, t23.z};
   const float s[4] = {t01.y, t01.w, t23.y, t23.w};
   uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  float amax = 0.f;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
+    const __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
     const float x0 = __low2float(pr), x1 = __high2float(pr);
-    pr = __floats2bfloat162_rn(c[j] * x0 - s[j] * x1, s[j] * x0 + c[j] * x1);
-    w[j] = *reinterpret_cast<uint32_t*>(&pr);
+    const float y0 = c[j] * x0 - s[j] * x1, y1 = s[j] * x0 + c[j] * x1;
+    amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
+    uint32_t h;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(y1), "f"(y0));
+    w[j] = h;
   }
   dst[idx] = make_uint4(w[0], w[1], w[2], w[3]);
+  if (!(amax <= 65504.f)) atomicCAS(err, 0u, 6u);  // also catches NaN
 }
 
 // ---------------------------------------------------------------- loss
@@ -215,38 +223,98 @@ __global__ void delta_bf16_kernel(const uint2* __restrict__ o, const uint2* __re
 
 // Padded per-row vectors for the tensor-core backward, over npad = ceil(n/128)*128 rows
 // per head: deltap = rowsum(dO o O) (0 past n) and lse2p = lse * log2(e) (+inf past n,
-// so that exp2(s - lse2) vanishes on the padding rows the tiles read).
+// so that exp2(s - lse2) vanishes on the padding rows the tiles read); and *dmax =
+// max_i |dO_i| (fp32 bits).  Grid-stride over rows with a fixed grid, so that the max
+// costs one atomic per block; non-negative floats order like their bit patterns, so the
+// integer atomicMax is exact and independent of the order of the updates.
+constexpr int kReduceBlocks = 1184;  // 8 per SM
+
+__device__ __forceinline__ void block_max_atomic(float v, uint32_t* dst) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  __shared__ float red[32];
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) m = fmaxf(m, red[w]);
+    atomicMax(dst, __float_as_uint(m));
+  }
+}
+
 template <int D>
-__global__ void bwd_pre_bf16_kernel(const uint2* __restrict__ o, const uint2* __restrict__ dO,
-                                    const float* __restrict__ lse, float* __restrict__ deltap,
-                                    float* __restrict__ lse2p, long long prow_count, int n,
-                                    int npad) {
+__global__ void __launch_bounds__(256)
+    bwd_pre_bf16_kernel(const uint2* __restrict__ o, const uint2* __restrict__ dO,
+                        const float* __restrict__ lse, float* __restrict__ deltap,
+                        float* __restrict__ lse2p, long long prow_count, int n, int npad,
+                        uint32_t* __restrict__ dmax) {
+  constexpr int LPR = D / 4, RPW = 32 / LPR;  // lanes per row, rows per warp
+  const int lane = threadIdx.x % 32;
+  const long long warps_total = (long long)gridDim.x * (blockDim.x / 32);
+  float mx = 0.f;
+  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+       wi * RPW < prow_count; wi += warps_total) {
+    const long long prow = wi * RPW + lane / LPR;
+    const long long bh = prow / npad;
+    const int i = (int)(prow % npad);
+    const bool live = prow < prow_count && i < n;
+    float acc = 0.f, sq = 0.f;
+    if (live) {
+      const long long idx = (bh * n + i) * LPR + lane % LPR;
+      uint2 a = o[idx], b = dO[idx];
+      const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
+      const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
+      const __nv_bfloat162 b0 = *reinterpret_cast<__nv_bfloat162*>(&b.x);
+      const __nv_bfloat162 b1 = *reinterpret_cast<__nv_bfloat162*>(&b.y);
+      acc = __low2float(a0) * __low2float(b0);
+      acc = fmaf(__high2float(a0), __high2float(b0), acc);
+      acc = fmaf(__low2float(a1), __low2float(b1), acc);
+      acc = fmaf(__high2float(a1), __high2float(b1), acc);
+      sq = __low2float(b0) * __low2float(b0);
+      sq = fmaf(__high2float(b0), __high2float(b0), sq);
+      sq = fmaf(__low2float(b1), __low2float(b1), sq);
+      sq = fmaf(__high2float(b1), __high2float(b1), sq);
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    }
+    if (prow < prow_count && lane % LPR == 0) {
+      deltap[prow] = acc;
+      lse2p[prow] = live ? lse[bh * n + i] * 1.4426950408889634f : __int_as_float(0x7f800000);
+    }
+    mx = fmaxf(mx, sqrtf(sq));
+  }
+  block_max_atomic(mx, dmax);
+}
+
+// max_j |v_j| over every row of V (bf16, d in {64, 128}) into *vmax (fp32 bits).
+template <int D>
+__global__ void __launch_bounds__(256)
+    vnorm_max_bf16_kernel(const uint2* __restrict__ v, long long rows, uint32_t* __restrict__ vmax) {
   constexpr int LPR = D / 4, RPW = 32 / LPR;
   const int lane = threadIdx.x % 32;
-  const long long prow =
-      ((long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32) * RPW + lane / LPR;
-  const long long bh = prow / npad;
-  const int i = (int)(prow % npad);
-  const bool live = prow < prow_count && i < n;
-  float acc = 0.f;
-  if (live) {
-    const long long idx = (bh * n + i) * LPR + lane % LPR;
-    uint2 a = o[idx], b = dO[idx];
-    const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
-    const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
-    const __nv_bfloat162 b0 = *reinterpret_cast<__nv_bfloat162*>(&b.x);
-    const __nv_bfloat162 b1 = *reinterpret_cast<__nv_bfloat162*>(&b.y);
-    acc = __low2float(a0) * __low2float(b0);
-    acc = fmaf(__high2float(a0), __high2float(b0), acc);
-    acc = fmaf(__low2float(a1), __low2float(b1), acc);
-    acc = fmaf(__high2float(a1), __high2float(b1), acc);
-  }
+  const long long warps_total = (long long)gridDim.x * (blockDim.x / 32);
+  float mx = 0.f;
+  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+       wi * RPW < rows; wi += warps_total) {
+    const long long row = wi * RPW + lane / LPR;
+    float sq = 0.f;
+    if (row < rows) {
+      uint2 a = v[row * LPR + lane % LPR];
+      const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
+      const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
+      sq = __low2float(a0) * __low2float(a0);
+      sq = fmaf(__high2float(a0), __high2float(a0), sq);
+      sq = fmaf(__low2float(a1), __low2float(a1), sq);
+      sq = fmaf(__high2float(a1), __high2float(a1), sq);
+    }
 #pragma unroll
-  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (prow < prow_count && lane % LPR == 0) {
-    deltap[prow] = acc;
-    lse2p[prow] = live ? lse[bh * n + i] * 1.4426950408889634f : __int_as_float(0x7f800000);
+    for (int off = LPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    mx = fmaxf(mx, sqrtf(sq));
   }
+  block_max_atomic(mx, vmax);
 }
 
 // ---------------------------------------------------------------- dalpha final
@@ -279,26 +347,21 @@ cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table,
 }
 
 cudaError_t launch_rotate(const ra_problem& p, const void* q, const void* k, void* qt, void* kt,
-                          const float2* table, cudaStream_t s) {
+                          const float2* table, uint32_t* err, cudaStream_t s) {
   const int M = (int)(p.d / 2);
   const long long rows = p.B * p.H * p.n;
   const int threads = 256;
-  if (p.dtype == RA_BF16 && M % 4 == 0) {
+  if (p.dtype == RA_BF16) {  // d in {64, 128}: M is a multiple of 4
     const long long total = rows * (M / 4);
     dim3 grid((unsigned)((total + threads - 1) / threads), 2);
-    rotate_bf16x8_kernel<<<grid, threads, 0, s>>>(
-        (const uint4*)q, (const uint4*)k, (uint4*)qt, (uint4*)kt, table, rows, (int)p.n, M);
+    rotate_bf16x8_kernel<<<grid, threads, 0, s>>>((const uint4*)q, (const uint4*)k,
+                                                  (uint4*)qt, (uint4*)kt, table, rows,
+                                                  (int)p.n, M, err);
   } else {
     const long long total = rows * M;
     dim3 grid((unsigned)((total + threads - 1) / threads), 2);
-    if (p.dtype == RA_BF16)
-      rotate_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(
-          (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (__nv_bfloat16*)qt,
-          (__nv_bfloat16*)kt, table, rows, (int)p.n, M);
-    else
-      rotate_kernel<float><<<grid, threads, 0, s>>>((const float*)q, (const float*)k,
-                                                    (float*)qt, (float*)kt, table, rows,
-                                                    (int)p.n, M);
+    rotate_kernel<float><<<grid, threads, 0, s>>>((const float*)q, (const float*)k, (float*)qt,
+                                                  (float*)kt, table, rows, (int)p.n, M);
   }
   return cudaGetLastError();
 }
@@ -350,19 +413,27 @@ cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, flo
 }
 
 cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
-                           float* deltap, float* lse2p, cudaStream_t s) {
+                           float* deltap, float* lse2p, uint32_t* stats, cudaStream_t s) {
   const int npad = (int)padded_rows(p.n);
   const long long prows = p.B * p.H * npad;
-  const int threads = 256, warps = threads / 32;
-  const int rpw = p.d == 64 ? 2 : 1;
-  const long long nwarps = (prows + rpw - 1) / rpw;
-  const unsigned blocks = (unsigned)((nwarps + warps - 1) / warps);
   if (p.d == 64)
-    bwd_pre_bf16_kernel<64><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
-                                                       deltap, lse2p, prows, (int)p.n, npad);
+    bwd_pre_bf16_kernel<64><<<kReduceBlocks, 256, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
+                                                          deltap, lse2p, prows, (int)p.n, npad,
+                                                          stats);
   else
-    bwd_pre_bf16_kernel<128><<<blocks, threads, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
-                                                        deltap, lse2p, prows, (int)p.n, npad);
+    bwd_pre_bf16_kernel<128><<<kReduceBlocks, 256, 0, s>>>((const uint2*)o, (const uint2*)dO,
+                                                           lse, deltap, lse2p, prows, (int)p.n,
+                                                           npad, stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vnorm_max(const ra_problem& p, const void* v, uint32_t* vmax,
+                             cudaStream_t s) {
+  const long long rows = p.B * p.H * p.n;
+  if (p.d == 64)
+    vnorm_max_bf16_kernel<64><<<kReduceBlocks, 256, 0, s>>>((const uint2*)v, rows, vmax);
+  else
+    vnorm_max_bf16_kernel<128><<<kReduceBlocks, 256, 0, s>>>((const uint2*)v, rows, vmax);
   return cudaGetLastError();
 }
 

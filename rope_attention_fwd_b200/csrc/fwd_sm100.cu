@@ -6,7 +6,8 @@
 // ("RoPE attention can be trained in almost-linear time", Metodologia 1: the
 // normalised softmax s(x) applied to the RoPE scores; Q~, K~ are the queries and
 // keys rotated band by band, "LeRoPE: learnable RoPE frequencies", Mecanismo
-// Central).  Exact: no approximation, fp32 accumulation, bf16 operands.
+// Central).  Exact: no approximation; fp32 accumulation; S from fp16 Q~, K~ (the score
+// rounding is what a sharp softmax amplifies), P V from bf16 P and V.
 //
 // CTA = 6 warps, one 128-row query tile, 1 CTA per SM:
 //   warps 0-3  softmax: thread t owns row t (= TMEM lane t) of S and O
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0, 0);
+      constexpr uint32_t idS = idesc_f16_f32(128, C::BN, 0, 0);  // fp16 Q~, K~
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_s = base_s + C::OFF_Q, k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
       const uint32_t p_s = base_s + C::OFF_P;

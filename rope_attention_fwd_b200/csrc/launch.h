@@ -14,8 +14,9 @@ struct DevCtl {
 };
 
 cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table, cudaStream_t s);
+// bf16 problems: Q~, K~ written as fp16; an entry beyond fp16 range sets err[0] = 6.
 cudaError_t launch_rotate(const ra_problem& p, const void* q, const void* k, void* qt, void* kt,
-                          const float2* table, cudaStream_t s);
+                          const float2* table, uint32_t* err, cudaStream_t s);
 cudaError_t launch_loss_partial(const ra_problem& p, const void* o, const void* e, void* dO,
                                 double* part, cudaStream_t s);
 cudaError_t launch_loss_final(const double* part, float* L, cudaStream_t s);
@@ -44,14 +45,19 @@ struct Sm100Maps {
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
 // Padded per-row vectors for the tensor-core backward: delta and lse * log2(e).
+// ... and max_i |dO_i| into stats[0] (fp32 bits, atomic max; stats zeroed by the caller).
 cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
-                           float* deltap, float* lse2p, cudaStream_t s);
+                           float* deltap, float* lse2p, uint32_t* stats, cudaStream_t s);
+// max_j |v_j| into *vmax (fp32 bits, atomic max; zeroed by the caller).
+cudaError_t launch_vnorm_max(const ra_problem& p, const void* v, uint32_t* vmax,
+                             cudaStream_t s);
+// stats: [0] max_i |dO_i|, [1] max_j |v_j| (fp32 bits) for the fp16 scale of dS.
 cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,
-                                  void* dk, void* dv, float* dpart, const DevCtl& ctl,
-                                  cudaStream_t s);
+                                  const uint32_t* stats, void* dk, void* dv, float* dpart,
+                                  const DevCtl& ctl, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                                const float* deltap, const float2* table, void* dq, float* dpart,
-                                const DevCtl& ctl, cudaStream_t s);
+                                const float* deltap, const float2* table, const uint32_t* stats,
+                                void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s);
 
 }  // namespace ra

@@ -3,7 +3,8 @@ times (the same kernels and tiles; the whole [B, H, n, d] problem in one call).
 
 * 1x1x256x64 fp32 and 4x16x2048x64 bf16: every output against the full oracle.
 * 2x32x8192x128, 1x8x32768x128, 8x16x4096x128 (bf16): the oracle is too slow for
-  every head, so it checks sampled heads -- O, dQ, dK, dV on sampled rows, and the
+  every head, so it checks sampled heads -- O and lse on every row, dQ, dK, dV on
+  sampled rows, and the
   head's own dalpha (the GPU's per-head dalpha comes from the same kernels run on that
   head alone) -- plus properties that hold at any size: dalpha of the whole problem is
   the sum of the per-head dalphas, dO is exactly the bf16 rounding of O - E, and L is
@@ -98,9 +99,11 @@ def test_config_sampled(cfg):
         do = o - e
         delta = np.sum(do * o, axis=1)
         rows = _sample_rows(wl.n, rng)
+        # O and lse of every row of the head (the oracle computes them all anyway): rare
+        # elements carry the largest error, so sampled rows alone can miss them
         go = g["o"][b, h].double().cpu().numpy()
-        assert np.max(np.abs(go[rows] - o[rows])) <= tol["o"]
-        assert np.max(np.abs(g["lse"][b, h].double().cpu().numpy()[rows] - lse[rows])) <= tol["lse"]
+        assert np.max(np.abs(go - o)) <= tol["o"]
+        assert np.max(np.abs(g["lse"][b, h].double().cpu().numpy() - lse)) <= tol["lse"]
         dqt = ref.head_backward_rows(qt, kt, v, do[rows], lse[rows], delta[rows], rows,
                                      wl.causal)
         dq = ref.rotate(dqt, phi[rows], sign=-1.0)

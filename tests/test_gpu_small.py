@@ -58,11 +58,9 @@ def test_bf16_many_heads_and_batches():
     compare(gpu_run(inp), oracle_run(inp), "bf16", small=True)
 
 
-@pytest.mark.xfail(reason="bf16 rounding of the rotated q, k perturbs the sharp scores of the "
-                          "bounded-entry regime by ~0.03; needs the split-precision score mode",
-                   strict=False)
 def test_bf16_large_entries():
-    """Bounded-entry regime at a small size: uniform[-3, 3] entries, sharp softmax."""
+    """Bounded-entry regime at a small size: uniform[-3, 3] entries, sharp softmax.  With bf16
+    score operands this case was 0.026 off in O; the fp16 score operands keep it in bounds."""
     wl = small_workload(1, 2, 300, 128, "bf16", False, base=5e5, seed=4, qkve="uniform")
     wl = wl.with_(lo=-3.0, hi=3.0)
     inp = make(wl)

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_PKG, "librope_attn.so")
 RA_F32, RA_BF16 = 0, 1
 _DTYPE = {torch.float32: RA_F32, torch.bfloat16: RA_BF16}
 STATUS = {0: "RA_OK", 1: "RA_ERR_INVALID_ARG", 2: "RA_ERR_UNSUPPORTED", 3: "RA_ERR_WORKSPACE",
-          4: "RA_ERR_CUDA", 5: "RA_ERR_TIMEOUT"}
+          4: "RA_ERR_CUDA", 5: "RA_ERR_TIMEOUT", 6: "RA_ERR_RANGE"}
 
 
 class RaProblem(ctypes.Structure):

@@ -288,18 +288,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: converged issue, one elected lane
       constexpr uint32_t idST = idesc_f16_f32(128, C::BQ, 0, 0);   // fp16 K~ Q~^T
       constexpr uint32_t idDPT = idesc_bf16_f32(128, C::BQ, 0, 0);  // bf16 V dO^T
       constexpr uint32_t idDV = idesc_bf16_f32(128, D, 0, 1);       // bf16 P^T dO
       constexpr uint32_t idDK = idesc_f16_f32(128, D, 0, 1);        // fp16 dS^T Q~
       const uint32_t k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
-      bool ok = mbar_wait(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      bool ok = mbar_wait_warp(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
       // S^T / dP^T of step `it` into TMEM buffer it & 1.  That buffer last held P^T / dS^T
       // of step it - 2, whose dV / dK MMAs were issued earlier by this thread (in order).
       auto issue_sdp = [&](int it) -> bool {
         const int s = it % C::NS, b = it & 1;
-        if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
+        if (!mbar_wait_warp(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
           return false;
         tc_fence_after();
         const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
@@ -307,43 +307,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + b * 128 + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
+          mma_ss_warp(tmem + b * 128 + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
                       sdesc_sw128(qb + kq, 16, 1024), idST, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + b * 128 + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
+          mma_ss_warp(tmem + b * 128 + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
                       sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idDPT, kk > 0);
         }
-        mma_commit(&bar[KB_SDP_FULL + b]);
+        mma_commit_warp(&bar[KB_SDP_FULL + b]);
         return true;
       };
       if (ok) ok = issue_sdp(0);
       for (int it = 0; ok && it < nq; ++it) {
         if (it + 1 < nq && !issue_sdp(it + 1)) break;
         const int s = it % C::NS, b = it & 1;
-        if (!mbar_wait(&bar[KB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
+        if (!mbar_wait_warp(&bar[KB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
           break;
         tc_fence_after();
         const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
         // dV += P^T dO_i and dK~ += dS^T Q~_i with P^T, dS^T read from TMEM
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_bf16_ts(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
+          mma_ts_warp(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
                       sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idDV,
                       (it > 0 || kk > 0));
 #pragma unroll
         for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_bf16_ts(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
+          mma_ts_warp(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
                       sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idDK, (it > 0 || kk > 0));
-        mma_commit(&bar[KB_Q_EMPTY + s]);
+        mma_commit_warp(&bar[KB_Q_EMPTY + s]);
       }
-      if (ok) mma_commit(&bar[KB_ACC_DONE]);
-      mma_commit(&bar[KB_DRAIN]);
+      if (ok) mma_commit_warp(&bar[KB_ACC_DONE]);
+      mma_commit_warp(&bar[KB_DRAIN]);
       int dummy = 0;
-      mbar_wait(&bar[KB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
+      mbar_wait_warp(&bar[KB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups
@@ -563,17 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: converged issue, one elected lane
       constexpr uint32_t idS = idesc_f16_f32(128, C::BK, 0, 0);    // fp16 Q~ K~^T
       constexpr uint32_t idDP = idesc_bf16_f32(128, C::BK, 0, 0);  // bf16 dO V^T
       constexpr uint32_t idDQ = idesc_f16_f32(128, D, 0, 1);       // fp16 dS K~
       const uint32_t q_s = base_s + C::OFF_Q, do_s = base_s + C::OFF_DO;
-      bool ok = mbar_wait(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
+      bool ok = mbar_wait_warp(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
       // S / dP of key tile j into TMEM buffer j & 1, which last held dS of tile j - 2;
       // the dQ MMA that read it was issued earlier by this thread (in-order execution).
       auto issue_sp = [&](int j) -> bool {
         const int s = j % C::NS, b = j & 1;
-        if (!mbar_wait(&bar[QB_KV_FULL + s], (j / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
+        if (!mbar_wait_warp(&bar[QB_KV_FULL + s], (j / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
           return false;
         tc_fence_after();
         const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
@@ -581,38 +581,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_S + b * 128, sdesc_sw128(q_s + ka, 16, 1024),
+          mma_ss_warp(tmem + C::COL_S + b * 128, sdesc_sw128(q_s + ka, 16, 1024),
                       sdesc_sw128(kb + kq, 16, 1024), idS, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_DP + b * 128, sdesc_sw128(do_s + ka, 16, 1024),
+          mma_ss_warp(tmem + C::COL_DP + b * 128, sdesc_sw128(do_s + ka, 16, 1024),
                       sdesc_sw128(kb + C::KTILE + kq, 16, 1024), idDP, kk > 0);
         }
-        mma_commit(&bar[QB_SP_FULL + b]);
+        mma_commit_warp(&bar[QB_SP_FULL + b]);
         return true;
       };
       if (ok) ok = issue_sp(0);
       for (int j = 0; ok && j < nk; ++j) {
         if (j + 1 < nk && !issue_sp(j + 1)) break;
         const int s = j % C::NS, b = j & 1;
-        if (!mbar_wait(&bar[QB_DS_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
+        if (!mbar_wait_warp(&bar[QB_DS_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
           break;
         tc_fence_after();
         const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
         // dQ~ += dS K~_j with dS read from TMEM
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_bf16_ts(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
+          mma_ts_warp(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
                       sdesc_sw128(kb + kk * 2048, C::KCH, 1024), idDQ, (j > 0 || kk > 0));
-        mma_commit(&bar[QB_KV_EMPTY + s]);
+        mma_commit_warp(&bar[QB_KV_EMPTY + s]);
       }
-      if (ok) mma_commit(&bar[QB_ACC_DONE]);
-      mma_commit(&bar[QB_DRAIN]);
+      if (ok) mma_commit_warp(&bar[QB_ACC_DONE]);
+      mma_commit_warp(&bar[QB_DRAIN]);
       int dummy = 0;
-      mbar_wait(&bar[QB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
+      mbar_wait_warp(&bar[QB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroups

@@ -208,19 +208,19 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp: converged issue, one elected lane
       constexpr uint32_t idS = idesc_f16_f32(128, C::BN, 0, 0);  // fp16 Q~, K~
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_s = base_s + C::OFF_Q, k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
       const uint32_t p_s = base_s + C::OFF_P;
-      bool ok = mbar_wait(&bar[B_Q_FULL], 0, abort_flag, err, K_FWD_SM100, 3, wait_ns);
+      bool ok = mbar_wait_warp(&bar[B_Q_FULL], 0, abort_flag, err, K_FWD_SM100, 3, wait_ns);
       tc_fence_after();
       auto issue_s = [&](int j) -> bool {
         const int s = j % C::NS, sb = j & 1;
-        if (!mbar_wait(&bar[B_K_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 4,
+        if (!mbar_wait_warp(&bar[B_K_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 4,
                        wait_ns))
           return false;
-        if (!mbar_wait(&bar[B_S_FREE + sb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 5,
+        if (!mbar_wait_warp(&bar[B_S_FREE + sb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 5,
                        wait_ns))
           return false;
         tc_fence_after();
@@ -228,21 +228,21 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_S + sb * 128, sdesc_sw128(q_s + koff, 16, 1024),
+          mma_ss_warp(tmem + C::COL_S + sb * 128, sdesc_sw128(q_s + koff, 16, 1024),
                       sdesc_sw128(kb + koff, 16, 1024), idS, kk > 0);
         }
-        mma_commit(&bar[B_S_FULL + sb]);
-        mma_commit(&bar[B_K_EMPTY + s]);
+        mma_commit_warp(&bar[B_S_FULL + sb]);
+        mma_commit_warp(&bar[B_K_EMPTY + s]);
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int j = 0; ok && j < nkv; ++j) {
         if (j + 1 < nkv && !issue_s(j + 1)) break;
         const int s = j % C::NS, pb = j & 1;
-        if (!mbar_wait(&bar[B_P_FULL + pb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 6,
+        if (!mbar_wait_warp(&bar[B_P_FULL + pb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 6,
                        wait_ns))
           break;
-        if (!mbar_wait(&bar[B_V_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 7,
+        if (!mbar_wait_warp(&bar[B_V_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 7,
                        wait_ns))
           break;
         tc_fence_after();
@@ -253,25 +253,25 @@ __global__ void __launch_bounds__(192, 1)
         // thread execute in issue order.
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_bf16_ts(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
+          mma_ts_warp(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
                       sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
 #else
         const uint32_t pbase = p_s + pb * C::PTILE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint32_t poff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_bf16_ss(tmem + C::COL_O, sdesc_sw128(pbase + poff, 16, 1024),
+          mma_ss_warp(tmem + C::COL_O, sdesc_sw128(pbase + poff, 16, 1024),
                       sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
         }
 #endif
-        mma_commit(&bar[B_P_FREE + pb]);
-        mma_commit(&bar[B_V_EMPTY + s]);
+        mma_commit_warp(&bar[B_P_FREE + pb]);
+        mma_commit_warp(&bar[B_V_EMPTY + s]);
       }
-      if (ok) mma_commit(&bar[B_O_DONE]);
+      if (ok) mma_commit_warp(&bar[B_O_DONE]);
       // Every MMA issued above has finished once this commit arrives.
-      mma_commit(&bar[B_DRAIN]);
+      mma_commit_warp(&bar[B_DRAIN]);
       int dummy = 0;
-      mbar_wait(&bar[B_DRAIN], 0, &dummy, err, K_FWD_SM100, 23, wait_ns);
+      mbar_wait_warp(&bar[B_DRAIN], 0, &dummy, err, K_FWD_SM100, 23, wait_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0-3

@@ -69,17 +69,31 @@ __device__ __forceinline__ float exp2_col(float x, int c) {
   return fast_exp2(x);
 }
 
+#ifndef RA_MMA_BATCH
+#define RA_MMA_BATCH 1
+#endif
 #ifndef RA_BWD_SOFT_WG
 #define RA_BWD_SOFT_WG 2
 #endif
-// Softmax warpgroups per CTA, in ping-pong: warpgroup g takes the streamed tiles
-// it = g, g + kSoftWG, ... (TMEM buffer it & 1), every row (TMEM lane) and all 64 columns
-// of its tile, so one warpgroup's TMEM round trips and barrier hand-offs overlap the
-// other's arithmetic.  The epilogue splits the D output columns between the warpgroups.
+#ifndef RA_BWD_SPLIT
+#define RA_BWD_SPLIT 1
+#endif
+// Softmax warpgroups per CTA, and how they share the streamed 64-column tiles:
+//  * ping-pong (RA_BWD_SPLIT 0): warpgroup g takes the tiles it = g, g + kSoftWG, ...
+//    (TMEM buffer it & 1), every row (TMEM lane) and all 64 columns, so one warpgroup's
+//    TMEM round trips and barrier hand-offs overlap the other's arithmetic;
+//  * column split (RA_BWD_SPLIT 1, two warpgroups): both take every tile, warpgroup g
+//    its columns 32g .. 32g + 31, which halves the latency from S / dP to dS.
+// The epilogue splits the D output columns between the warpgroups.
 constexpr int kSoftWG = RA_BWD_SOFT_WG;
+constexpr bool kSplit = RA_BWD_SPLIT != 0;
+static_assert(!kSplit || kSoftWG == 2, "the column split takes two warpgroups");
 constexpr int kSoftThreads = 128 * kSoftWG;
 constexpr int kThreads = kSoftThreads + 64;  // + TMA producer warp + MMA warp
-constexpr int kCols = 64;                     // streamed columns per softmax thread
+constexpr int kCols = kSplit ? 32 : 64;       // streamed columns per softmax thread and tile
+constexpr int kTileStep = kSplit ? 1 : kSoftWG;   // tiles between one warpgroup's tiles
+constexpr int kHalves = kSplit ? 1 : 2;           // 32-column halves per thread and tile
+constexpr int kDsArrivals = kSplit ? kSoftThreads : 128;
 constexpr int kProdWarp = 4 * kSoftWG, kMmaWarp = 4 * kSoftWG + 1;
 
 __device__ __forceinline__ uint32_t pack_g(float lo, float hi) {
@@ -148,6 +162,23 @@ __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_
   }
 }
 
+// Row t of a 128B-swizzled 16-bit tile (D columns in D/64 chunks, `chunk` bytes apart)
+// into this thread's TMEM lane from column taddr on: elements 2w, 2w+1 land in column w
+// (low, high half), the packing of an MMA A operand read from TMEM.
+template <int D>
+__device__ __forceinline__ void tile_row_to_tmem(uint32_t tile_s, uint32_t chunk, int t,
+                                                 uint32_t taddr) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    uint32_t w[32];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      ld_shared_v4(tile_s + c * chunk + sw128_off(t, u), w[4 * u], w[4 * u + 1], w[4 * u + 2],
+                   w[4 * u + 3]);
+    tmem_st32(taddr + 32 * c, w);
+  }
+}
+
 // Fixed-order per-band sums of the torques of rows 0-63 and 64-127 (red is [128][M+1]),
 // written as the partials of 64-row tiles 2*tile128 and 2*tile128+1 (when they exist).
 template <int D>
@@ -188,7 +219,7 @@ enum DkdvBar {
   KB_Q_FULL = 1,                        // +stage
   KB_Q_EMPTY = 1 + RA_DKDV_STAGES,      // +stage
   KB_SDP_FULL = 1 + 2 * RA_DKDV_STAGES, // +buffer: S^T and dP^T of that buffer computed
-  KB_DS_FULL = KB_SDP_FULL + 2,         // +buffer: P^T, dS^T written (kSoftThreads arrivals)
+  KB_DS_FULL = KB_SDP_FULL + 2,         // +buffer: P^T, dS^T written (kDsArrivals arrivals)
   KB_ACC_DONE = KB_DS_FULL + 2,
   KB_DRAIN,
   KB_COUNT
@@ -231,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == kSoftThreads) {
     for (int i = 0; i < KB_COUNT; ++i)
-      mbar_init(&bar[i], (i == KB_DS_FULL || i == KB_DS_FULL + 1) ? 128 : 1);
+      mbar_init(&bar[i], (i == KB_DS_FULL || i == KB_DS_FULL + 1) ? kDsArrivals : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -293,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idDPT = idesc_bf16_f32(128, C::BQ, 0, 0);  // bf16 V dO^T
       constexpr uint32_t idDV = idesc_bf16_f32(128, D, 0, 1);       // bf16 P^T dO
       constexpr uint32_t idDK = idesc_f16_f32(128, D, 0, 1);        // fp16 dS^T Q~
-      const uint32_t k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
+      const SDesc dkm = sdesc_split(base_s, 16, 1024);       // K-major tiles
+      const SDesc dmn = sdesc_split(base_s, C::QCH, 1024);   // Q~ / dO tiles read MN-major
       bool ok = mbar_wait_warp(&bar[KB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
       // S^T / dP^T of step `it` into TMEM buffer it & 1.  That buffer last held P^T / dS^T
       // of step it - 2, whose dV / dK MMAs were issued earlier by this thread (in order).
@@ -302,20 +334,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_warp(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
           return false;
         tc_fence_after();
-        const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
-          const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_ss_warp(tmem + b * 128 + C::COL_ST, sdesc_sw128(k_s + ka, 16, 1024),
-                      sdesc_sw128(qb + kq, 16, 1024), idST, kk > 0);
+        const SDesc qs = sdesc_advance(dkm, C::OFF_ST + s * C::STAGE);
+        if constexpr (D == 128 && RA_MMA_BATCH) {
+          mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K),
+                                             sdesc_at(qs, 0), idST, 0);
+          mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_DPT,
+                                             sdesc_at(dkm, C::OFF_V), sdesc_at(qs, C::QTILE),
+                                             idDPT, 0);
+          mma_commit_warp(&bar[KB_SDP_FULL + b]);
+          return true;
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
           const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-          mma_ss_warp(tmem + b * 128 + C::COL_DPT, sdesc_sw128(v_s + ka, 16, 1024),
-                      sdesc_sw128(qb + C::QTILE + kq, 16, 1024), idDPT, kk > 0);
+          mma_ss_warp(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K + ka), sdesc_at(qs, kq),
+                      idST, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
+          const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
+          mma_ss_warp(tmem + b * 128 + C::COL_DPT, sdesc_at(dkm, C::OFF_V + ka),
+                      sdesc_at(qs, C::QTILE + kq), idDPT, kk > 0);
         }
         mma_commit_warp(&bar[KB_SDP_FULL + b]);
         return true;
@@ -327,17 +368,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_warp(&bar[KB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
           break;
         tc_fence_after();
-        const uint32_t qb = base_s + C::OFF_ST + s * C::STAGE;
+        const SDesc qm = sdesc_advance(dmn, C::OFF_ST + s * C::STAGE);
         // dV += P^T dO_i and dK~ += dS^T Q~_i with P^T, dS^T read from TMEM
+        if constexpr (RA_MMA_BATCH) {
+          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+              tmem + C::COL_DV, tmem + b * 128 + C::COL_ST, sdesc_at(qm, C::QTILE), idDV, it > 0);
+          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+              tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT, sdesc_at(qm, 0), idDK, it > 0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
-                      sdesc_sw128(qb + C::QTILE + kk * 2048, C::QCH, 1024), idDV,
-                      (it > 0 || kk > 0));
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            mma_ts_warp(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
+                        sdesc_at(qm, C::QTILE + kk * 2048), idDV, (it > 0 || kk > 0));
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
-                      sdesc_sw128(qb + kk * 2048, C::QCH, 1024), idDK, (it > 0 || kk > 0));
+          for (int kk = 0; kk < C::BQ / 16; ++kk)
+            mma_ts_warp(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
+                        sdesc_at(qm, kk * 2048), idDK, (it > 0 || kk > 0));
+        }
         mma_commit_warp(&bar[KB_Q_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[KB_ACC_DONE]);
@@ -354,11 +401,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float scale_log2 = kLog2e / sqrtf((float)D);
     const float dss = ds_scale(stats);
     bool ok = true;
-    for (int it = half; it < nq; it += kSoftWG) {
+    for (int it = kSplit ? 0 : half; it < nq; it += kTileStep) {
       const int s = it % C::NS, b = it & 1;
       const int i0 = qstart + it * C::BQ;
-      if (!mbar_wait(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6, wait_ns) ||
-          !mbar_wait(&bar[KB_SDP_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 7, wait_ns)) {
+      if (!mbar_wait_warp(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6, wait_ns) ||
+          !mbar_wait_warp(&bar[KB_SDP_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 7, wait_ns)) {
         ok = false;
         break;
       }
@@ -372,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 32 columns at a time: load S^T, dP^T; P^T, dS^T back as bf16 over the first 16
       // columns of each half (packed_col order), all before this warpgroup's arrival
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < kHalves; ++hh) {
+        const int h = kSplit ? half : hh;
         uint32_t sr[32], dr[32];
         tmem_ld32(st_base + 32 * h, sr);
         tmem_ld32(dpt_base + 32 * h, dr);
@@ -404,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar[KB_DS_FULL + b]);
     }
-    if (ok && mbar_wait(&bar[KB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
+    if (ok && mbar_wait_warp(&bar[KB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
       tc_fence_after();
       const bool live = key < n;
       // dV row (this thread's D / kSoftWG columns)
@@ -451,6 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #ifndef RA_DQ_STAGES
 #define RA_DQ_STAGES 4
 #endif
+#ifndef RA_DQ_BUFS
+#define RA_DQ_BUFS 2
+#endif
 
 template <int D>
 struct DqCfg {
@@ -463,9 +514,19 @@ struct DqCfg {
   static constexpr uint32_t STAGE = 2 * KTILE;  // K~_j, V_j
   static constexpr uint32_t OFF_BAR = OFF_ST + NS * STAGE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  // TMEM: two buffers of [S (64 fp32) | dP (64 fp32)] at 128 * b, dS written back as bf16
-  // over the start of each thread's S slice; dQ~ accumulator at 256.
-  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 256;
+  // TMEM: NB buffers of [S (64 fp32) | dP (64 fp32)] at 128 * b, dS written back as fp16
+  // over the start of each thread's S slice, then the dQ~ accumulator.
+  //  * NB = 3: the issuer runs two key tiles ahead of the softmax, so the S -> dS latency
+  //    of a tile hides behind two tiles of MMAs; Q~ and dO stay in shared memory.
+  //  * NB = 2: only one tile ahead, but the stationary Q~ (fp16) and dO (bf16) tiles sit in
+  //    TMEM (two per column) as the A operands of the S and dP MMAs, which then read only
+  //    their 2 KB B tile from shared memory and run at the tensor rate (from shared memory,
+  //    4 KB more per K-step, an M=128, N=64 MMA is bandwidth-bound).
+  static constexpr int NB = RA_DQ_BUFS;
+  static_assert(NB == 2 || NB == 3, "two or three S/dP buffers");
+  static_assert(NS >= NB, "the K~/V ring holds every key tile whose S, dP are in flight");
+  static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 128 * NB;
+  static constexpr uint32_t COL_QT = 256 + D, COL_DOT = 256 + D + D / 2;  // NB == 2 only
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
 };
@@ -475,9 +536,10 @@ enum DqBar {
   QB_KV_FULL = 1,                      // +stage
   QB_KV_EMPTY = 1 + RA_DQ_STAGES,      // +stage
   QB_SP_FULL = 1 + 2 * RA_DQ_STAGES,   // +buffer
-  QB_DS_FULL = QB_SP_FULL + 2,         // +buffer, kSoftThreads arrivals
-  QB_ACC_DONE = QB_DS_FULL + 2,
+  QB_DS_FULL = QB_SP_FULL + RA_DQ_BUFS,  // +buffer, kDsArrivals arrivals
+  QB_ACC_DONE = QB_DS_FULL + RA_DQ_BUFS,
   QB_DRAIN,
+  QB_QT_READY,                         // Q~, dO copied into TMEM (one arrival per softmax warp)
   QB_COUNT
 };
 
@@ -512,7 +574,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == kSoftThreads) {
     for (int i = 0; i < QB_COUNT; ++i)
-      mbar_init(&bar[i], (i == QB_DS_FULL || i == QB_DS_FULL + 1) ? 128 : 1);
+      mbar_init(&bar[i], (i >= QB_DS_FULL && i < QB_DS_FULL + RA_DQ_BUFS) ? kDsArrivals
+                         : i == QB_QT_READY                       ? kSoftThreads / 32
+                                                                  : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -567,46 +631,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = idesc_f16_f32(128, C::BK, 0, 0);    // fp16 Q~ K~^T
       constexpr uint32_t idDP = idesc_bf16_f32(128, C::BK, 0, 0);  // bf16 dO V^T
       constexpr uint32_t idDQ = idesc_f16_f32(128, D, 0, 1);       // fp16 dS K~
-      const uint32_t q_s = base_s + C::OFF_Q, do_s = base_s + C::OFF_DO;
-      bool ok = mbar_wait_warp(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 2, wait_ns);
-      // S / dP of key tile j into TMEM buffer j & 1, which last held dS of tile j - 2;
+      const SDesc dqd = sdesc_split(base_s, 16, 1024);                   // Q~, dO K-major
+      const SDesc dkm = sdesc_split(base_s + C::OFF_ST, 16, 1024);      // K~_j, V_j K-major
+      const SDesc dmn = sdesc_split(base_s + C::OFF_ST, C::KCH, 1024);  // K~_j read MN-major
+      bool ok = mbar_wait_warp(&bar[C::NB == 2 ? QB_QT_READY : QB_Q_FULL], 0, abort_flag, err,
+                               KID, 2, wait_ns);
+      // S / dP of key tile j into TMEM buffer j % NB, which last held dS of tile j - NB;
       // the dQ MMA that read it was issued earlier by this thread (in-order execution).
       auto issue_sp = [&](int j) -> bool {
-        const int s = j % C::NS, b = j & 1;
+        const int s = j % C::NS, b = j % C::NB;
         if (!mbar_wait_warp(&bar[QB_KV_FULL + s], (j / C::NS) & 1, abort_flag, err, KID, 3, wait_ns))
           return false;
         tc_fence_after();
-        const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
+        const SDesc ks = sdesc_advance(dkm, s * C::STAGE);
+        if constexpr (C::NB == 2 && D == 128 && RA_MMA_BATCH) {
+          mma8_kmajor<true, 0, C::KCH>(tmem + C::COL_S + b * 128, tmem + C::COL_QT,
+                                       sdesc_at(ks, 0), idS, 0);
+          mma8_kmajor<true, 0, C::KCH>(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT,
+                                       sdesc_at(ks, C::KTILE), idDP, 0);
+        } else if constexpr (C::NB == 2) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
-          const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_S + b * 128, sdesc_sw128(q_s + ka, 16, 1024),
-                      sdesc_sw128(kb + kq, 16, 1024), idS, kk > 0);
-        }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+            mma_ts_warp(tmem + C::COL_S + b * 128, tmem + C::COL_QT + 8 * kk, sdesc_at(ks, kq),
+                        idS, kk > 0);
+          }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
-          const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_DP + b * 128, sdesc_sw128(do_s + ka, 16, 1024),
-                      sdesc_sw128(kb + C::KTILE + kq, 16, 1024), idDP, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+            mma_ts_warp(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT + 8 * kk,
+                        sdesc_at(ks, C::KTILE + kq), idDP, kk > 0);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
+            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+            mma_ss_warp(tmem + C::COL_S + b * 128, sdesc_at(dqd, C::OFF_Q + ka),
+                        sdesc_at(ks, kq), idS, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
+            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
+            mma_ss_warp(tmem + C::COL_DP + b * 128, sdesc_at(dqd, C::OFF_DO + ka),
+                        sdesc_at(ks, C::KTILE + kq), idDP, kk > 0);
+          }
         }
         mma_commit_warp(&bar[QB_SP_FULL + b]);
         return true;
       };
-      if (ok) ok = issue_sp(0);
+      for (int j = 0; ok && j < min(nk, C::NB - 1); ++j) ok = issue_sp(j);
       for (int j = 0; ok && j < nk; ++j) {
-        if (j + 1 < nk && !issue_sp(j + 1)) break;
-        const int s = j % C::NS, b = j & 1;
-        if (!mbar_wait_warp(&bar[QB_DS_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
+        if (j + C::NB - 1 < nk && !issue_sp(j + C::NB - 1)) break;
+        const int s = j % C::NS, b = j % C::NB;
+        if (!mbar_wait_warp(&bar[QB_DS_FULL + b], (j / C::NB) & 1, abort_flag, err, KID, 5,
+                            wait_ns))
           break;
         tc_fence_after();
-        const uint32_t kb = base_s + C::OFF_ST + s * C::STAGE;
+        const SDesc km = sdesc_advance(dmn, s * C::STAGE);
         // dQ~ += dS K~_j with dS read from TMEM
+        if constexpr (RA_MMA_BATCH) {
+          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+              tmem + C::COL_DQ, tmem + C::COL_S + b * 128, sdesc_at(km, 0), idDQ, j > 0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
-                      sdesc_sw128(kb + kk * 2048, C::KCH, 1024), idDQ, (j > 0 || kk > 0));
+          for (int kk = 0; kk < C::BK / 16; ++kk)
+            mma_ts_warp(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
+                        sdesc_at(km, kk * 2048), idDQ, (j > 0 || kk > 0));
+        }
         mma_commit_warp(&bar[QB_KV_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[QB_ACC_DONE]);
@@ -625,9 +718,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float dlt = deltap[(size_t)bh * npad + row];
     const float dss = ds_scale(stats);
     bool ok = true;
-    for (int j = half; j < nk; j += kSoftWG) {
-      const int b = j & 1;
-      if (!mbar_wait(&bar[QB_SP_FULL + b], (j >> 1) & 1, abort_flag, err, KID, 6, wait_ns)) {
+    if constexpr (C::NB == 2) {
+      // the stationary Q~ and dO rows into TMEM (warpgroup g copies tiles g, g + kSoftWG, ...)
+      ok = mbar_wait_warp(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 11, wait_ns);
+      if (ok) {
+        for (int src = half; src < 2; src += kSoftWG)
+          tile_row_to_tmem<D>(base_s + (src == 0 ? C::OFF_Q : C::OFF_DO), C::QCH, t,
+                              lane_base + (src == 0 ? C::COL_QT : C::COL_DOT));
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[QB_QT_READY]);
+    }
+    for (int j = kSplit ? 0 : half; ok && j < nk; j += kTileStep) {
+      const int b = j % C::NB;
+      if (!mbar_wait_warp(&bar[QB_SP_FULL + b], (j / C::NB) & 1, abort_flag, err, KID, 6,
+                          wait_ns)) {
         ok = false;
         break;
       }
@@ -637,7 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key0 = j * C::BK;
       const bool need_mask = (causal && key0 + C::BK - 1 > qtile * C::BM) || (key0 + C::BK > n);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < kHalves; ++hh) {
+        const int h = kSplit ? half : hh;
         uint32_t sr[32], dr[32];
         tmem_ld32(s_base + 32 * h, sr);
         tmem_ld32(dp_base + 32 * h, dr);
@@ -665,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar[QB_DS_FULL + b]);
     }
-    if (ok && mbar_wait(&bar[QB_ACC_DONE], 0, abort_flag, err, KID, 8, wait_ns)) {
+    if (ok && mbar_wait_warp(&bar[QB_ACC_DONE], 0, abort_flag, err, KID, 8, wait_ns)) {
       tc_fence_after();
       const bool live = row < n;
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);

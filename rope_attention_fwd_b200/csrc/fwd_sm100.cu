@@ -81,6 +81,9 @@ enum FwdBar {
 #ifndef RA_FWD_RESCALE_TAU
 #define RA_FWD_RESCALE_TAU 8.0f
 #endif
+#ifndef RA_MMA_BATCH
+#define RA_MMA_BATCH 1
+#endif
 #ifndef RA_FWD_PACK_ALU
 #define RA_FWD_PACK_ALU 0
 #endif
@@ -211,8 +214,8 @@ __global__ void __launch_bounds__(192, 1)
     {  // the whole warp: converged issue, one elected lane
       constexpr uint32_t idS = idesc_f16_f32(128, C::BN, 0, 0);  // fp16 Q~, K~
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_s = base_s + C::OFF_Q, k_s = base_s + C::OFF_K, v_s = base_s + C::OFF_V;
-      const uint32_t p_s = base_s + C::OFF_P;
+      const SDesc dkm = sdesc_split(base_s, 16, 1024);        // K-major tiles
+      const SDesc dmn = sdesc_split(base_s, C::CHUNK, 1024);  // V tiles read MN-major
       bool ok = mbar_wait_warp(&bar[B_Q_FULL], 0, abort_flag, err, K_FWD_SM100, 3, wait_ns);
       tc_fence_after();
       auto issue_s = [&](int j) -> bool {
@@ -224,12 +227,17 @@ __global__ void __launch_bounds__(192, 1)
                        wait_ns))
           return false;
         tc_fence_after();
-        const uint32_t kb = k_s + s * C::TILE;
+        const SDesc ks = sdesc_advance(dkm, C::OFF_K + s * C::TILE);
+        if constexpr (D == 128 && RA_MMA_BATCH) {
+          mma8_kmajor<false, C::CHUNK, C::CHUNK>(tmem + C::COL_S + sb * 128,
+                                                 sdesc_at(dkm, C::OFF_Q), sdesc_at(ks, 0), idS, 0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_S + sb * 128, sdesc_sw128(q_s + koff, 16, 1024),
-                      sdesc_sw128(kb + koff, 16, 1024), idS, kk > 0);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+            mma_ss_warp(tmem + C::COL_S + sb * 128, sdesc_at(dkm, C::OFF_Q + koff),
+                        sdesc_at(ks, koff), idS, kk > 0);
+          }
         }
         mma_commit_warp(&bar[B_S_FULL + sb]);
         mma_commit_warp(&bar[B_K_EMPTY + s]);
@@ -246,22 +254,25 @@ __global__ void __launch_bounds__(192, 1)
                        wait_ns))
           break;
         tc_fence_after();
-        const uint32_t vb = v_s + s * C::TILE;
+        const SDesc vs = sdesc_advance(dmn, C::OFF_V + s * C::TILE);
 #if RA_FWD_P_TMEM
         // P_j (bf16, two per column) sits over S_j in TMEM buffer pb; the S MMA that next
         // overwrites that buffer is issued after this one, and tcgen05.mma ops from one
         // thread execute in issue order.
+        if constexpr (C::BN == 128 && RA_MMA_BATCH) {
+          mma8_ts_mn(tmem + C::COL_O, tmem + C::COL_S + pb * 128, sdesc_at(vs, 0), idO, j > 0);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
-                      sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
+          for (int kk = 0; kk < C::BN / 16; ++kk)
+            mma_ts_warp(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
+                        sdesc_at(vs, kk * 2048), idO, (j > 0 || kk > 0));
+        }
 #else
-        const uint32_t pbase = p_s + pb * C::PTILE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint32_t poff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_O, sdesc_sw128(pbase + poff, 16, 1024),
-                      sdesc_sw128(vb + kk * 2048, C::CHUNK, 1024), idO, (j > 0 || kk > 0));
+          mma_ss_warp(tmem + C::COL_O, sdesc_at(dkm, C::OFF_P + pb * C::PTILE + poff),
+                      sdesc_at(vs, kk * 2048), idO, (j > 0 || kk > 0));
         }
 #endif
         mma_commit_warp(&bar[B_P_FREE + pb]);

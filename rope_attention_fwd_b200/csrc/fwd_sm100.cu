@@ -1,6 +1,6 @@
 // fwd_sm100.cu -- exact RoPE attention forward on B200 tensor cores (tcgen05).
 //
-// Computes, for one 128-row tile of queries of one (batch, head):
+// Computes, for two 128-row tiles of queries of one (batch, head):
 //   S = Q~ K~^T / sqrt(d) tile by tile, the online-softmax row max and row sum,
 //   O = sum_j P_j V_j / l and lse = log sum_j exp(S_ij)
 // ("RoPE attention can be trained in almost-linear time", Metodologia 1: the
@@ -9,15 +9,22 @@
 // Central).  Exact: no approximation; fp32 accumulation; S from fp16 Q~, K~ (the score
 // rounding is what a sharp softmax amplifies), P V from bf16 P and V.
 //
-// CTA = 6 warps, one 128-row query tile, 1 CTA per SM:
-//   warps 0-3  softmax: thread t owns row t (= TMEM lane t) of S and O
-//   warp  4    TMA producer: Q~ once, then K~_j / V_j into a 2-stage ring
-//   warp  5    TMEM allocator + single-thread tcgen05.mma issuer
-// TMEM (512 columns): S double buffer at columns 0 and 128, O at column 256.
-// Shared memory: Q~, the K~/V rings and a double-buffered P tile (bf16, K-major,
-// 128B swizzle), so P_{j+1} can be written while O += P_j V_j is still running.
-// The issuer runs one tile ahead: S_{j+1} is on the tensor core while the softmax
-// warps turn S_j into P_j.
+// Why two query tiles per CTA: every K~_j / V_j tile a CTA streams in serves all of its
+// query rows, and streaming those tiles from L2 (about 9 GB per launch with one 128-row
+// tile per CTA on 2 x 32 x 8192 x 128) runs into the on-chip L2 -> SM bandwidth before
+// the tensor cores are busy.  With 256 rows per CTA the traffic halves.
+//
+// CTA = 10 warps, query tiles a = 2T, b = 2T + 1, 1 CTA per SM:
+//   warps 0-3 / 4-7  softmax of tile a / b: thread t owns row t (TMEM lane t) of S and O
+//   warp  8          TMA producer: Q~_a, Q~_b once, then K~_j (3-stage ring), V_j (2 stages)
+//   warp  9          TMEM allocator + tcgen05.mma issuer (converged warp, one elected lane)
+// TMEM (512 columns): S_x at 128 x with P_x (bf16, two per column) written over its first
+// 64 columns, O_x at 256 + 128 x.  One S buffer per tile: the MMAs alternate between the
+// tiles, S_a(j+1) running on the tensor core while the softmax of tile b turns S_b(j) into
+// P_b(j) and the reverse, in the issue order
+//   S_a(0) S_b(0) | PV_a(0) S_a(1) PV_b(0) S_b(1) | PV_a(1) S_a(2) PV_b(1) S_b(2) | ...
+// (S_x(j+1) overwrites P_x(j) after the PV MMA that read it: one thread's tcgen05.mma ops
+// execute in issue order).
 //
 // Online softmax with a lazy rescale: a row keeps its running max m until a tile's
 // max exceeds it by more than kRescaleTau (log2 units); until then P = 2^(s - m) may
@@ -32,8 +39,6 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
-#include <type_traits>
-
 #include "common.h"
 #include "launch.h"
 #include "sm100.cuh"
@@ -41,23 +46,17 @@
 namespace ra {
 namespace {
 
-#ifndef RA_FWD_P_TMEM
-#define RA_FWD_P_TMEM 1
-#endif
-
 template <int D>
 struct FwdCfg {
-  // P in TMEM frees the shared-memory P buffers for a third K~/V stage.
-  static constexpr int BM = 128, BN = 128, NS = RA_FWD_P_TMEM ? 3 : 2;
+  static constexpr int BM = 128, BN = 128;   // rows per query tile (two per CTA), keys per tile
+  static constexpr int NSK = 3, NSV = 2;     // K~ and V ring stages
   static constexpr int CH = D / 64;                       // 64-column chunks per row
   static constexpr uint32_t CHUNK = 128u * 128u;          // [128 rows][128 B]
-  static constexpr uint32_t TILE = CHUNK * CH;            // [128][D] bf16
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + TILE;
-  static constexpr uint32_t OFF_V = OFF_K + NS * TILE;
-  static constexpr uint32_t PTILE = 2 * CHUNK;             // [128][128] bf16 = 2 chunks
-  static constexpr uint32_t OFF_P = OFF_V + NS * TILE;    // 2 P buffers (P in smem only)
-  static constexpr uint32_t OFF_BAR = OFF_P + (RA_FWD_P_TMEM ? 0 : 2 * PTILE);
+  static constexpr uint32_t TILE = CHUNK * CH;            // [128][D] 16-bit
+  static constexpr uint32_t OFF_Q = 0;                    // Q~_a, Q~_b
+  static constexpr uint32_t OFF_K = 2 * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + NSK * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + NSV * TILE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_O = 256;
@@ -65,17 +64,16 @@ struct FwdCfg {
 
 enum FwdBar {
   B_Q_FULL = 0,
-  B_K_FULL = 1,   // +stage (3)
-  B_K_EMPTY = 4,  // +stage (3)
-  B_V_FULL = 7,   // +stage (3)
-  B_V_EMPTY = 10, // +stage (3)
-  B_S_FULL = 13,  // +buffer
-  B_S_FREE = 15,  // +buffer, 128 arrivals
-  B_P_FULL = 17,  // +buffer, 128 arrivals
-  B_P_FREE = 19,  // +buffer: the PV MMA of that buffer's P has completed
-  B_O_DONE = 21,
-  B_DRAIN = 22,
-  B_COUNT = 23
+  B_K_FULL = 1,               // +stage (3)
+  B_K_EMPTY = 4,              // +stage (3)
+  B_V_FULL = 7,               // +stage (2)
+  B_V_EMPTY = 9,              // +stage (2)
+  B_S_FULL = 11,              // +tile: S_x(j) computed
+  B_P_FULL = 13,              // +tile: P_x(j) written (and O_x rescaled); 4 warp arrivals
+  B_PV_DONE = 15,             // +tile: O_x += P_x(j) V_j has completed
+  B_O_DONE = 17,
+  B_DRAIN = 18,
+  B_COUNT = 19
 };
 
 #ifndef RA_FWD_RESCALE_TAU
@@ -84,52 +82,31 @@ enum FwdBar {
 #ifndef RA_MMA_BATCH
 #define RA_MMA_BATCH 1
 #endif
-#ifndef RA_FWD_PACK_ALU
-#define RA_FWD_PACK_ALU 0
-#endif
 #ifndef RA_FWD_POLY_EVERY
 #define RA_FWD_POLY_EVERY 0
 #endif
 constexpr float kRescaleTau = RA_FWD_RESCALE_TAU;
+constexpr int kFwdThreads = 320;
+constexpr int kFwdProdWarp = 8, kFwdMmaWarp = 9;
 
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
-#if RA_FWD_PACK_ALU
-  return pack_bf16x2_alu(lo, hi);
-#else
-  return pack_bf16x2(lo, hi);
-#endif
-}
-
-template <int I>
-__device__ __forceinline__ float exp2_elem(float x) {
+// 2^x of column c: every RA_FWD_POLY_EVERY-th column on the FMA pipe (exp2_poly), the
+// others on MUFU, to split the exponential load off the XU pipe.
+__device__ __forceinline__ float exp2_col(float x, int c) {
 #if RA_FWD_POLY_EVERY > 0
-  if constexpr (I % RA_FWD_POLY_EVERY == RA_FWD_POLY_EVERY - 1) return exp2_poly(x);
+  if (c % RA_FWD_POLY_EVERY == RA_FWD_POLY_EVERY - 1) return exp2_poly(x);
 #endif
   return fast_exp2(x);
 }
 
-template <int I, int N>
-struct Unroll {
-  template <typename F>
-  __device__ __forceinline__ static void run(F&& f) {
-    f(std::integral_constant<int, I>{});
-    Unroll<I + 1, N>::run(f);
-  }
-};
-template <int N>
-struct Unroll<N, N> {
-  template <typename F>
-  __device__ __forceinline__ static void run(F&&) {}
-};
-
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
                      const __grid_constant__ CUtensorMap map_k,
                      const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
                      float* __restrict__ lse, int n, int BH, int causal, uint32_t* err,
                      uint64_t wait_ns, int starve_block) {
   using C = FwdCfg<D>;
+  constexpr int KID = K_FWD_SM100;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -140,21 +117,27 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
-  const int tile = ntq - 1 - (int)(blockIdx.x / BH);  // heaviest causal tiles first
+  const int ntp = (ntq + 1) / 2;
+  const int T = ntp - 1 - (int)(blockIdx.x / BH);  // heaviest causal tile pairs first
   const int bh = (int)(blockIdx.x % BH);
   const int ntk = (n + C::BN - 1) / C::BN;
-  const int nkv = causal ? min(tile + 1, ntk) : ntk;
+  // key tiles of query tile x (0 when the tile lies past the end of the sequence)
+  auto nkv_of = [&](int x) -> int {
+    const int qt = 2 * T + x;
+    if (qt >= ntq) return 0;
+    return causal ? min(qt + 1, ntk) : ntk;
+  };
+  const int nkv_a = nkv_of(0), nkv_b = nkv_of(1);
+  const int nkv = max(nkv_a, nkv_b);
+  const bool has_b = nkv_b > 0;
 
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i)
-      mbar_init(&bar[i], (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL ||
-                          i == B_P_FULL + 1)
-                             ? 128
-                             : 1);
+      mbar_init(&bar[i], (i == B_P_FULL || i == B_P_FULL + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -163,7 +146,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kFwdProdWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
@@ -173,23 +156,32 @@ __global__ void __launch_bounds__(192, 1)
       // bounded wait must expire and report RA_ERR_TIMEOUT instead of hanging.
       const bool load_q = (int)blockIdx.x != starve_block;
       if (load_q) {
-        mbar_arrive_expect_tx(&bar[B_Q_FULL], C::TILE);
-        for (int c = 0; c < C::CH; ++c)
-          tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &map_q, &bar[B_Q_FULL], c * 64,
-                      tile * C::BM, bh);
+        mbar_arrive_expect_tx(&bar[B_Q_FULL], (has_b ? 2 : 1) * C::TILE);
+        for (int x = 0; x < (has_b ? 2 : 1); ++x)
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(base + C::OFF_Q + x * C::TILE + c * C::CHUNK, &map_q, &bar[B_Q_FULL],
+                        c * 64, (2 * T + x) * C::BM, bh);
       }
       int issued_k = -1, issued_v = -1;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % C::NS;
-        const uint32_t ph = (j / C::NS) & 1;
-        if (!mbar_wait(&bar[B_K_EMPTY + s], ph ^ 1, abort_flag, err, K_FWD_SM100, 1, wait_ns))
-          break;
+      auto load_k = [&](int j) -> bool {
+        const int s = j % C::NSK;
+        if (!mbar_wait(&bar[B_K_EMPTY + s], ((j / C::NSK) & 1) ^ 1, abort_flag, err, KID, 1,
+                       wait_ns))
+          return false;
         mbar_arrive_expect_tx(&bar[B_K_FULL + s], C::TILE);
         for (int c = 0; c < C::CH; ++c)
           tma_load_3d(base + C::OFF_K + s * C::TILE + c * C::CHUNK, &map_k, &bar[B_K_FULL + s],
                       c * 64, j * C::BN, bh);
         issued_k = j;
-        if (!mbar_wait(&bar[B_V_EMPTY + s], ph ^ 1, abort_flag, err, K_FWD_SM100, 2, wait_ns))
+        return true;
+      };
+      // K~ runs one tile ahead of V: S_x(j + 1) is issued right after PV_x(j)
+      bool ok = nkv > 0 ? load_k(0) : true;
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv && !load_k(j + 1)) break;
+        const int s = j % C::NSV;
+        if (!mbar_wait(&bar[B_V_EMPTY + s], ((j / C::NSV) & 1) ^ 1, abort_flag, err, KID, 2,
+                       wait_ns))
           break;
         mbar_arrive_expect_tx(&bar[B_V_FULL + s], C::TILE);
         for (int c = 0; c < C::CH; ++c)
@@ -200,135 +192,135 @@ __global__ void __launch_bounds__(192, 1)
       if (*abort_flag) {
         // Let every copy already in flight land before the CTA's shared memory goes away.
         int dummy = 0;
-        if (load_q) mbar_wait(&bar[B_Q_FULL], 0, &dummy, err, K_FWD_SM100, 20, wait_ns);
-        for (int j = max(0, issued_k - C::NS + 1); j <= issued_k; ++j)
-          mbar_wait(&bar[B_K_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, K_FWD_SM100, 21,
-                    wait_ns);
-        for (int j = max(0, issued_v - C::NS + 1); j <= issued_v; ++j)
-          mbar_wait(&bar[B_V_FULL + j % C::NS], (j / C::NS) & 1, &dummy, err, K_FWD_SM100, 22,
-                    wait_ns);
+        if (load_q) mbar_wait(&bar[B_Q_FULL], 0, &dummy, err, KID, 20, wait_ns);
+        for (int j = max(0, issued_k - C::NSK + 1); j <= issued_k; ++j)
+          mbar_wait(&bar[B_K_FULL + j % C::NSK], (j / C::NSK) & 1, &dummy, err, KID, 21, wait_ns);
+        for (int j = max(0, issued_v - C::NSV + 1); j <= issued_v; ++j)
+          mbar_wait(&bar[B_V_FULL + j % C::NSV], (j / C::NSV) & 1, &dummy, err, KID, 22, wait_ns);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kFwdMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    {  // the whole warp: converged issue, one elected lane
-      constexpr uint32_t idS = idesc_f16_f32(128, C::BN, 0, 0);  // fp16 Q~, K~
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-      const SDesc dkm = sdesc_split(base_s, 16, 1024);        // K-major tiles
-      const SDesc dmn = sdesc_split(base_s, C::CHUNK, 1024);  // V tiles read MN-major
-      bool ok = mbar_wait_warp(&bar[B_Q_FULL], 0, abort_flag, err, K_FWD_SM100, 3, wait_ns);
-      tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % C::NS, sb = j & 1;
-        if (!mbar_wait_warp(&bar[B_K_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 4,
-                       wait_ns))
-          return false;
-        if (!mbar_wait_warp(&bar[B_S_FREE + sb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 5,
-                       wait_ns))
-          return false;
-        tc_fence_after();
-        const SDesc ks = sdesc_advance(dkm, C::OFF_K + s * C::TILE);
-        if constexpr (D == 128 && RA_MMA_BATCH) {
-          mma8_kmajor<false, C::CHUNK, C::CHUNK>(tmem + C::COL_S + sb * 128,
-                                                 sdesc_at(dkm, C::OFF_Q), sdesc_at(ks, 0), idS, 0);
-        } else {
+    constexpr uint32_t idS = idesc_f16_f32(128, C::BN, 0, 0);  // fp16 Q~, K~
+    constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);     // bf16 P, V
+    const SDesc dkm = sdesc_split(base_s, 16, 1024);        // K-major tiles
+    const SDesc dmn = sdesc_split(base_s, C::CHUNK, 1024);  // V tiles read MN-major
+    bool ok = mbar_wait_warp(&bar[B_Q_FULL], 0, abort_flag, err, KID, 3, wait_ns);
+    tc_fence_after();
+    const int nkv_x[2] = {nkv_a, nkv_b};
+    // S_x(j) = Q~_x K~_j^T into TMEM buffer x (K~_j already waited for)
+    auto issue_s = [&](int x, int j) {
+      const SDesc ks = sdesc_advance(dkm, C::OFF_K + (j % C::NSK) * C::TILE);
+      const uint32_t q_off = C::OFF_Q + x * C::TILE;
+      if constexpr (D == 128 && RA_MMA_BATCH) {
+        mma8_kmajor<false, C::CHUNK, C::CHUNK>(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off),
+                                               sdesc_at(ks, 0), idS, 0);
+      } else {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-            mma_ss_warp(tmem + C::COL_S + sb * 128, sdesc_at(dkm, C::OFF_Q + koff),
-                        sdesc_at(ks, koff), idS, kk > 0);
-          }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss_warp(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off + koff), sdesc_at(ks, koff),
+                      idS, kk > 0);
         }
-        mma_commit_warp(&bar[B_S_FULL + sb]);
-        mma_commit_warp(&bar[B_K_EMPTY + s]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv && !issue_s(j + 1)) break;
-        const int s = j % C::NS, pb = j & 1;
-        if (!mbar_wait_warp(&bar[B_P_FULL + pb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 6,
-                       wait_ns))
-          break;
-        if (!mbar_wait_warp(&bar[B_V_FULL + s], (j / C::NS) & 1, abort_flag, err, K_FWD_SM100, 7,
-                       wait_ns))
+      }
+      mma_commit_warp(&bar[B_S_FULL + x]);
+    };
+    auto wait_k = [&](int j) -> bool {
+      if (!mbar_wait_warp(&bar[B_K_FULL + j % C::NSK], (j / C::NSK) & 1, abort_flag, err, KID, 4,
+                          wait_ns))
+        return false;
+      tc_fence_after();
+      return true;
+    };
+    if (ok && nkv > 0) {
+      ok = wait_k(0);
+      if (ok) {
+        for (int x = 0; x < 2; ++x)
+          if (nkv_x[x] > 0) issue_s(x, 0);
+        mma_commit_warp(&bar[B_K_EMPTY + 0]);
+      }
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const bool next = j + 1 < nkv;
+      if (next && !(ok = wait_k(j + 1))) break;
+      if (!(ok = mbar_wait_warp(&bar[B_V_FULL + j % C::NSV], (j / C::NSV) & 1, abort_flag, err,
+                                KID, 7, wait_ns)))
+        break;
+      for (int x = 0; x < 2; ++x) {
+        if (j >= nkv_x[x]) continue;
+        if (!(ok = mbar_wait_warp(&bar[B_P_FULL + x], j & 1, abort_flag, err, KID, 6, wait_ns)))
           break;
         tc_fence_after();
-        const SDesc vs = sdesc_advance(dmn, C::OFF_V + s * C::TILE);
-#if RA_FWD_P_TMEM
-        // P_j (bf16, two per column) sits over S_j in TMEM buffer pb; the S MMA that next
-        // overwrites that buffer is issued after this one, and tcgen05.mma ops from one
-        // thread execute in issue order.
+        // O_x += P_x(j) V_j with P_x(j) read from TMEM buffer x
+        const SDesc vs = sdesc_advance(dmn, C::OFF_V + (j % C::NSV) * C::TILE);
         if constexpr (C::BN == 128 && RA_MMA_BATCH) {
-          mma8_ts_mn(tmem + C::COL_O, tmem + C::COL_S + pb * 128, sdesc_at(vs, 0), idO, j > 0);
+          mma8_ts_mn(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128, sdesc_at(vs, 0), idO,
+                     j > 0);
         } else {
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
-            mma_ts_warp(tmem + C::COL_O, tmem + C::COL_S + pb * 128 + kk * 8,
+            mma_ts_warp(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128 + kk * 8,
                         sdesc_at(vs, kk * 2048), idO, (j > 0 || kk > 0));
         }
-#else
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint32_t poff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_O, sdesc_at(dkm, C::OFF_P + pb * C::PTILE + poff),
-                      sdesc_at(vs, kk * 2048), idO, (j > 0 || kk > 0));
-        }
-#endif
-        mma_commit_warp(&bar[B_P_FREE + pb]);
-        mma_commit_warp(&bar[B_V_EMPTY + s]);
+        mma_commit_warp(&bar[B_PV_DONE + x]);
+        if (next && j + 1 < nkv_x[x]) issue_s(x, j + 1);
       }
-      if (ok) mma_commit_warp(&bar[B_O_DONE]);
-      // Every MMA issued above has finished once this commit arrives.
-      mma_commit_warp(&bar[B_DRAIN]);
-      int dummy = 0;
-      mbar_wait_warp(&bar[B_DRAIN], 0, &dummy, err, K_FWD_SM100, 23, wait_ns);
+      if (!ok) break;
+      mma_commit_warp(&bar[B_V_EMPTY + j % C::NSV]);
+      if (next) mma_commit_warp(&bar[B_K_EMPTY + (j + 1) % C::NSK]);
     }
+    if (ok) mma_commit_warp(&bar[B_O_DONE]);
+    // Every MMA issued above has finished once this commit arrives.
+    mma_commit_warp(&bar[B_DRAIN]);
+    int dummy = 0;
+    mbar_wait_warp(&bar[B_DRAIN], 0, &dummy, err, KID, 23, wait_ns);
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int t = threadIdx.x;  // row within the tile == TMEM lane
-    const int row = tile * C::BM + t;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // ------------------------------------------------------------ softmax warpgroups
+    const int x = warp / 4;            // query tile a (0) or b (1)
+    const int t = threadIdx.x % 128;   // row within the tile == TMEM lane
+    const int qt = 2 * T + x;
+    const int row = qt * C::BM + t;
+    const int my_nkv = x == 0 ? nkv_a : nkv_b;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t s_base = lane_base + C::COL_S + x * 128;
+    const uint32_t o_base = lane_base + C::COL_O + x * 128;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
     float m = -CUDART_INF_F, l = 0.f;  // running max (log2 units, scaled) and row sum
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1, pb = j & 1;
-      if (!mbar_wait(&bar[B_S_FULL + sb], (j >> 1) & 1, abort_flag, err, K_FWD_SM100, 8,
-                     wait_ns)) {
+    for (int j = 0; j < my_nkv; ++j) {
+      if (!mbar_wait_warp(&bar[B_S_FULL + x], j & 1, abort_flag, err, KID, 8, wait_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float x[128];
-      {
-        uint32_t r[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + C::COL_S + sb * 128 + 32 * c, r[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_wait_ld(r[c]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(r[c][i]);
-      }
-      tc_fence_before();
-      mbar_arrive(&bar[B_S_FREE + sb]);
-
       const int key0 = j * C::BN;
-      if ((key0 + C::BN > n) || (causal && j == tile)) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int key = key0 + i;
-          if (key >= n || (causal && key > row)) x[i] = -CUDART_INF_F;
-        }
-      }
-      // row max of the raw scores, 8 independent chains
+      // columns of this row that hold a key (all of them except on the diagonal tile and
+      // the ragged last tile)
+      const bool need_mask = (key0 + C::BN > n) || (causal && j == qt);
+      const int nvalid =
+          need_mask ? max(0, min(C::BN, (causal ? min(n, row + 1) : n) - key0)) : C::BN;
+      // pass 1: the row max of the raw scores (masked entries excluded)
       float mp[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mp[a] = x[a];
+      for (int a = 0; a < 8; ++a) mp[a] = -CUDART_INF_F;
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], x[i]);
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(s_base + 64 * c2, r0);
+        tmem_ld32(s_base + 64 * c2 + 32, r1);
+        tmem_wait_ld(r0);
+        tmem_wait_ld(r1);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (64 * c2 + i >= nvalid) r0[i] = __float_as_uint(-CUDART_INF_F);
+            if (64 * c2 + 32 + i >= nvalid) r1[i] = __float_as_uint(-CUDART_INF_F);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          mp[i & 7] = fmaxf(mp[i & 7], fmaxf(__uint_as_float(r0[i]), __uint_as_float(r1[i])));
+      }
       const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * scale_log2;
       // lazy rescale: move the reference max only when some row of the warp needs it
@@ -341,49 +333,37 @@ __global__ void __launch_bounds__(192, 1)
         m = m_new;
       }
       const float m_use = m == -CUDART_INF_F ? 0.f : m;
+      // pass 2: P = 2^(s scale - m) chunk by chunk, summed and written as bf16 over S.
+      // Chunk c (columns 32c..32c+31) lands in columns 16c..16c+15, inside chunks this
+      // thread has already read.
       float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      Unroll<0, 128>::run([&](auto I) {
-        constexpr int i = decltype(I)::value;
-        x[i] = exp2_elem<i>(fmaf(x[i], scale_log2, -m_use));
-        sp[i & 7] += x[i];
-      });
-      l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
-
-#if RA_FWD_P_TMEM
-      // P_j -> TMEM over S_j (this thread's lane, 64 columns of bf16 pairs).  The PV MMA
-      // that read this buffer two tiles ago completed before S_j did.
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w[32];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(s_base + 32 * c, r);
+        tmem_wait_ld(r);
+        float pv[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = pack_p(x[64 * h + 2 * i], x[64 * h + 2 * i + 1]);
-        tmem_st32(lane_base + C::COL_S + sb * 128 + 32 * h, w);
-      }
-      tmem_wait_st();
-#else
-      // P_j -> shared memory buffer pb once O += P_{j-2} V_{j-2} has released it
-      if (!mbar_wait(&bar[B_P_FREE + pb], ((j >> 1) & 1) ^ 1, abort_flag, err, K_FWD_SM100, 9,
-                     wait_ns)) {
-        ok = false;
-        break;
-      }
-      const uint32_t p_row = base_s + C::OFF_P + pb * C::PTILE;
+        for (int i = 0; i < 32; ++i)
+          pv[i] = exp2_col(fmaf(__uint_as_float(r[i]), scale_log2, -m_use), 32 * c + i);
+        if (need_mask) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float* src = &x[h * 64 + u * 8];
-          st_shared_v4(p_row + h * C::CHUNK + sw128_off(t, u), pack_p(src[0], src[1]),
-                       pack_p(src[2], src[3]), pack_p(src[4], src[5]), pack_p(src[6], src[7]));
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= nvalid) pv[i] = 0.f;
         }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sp[i & 7] += pv[i];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) w[i2] = pack_bf16x2(pv[2 * i2], pv[2 * i2 + 1]);
+        tmem_st16(s_base + 16 * c, w);
       }
-      fence_proxy_async_smem();
-#endif
+      l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
+      tmem_wait_st();
       if (warp_rescale && j > 0) {
-        // O must hold every P_{j'} V_{j'} with j' < j: wait for the PV MMA of step j-1
-        const int pj = j - 1;
-        if (!mbar_wait(&bar[B_P_FREE + (pj & 1)], (pj >> 1) & 1, abort_flag, err, K_FWD_SM100,
-                       11, wait_ns)) {
+        // O_x must hold every P_x(j') V_j' with j' < j: wait for the PV MMA of step j-1
+        if (!mbar_wait_warp(&bar[B_PV_DONE + x], (j - 1) & 1, abort_flag, err, KID, 11,
+                            wait_ns)) {
           ok = false;
           break;
         }
@@ -391,24 +371,26 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(lane_base + C::COL_O + 32 * c, r);
+          tmem_ld32(o_base + 32 * c, r);
           tmem_wait_ld(r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-          tmem_st32(lane_base + C::COL_O + 32 * c, r);
+          tmem_st32(o_base + 32 * c, r);
         }
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&bar[B_P_FULL + pb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_P_FULL + x]);
     }
-    if (ok && mbar_wait(&bar[B_O_DONE], 0, abort_flag, err, K_FWD_SM100, 10, wait_ns)) {
+    if (ok && my_nkv > 0 &&
+        mbar_wait_warp(&bar[B_O_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
       tc_fence_after();
       const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(lane_base + C::COL_O + 32 * c, r);
+        tmem_ld32(o_base + 32 * c, r);
         tmem_wait_ld(r);
         if (row < n) {
           uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * n + row) * D + 32 * c);
@@ -428,7 +410,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -443,7 +425,8 @@ cudaError_t launch_fwd_d(const ra_problem& p, const Sm100Maps& maps, void* o, fl
   if (e != cudaSuccess) return e;
   const int BH = (int)(p.B * p.H);
   const long long ntq = (p.n + C::BM - 1) / C::BM;
-  fwd_sm100_kernel<D><<<(unsigned)(ntq * BH), 192, C::SMEM, s>>>(
+  const long long ntp = (ntq + 1) / 2;
+  fwd_sm100_kernel<D><<<(unsigned)(ntp * BH), kFwdThreads, C::SMEM, s>>>(
       maps.qt, maps.kt, maps.v, (__nv_bfloat16*)o, lse, (int)p.n, BH, p.causal, ctl.err,
       ctl.wait_ns, ctl.starve_block);
   return cudaGetLastError();

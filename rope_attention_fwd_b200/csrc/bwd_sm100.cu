@@ -117,14 +117,56 @@ __device__ __forceinline__ float ds_scale(const uint32_t* __restrict__ stats) {
   return exp2f(e);
 }
 
+// Table rows staged in shared memory for the epilogues: a row of D/2 (cos, sin) pairs is
+// D*4 bytes; the stride adds 16 bytes so that the 16-byte reads of 8 consecutive threads
+// (one shared-memory phase), each in its own row, fall in distinct banks.
+template <int D>
+struct TabStage {
+  static constexpr int ROWB = D / 2 * 8, STRIDE = ROWB + 16, UNITS = ROWB / 16;
+  static constexpr uint32_t BYTES = 128u * STRIDE;
+};
+
+// The cos/sin table rows [row0, row0 + 128) into shared memory at dst, by the kSoftThreads
+// softmax threads with coalesced 16-byte loads (one row per thread, read from global, is
+// 32 separate sectors per warp load); rows at or past n hold (cos, sin) = (1, 0).  The
+// caller syncs the group before the rows are read.
+template <int D>
+__device__ __forceinline__ void stage_table(const float2* __restrict__ table, int row0, int n,
+                                            uint8_t* dst) {
+  using TS = TabStage<D>;
+  constexpr int PER = 128 * TS::UNITS / kSoftThreads;  // 16-byte units per thread
+  constexpr int BATCH = PER < 8 ? PER : 8;             // loads in flight before the stores
+  static_assert(PER * kSoftThreads == 128 * TS::UNITS && PER % BATCH == 0, "even split");
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(table);
+#pragma unroll
+  for (int k0 = 0; k0 < PER; k0 += BATCH) {
+    uint4 v[BATCH];
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int i = threadIdx.x + (k0 + k) * kSoftThreads;
+      const int r = i / TS::UNITS, u = i % TS::UNITS;
+      v[k] = make_uint4(0x3f800000u, 0u, 0x3f800000u, 0u);
+      if (row0 + r < n)
+        v[k] = *reinterpret_cast<const uint4*>(src + (size_t)(row0 + r) * TS::ROWB + u * 16);
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int i = threadIdx.x + (k0 + k) * kSoftThreads;
+      const int r = i / TS::UNITS, u = i % TS::UNITS;
+      *reinterpret_cast<uint4*>(dst + r * TS::STRIDE + u * 16) = v[k];
+    }
+  }
+}
+
 // Epilogue of one gradient row held in TMEM (D fp32 columns from tmem_acc, this
 // thread's lane): g = acc * scale is dX~ of position `pos`; writes R(-pos theta_hat) g as
 // bf16 to out_row (when live) and the band torques w * (g1 x0 - g0 x1) to red_row, where
-// x~ is row t of the 128B-swizzled fp16 tile at x_tile_s (chunk stride x_chunk).
+// x~ is row t of the 128B-swizzled fp16 tile at x_tile_s (chunk stride x_chunk) and the
+// (cos, sin) pairs of position pos are the staged table row at tab_row.
 template <int D>
 __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_tile_s,
                                                   uint32_t x_chunk, int t,
-                                                  const float2* __restrict__ trow, float scale,
+                                                  const uint8_t* tab_row, float scale,
                                                   float w, bool live,
                                                   __nv_bfloat16* __restrict__ out_row,
                                                   float* red_row, int half) {
@@ -142,6 +184,15 @@ __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_
     for (int u = 0; u < 4; ++u)
       ld_shared_v4(ch + sw128_off(t, u0 + u), xw[4 * u], xw[4 * u + 1], xw[4 * u + 2],
                    xw[4 * u + 3]);
+    float csv[32];  // (cos, sin) of bands 16c .. 16c + 15
+#pragma unroll
+    for (int k2 = 0; k2 < 8; ++k2) {
+      const float4 v = *reinterpret_cast<const float4*>(tab_row + (16 * c + 2 * k2) * 8);
+      csv[4 * k2] = v.x;
+      csv[4 * k2 + 1] = v.y;
+      csv[4 * k2 + 2] = v.z;
+      csv[4 * k2 + 3] = v.w;
+    }
     uint32_t ow[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -149,8 +200,8 @@ __device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_
       const float g1 = __uint_as_float(r[2 * k + 1]) * scale;
       const __half2 xp = *reinterpret_cast<const __half2*>(&xw[k]);
       const float x0 = __low2float(xp), x1 = __high2float(xp);
-      const float2 cs = live ? trow[16 * c + k] : make_float2(1.f, 0.f);
-      ow[k] = pack_bf16x2(cs.x * g0 + cs.y * g1, cs.x * g1 - cs.y * g0);
+      const float cs_x = csv[2 * k], cs_y = csv[2 * k + 1];
+      ow[k] = pack_bf16x2(cs_x * g0 + cs_y * g1, cs_x * g1 - cs_y * g0);
       red_row[16 * c + k] = live ? w * (g1 * x0 - g0 * x1) : 0.f;
     }
     if (live) {
@@ -211,7 +262,9 @@ struct DkdvCfg {
   // written back as bf16 over the first half of each thread's S^T / dP^T slice.
   static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
+  static constexpr uint32_t RED_BYTES = (128u * (D / 2 + 1) * 4u + 1023u) / 1024u * 1024u;
+  static_assert(NS * STAGE >= RED_BYTES + TabStage<D>::BYTES,
+                "torque buffer and staged table fit the stages");
 };
 
 enum DkdvBar {
@@ -455,6 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait_warp(&bar[KB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
       tc_fence_after();
       const bool live = key < n;
+      // every Q~/dO stage has been consumed: the ring holds the torque buffer and the table
+      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
+      uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
+      stage_table<D>(table, jt * C::BN, n, tab);
       // dV row (this thread's D / kSoftWG columns)
 #pragma unroll
       for (int cc = 0; cc < D / 32 / kSoftWG; ++cc) {
@@ -473,9 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // dK row, its inverse rotation and the K-side torques
-      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
+      softmax_group_sync();
       grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
-                           table + (size_t)(live ? key : 0) * (D / 2), rsqrtf((float)D) / dss,
+                           tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
                            (float)key - 0.5f * (float)(n - 1), live,
                            dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
                            half);
@@ -528,7 +585,9 @@ struct DqCfg {
   static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 128 * NB;
   static constexpr uint32_t COL_QT = 256 + D, COL_DOT = 256 + D + D / 2;  // NB == 2 only
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(NS * STAGE >= 128u * (D / 2 + 1) * 4u, "torque buffer fits the stages");
+  static constexpr uint32_t RED_BYTES = (128u * (D / 2 + 1) * 4u + 1023u) / 1024u * 1024u;
+  static_assert(NS * STAGE >= RED_BYTES + TabStage<D>::BYTES,
+                "torque buffer and staged table fit the stages");
 };
 
 enum DqBar {
@@ -776,9 +835,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && mbar_wait_warp(&bar[QB_ACC_DONE], 0, abort_flag, err, KID, 8, wait_ns)) {
       tc_fence_after();
       const bool live = row < n;
+      // every K~/V stage has been consumed: the ring holds the torque buffer and the table
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);
+      uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
+      stage_table<D>(table, qtile * C::BM, n, tab);
+      softmax_group_sync();
       grad_row_epilogue<D>(lane_base + C::COL_DQ, base_s + C::OFF_Q, C::QCH, t,
-                           table + (size_t)(live ? row : 0) * (D / 2), rsqrtf((float)D) / dss,
+                           tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
                            (float)row - 0.5f * (float)(n - 1), live,
                            dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1),
                            half);

@@ -107,6 +107,21 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
                         void* dq, void* dk, void* dv, float* dalpha,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* Backward from the forward's saved operands: the same dq, dk, dv, dalpha as
+ * rope_attn_bwd, but the table, Q~ and K~ are taken from ws as the most recent
+ * rope_attn_fwd on this ws left them (the saved-for-backward tensors of a training
+ * step), so q and k are not passed and the rotation is not redone.
+ * Caller contract: that forward ran on the same problem, q, k and alpha (their
+ * contents unchanged since), on a stream ordered before this call, and nothing wrote
+ * ws in between except rope_attn_loss.  Nothing checks the contract: other contents of
+ * those regions give wrong gradients, not an error.  alpha is still read (dalpha is
+ * theta_hat times the summed torques).  Leaves the device error word as the forward
+ * set it (an RA_ERR_RANGE from the forward's rotation stays visible). */
+ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
+                              const float* lse, const void* dO, const float* alpha,
+                              void* dq, void* dk, void* dv, float* dalpha,
+                              void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, reads and clears the device error word in ws.
  * Returns RA_OK; RA_ERR_TIMEOUT if a kernel gave up on a wait during the most recent
  * call on ws (kernel id / wait site / block id are written to info[0..2] when info is

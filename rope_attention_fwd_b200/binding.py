@@ -51,6 +51,8 @@ def lib():
         L.rope_attn_loss.restype = ctypes.c_int
         L.rope_attn_bwd.argtypes = [P] + [vp] * 12 + [sz, vp]
         L.rope_attn_bwd.restype = ctypes.c_int
+        L.rope_attn_bwd_saved.argtypes = [P] + [vp] * 10 + [sz, vp]
+        L.rope_attn_bwd_saved.restype = ctypes.c_int
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -158,6 +160,21 @@ def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
         _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(),
         _stream(q.device)))
+    return dq, dk, dv, dalpha
+
+
+def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None, dv=None,
+                        dalpha=None):
+    """rope_attn_bwd from the table, Q~ and K~ the preceding rope_attn_fwd left in ws
+    (same problem, q, k and alpha; see include/rope_attn.h)."""
+    prob = _problem_of(v, causal, base)
+    dq = torch.empty_like(v) if dq is None else dq
+    dk = torch.empty_like(v) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dalpha = torch.empty_like(alpha) if dalpha is None else dalpha
+    _check("rope_attn_bwd_saved", lib().rope_attn_bwd_saved(
+        ctypes.byref(prob), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha), _ptr(dq),
+        _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(v.device)))
     return dq, dk, dv, dalpha
 
 

@@ -221,20 +221,32 @@ ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e, floa
   return RA_OK;
 }
 
-ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
-                        const void* o, const float* lse, const void* dO, const float* alpha,
-                        void* dq, void* dk, void* dv, float* dalpha, void* ws, size_t ws_bytes,
-                        void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Backward body shared by rope_attn_bwd (saved = false: clears the error word, builds the
+// table and rotates q, k into ws) and rope_attn_bwd_saved (saved = true: uses the table,
+// Q~ and K~ a previous forward left in ws and clears only the two max statistics).
+ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void* v,
+                   const void* o, const float* lse, const void* dO, const float* alpha,
+                   void* dq, void* dk, void* dv, float* dalpha, void* ws, size_t ws_bytes,
+                   void* stream, bool saved) {
   ra_status st = check_problem(p);
   if (st != RA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
-      !aligned16(dO) || !aligned16(alpha) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      !aligned16(dalpha))
+  if ((!saved && (!aligned16(q) || !aligned16(k))) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(lse) || !aligned16(dO) || !aligned16(alpha) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(dalpha))
     return RA_ERR_INVALID_ARG;
   if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(*p);
-  if ((st = prepare(p, q, k, alpha, ws, L, s)) != RA_OK) return st;
+  if (saved) {
+    // the two max statistics (words 8, 9 of the error region) start from zero
+    if (cudaMemsetAsync(at<uint8_t>(ws, L.err) + 32, 0, 8, s) != cudaSuccess) return RA_ERR_CUDA;
+  } else if ((st = prepare(p, q, k, alpha, ws, L, s)) != RA_OK) {
+    return st;
+  }
   float* delta = at<float>(ws, L.delta);
   float* dpart = at<float>(ws, L.dpart);
   const float2* table = at<float2>(ws, L.table);
@@ -251,8 +263,7 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
   } else {
     float* lse2 = at<float>(ws, L.lse2);
     uint32_t* stats = at<uint32_t>(ws, L.err) + 8;  // zeroed with the error word in prepare()
-    RA_LAUNCH(K_BWD_DELTA, s, launch_bwd_pre(*p, o, dO, lse, delta, lse2, stats, s));
-    RA_LAUNCH(K_BWD_DELTA, s, launch_vnorm_max(*p, v, stats + 1, s));
+    RA_LAUNCH(K_BWD_DELTA, s, launch_bwd_pre(*p, o, dO, v, lse, delta, lse2, stats, s));
     Sm100Maps maps;
     std::memset(&maps, 0, sizeof(maps));
     void* qt = at<void>(ws, L.qt);
@@ -270,6 +281,26 @@ ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const
   }
   RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
+                        const void* o, const float* lse, const void* dO, const float* alpha,
+                        void* dq, void* dk, void* dv, float* dalpha, void* ws, size_t ws_bytes,
+                        void* stream) {
+  return bwd_impl(p, q, k, v, o, lse, dO, alpha, dq, dk, dv, dalpha, ws, ws_bytes, stream,
+                  false);
+}
+
+ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
+                              const float* lse, const void* dO, const float* alpha, void* dq,
+                              void* dk, void* dv, float* dalpha, void* ws, size_t ws_bytes,
+                              void* stream) {
+  return bwd_impl(p, nullptr, nullptr, v, o, lse, dO, alpha, dq, dk, dv, dalpha, ws, ws_bytes,
+                  stream, true);
 }
 
 ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32_t info[3]) {

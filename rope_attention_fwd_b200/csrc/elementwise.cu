@@ -242,79 +242,118 @@ __device__ __forceinline__ void block_max_atomic(float v, uint32_t* dst) {
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(256)
-    bwd_pre_bf16_kernel(const uint2* __restrict__ o, const uint2* __restrict__ dO,
-                        const float* __restrict__ lse, float* __restrict__ deltap,
-                        float* __restrict__ lse2p, long long prow_count, int n, int npad,
-                        uint32_t* __restrict__ dmax) {
-  constexpr int LPR = D / 4, RPW = 32 / LPR;  // lanes per row, rows per warp
-  const int lane = threadIdx.x % 32;
-  const long long warps_total = (long long)gridDim.x * (blockDim.x / 32);
-  float mx = 0.f;
-  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-       wi * RPW < prow_count; wi += warps_total) {
-    const long long prow = wi * RPW + lane / LPR;
-    const long long bh = prow / npad;
-    const int i = (int)(prow % npad);
-    const bool live = prow < prow_count && i < n;
-    float acc = 0.f, sq = 0.f;
-    if (live) {
-      const long long idx = (bh * n + i) * LPR + lane % LPR;
-      uint2 a = o[idx], b = dO[idx];
-      const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
-      const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
-      const __nv_bfloat162 b0 = *reinterpret_cast<__nv_bfloat162*>(&b.x);
-      const __nv_bfloat162 b1 = *reinterpret_cast<__nv_bfloat162*>(&b.y);
-      acc = __low2float(a0) * __low2float(b0);
-      acc = fmaf(__high2float(a0), __high2float(b0), acc);
-      acc = fmaf(__low2float(a1), __low2float(b1), acc);
-      acc = fmaf(__high2float(a1), __high2float(b1), acc);
-      sq = __low2float(b0) * __low2float(b0);
-      sq = fmaf(__high2float(b0), __high2float(b0), sq);
-      sq = fmaf(__low2float(b1), __low2float(b1), sq);
-      sq = fmaf(__high2float(b1), __high2float(b1), sq);
-    }
+// The two block maxima in one reduction, each to its own fp32-bits word with one atomic.
+__device__ __forceinline__ void block_max2_atomic(float v0, float v1, uint32_t* dst0,
+                                                  uint32_t* dst1) {
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) {
-      acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    }
-    if (prow < prow_count && lane % LPR == 0) {
-      deltap[prow] = acc;
-      lse2p[prow] = live ? lse[bh * n + i] * 1.4426950408889634f : __int_as_float(0x7f800000);
-    }
-    mx = fmaxf(mx, sqrtf(sq));
+  for (int off = 16; off > 0; off >>= 1) {
+    v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, off));
+    v1 = fmaxf(v1, __shfl_xor_sync(0xffffffffu, v1, off));
   }
-  block_max_atomic(mx, dmax);
+  __shared__ float red2[2][32];
+  if (threadIdx.x % 32 == 0) {
+    red2[0][threadIdx.x / 32] = v0;
+    red2[1][threadIdx.x / 32] = v1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m0 = 0.f, m1 = 0.f;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) {
+      m0 = fmaxf(m0, red2[0][w]);
+      m1 = fmaxf(m1, red2[1][w]);
+    }
+    atomicMax(dst0, __float_as_uint(m0));
+    atomicMax(dst1, __float_as_uint(m1));
+  }
 }
 
-// max_j |v_j| over every row of V (bf16, d in {64, 128}) into *vmax (fp32 bits).
+// Backward preprocess of the bf16 path in one pass over O, dO and V (d in {64, 128}):
+//   Delta_i = rowsum(dO_i o O_i) and lse2_i = lse_i log2(e) over the padded rows
+//   (+inf past n, so that P = 0 there), max_i |dO_i| into stats[0] and max_j |v_j| into
+//   stats[1] (fp32 bits; one atomic max per block each).
+// A lane reads 16 bytes (8 elements) of a row, D/8 lanes per row, and each warp keeps
+// kPreUnroll row groups of loads in flight.
+constexpr int kPreUnroll = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256)
-    vnorm_max_bf16_kernel(const uint2* __restrict__ v, long long rows, uint32_t* __restrict__ vmax) {
-  constexpr int LPR = D / 4, RPW = 32 / LPR;
+    bwd_pre_bf16_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
+                        const uint4* __restrict__ v, const float* __restrict__ lse,
+                        float* __restrict__ deltap, float* __restrict__ lse2p,
+                        long long bh_count, int n, int npad, uint32_t* __restrict__ stats) {
+  constexpr int LPR = D / 8, RPW = 32 / LPR, U = kPreUnroll;  // lanes per row, rows per warp
   const int lane = threadIdx.x % 32;
   const long long warps_total = (long long)gridDim.x * (blockDim.x / 32);
-  float mx = 0.f;
-  for (long long wi = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-       wi * RPW < rows; wi += warps_total) {
-    const long long row = wi * RPW + lane / LPR;
-    float sq = 0.f;
-    if (row < rows) {
-      uint2 a = v[row * LPR + lane % LPR];
-      const __nv_bfloat162 a0 = *reinterpret_cast<__nv_bfloat162*>(&a.x);
-      const __nv_bfloat162 a1 = *reinterpret_cast<__nv_bfloat162*>(&a.y);
-      sq = __low2float(a0) * __low2float(a0);
-      sq = fmaf(__high2float(a0), __high2float(a0), sq);
-      sq = fmaf(__low2float(a1), __low2float(a1), sq);
-      sq = fmaf(__high2float(a1), __high2float(a1), sq);
+  const long long w0 = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  // Row counts stay below 2^32 (a bf16 tensor of 2^32 rows would not fit in device
+  // memory), so the (batch-head, row) split uses 32-bit division.
+  const long long prows = bh_count * npad, rows = bh_count * n;
+  float mdo = 0.f, mv = 0.f;
+  for (long long r0 = w0 * RPW * U; r0 < prows; r0 += warps_total * RPW * U) {
+    uint4 a[U], g[U];
+    uint32_t pbh[U], pi[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long prow = r0 + u * RPW + lane / LPR;
+      pbh[u] = (uint32_t)prow / (uint32_t)npad;
+      pi[u] = (uint32_t)prow - pbh[u] * (uint32_t)npad;
+      a[u] = g[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (prow < prows && pi[u] < (uint32_t)n) {
+        const long long idx = ((long long)pbh[u] * n + pi[u]) * LPR + lane % LPR;
+        a[u] = o[idx];
+        g[u] = dO[idx];
+      }
     }
 #pragma unroll
-    for (int off = LPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-    mx = fmaxf(mx, sqrtf(sq));
+    for (int u = 0; u < U; ++u) {
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+      const __nv_bfloat162* pg = reinterpret_cast<const __nv_bfloat162*>(&g[u]);
+      float acc = 0.f, sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(pa[e]), fg = __bfloat1622float2(pg[e]);
+        acc = fmaf(fa.x, fg.x, acc);
+        acc = fmaf(fa.y, fg.y, acc);
+        sq = fmaf(fg.x, fg.x, sq);
+        sq = fmaf(fg.y, fg.y, sq);
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) {
+        acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      }
+      const long long prow = r0 + u * RPW + lane / LPR;
+      if (prow < prows && lane % LPR == 0) {
+        deltap[prow] = acc;
+        lse2p[prow] = pi[u] < (uint32_t)n ? lse[(long long)pbh[u] * n + pi[u]] * 1.4426950408889634f
+                                          : __int_as_float(0x7f800000);
+      }
+      mdo = fmaxf(mdo, sqrtf(sq));
+    }
   }
-  block_max_atomic(mx, vmax);
+  for (long long r0 = w0 * RPW * U; r0 < rows; r0 += warps_total * RPW * U) {
+    uint4 a[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long row = r0 + u * RPW + lane / LPR;
+      a[u] = row < rows ? v[row * LPR + lane % LPR] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+      float sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(pa[e]);
+        sq = fmaf(fa.x, fa.x, sq);
+        sq = fmaf(fa.y, fa.y, sq);
+      }
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      mv = fmaxf(mv, sqrtf(sq));
+    }
+  }
+  block_max2_atomic(mdo, mv, stats, stats + 1);
 }
 
 // ---------------------------------------------------------------- dalpha final
@@ -412,28 +451,19 @@ cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, flo
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
-                           float* deltap, float* lse2p, uint32_t* stats, cudaStream_t s) {
+cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const void* v,
+                           const float* lse, float* deltap, float* lse2p, uint32_t* stats,
+                           cudaStream_t s) {
   const int npad = (int)padded_rows(p.n);
-  const long long prows = p.B * p.H * npad;
+  const long long bh = p.B * p.H;
   if (p.d == 64)
-    bwd_pre_bf16_kernel<64><<<kReduceBlocks, 256, 0, s>>>((const uint2*)o, (const uint2*)dO, lse,
-                                                          deltap, lse2p, prows, (int)p.n, npad,
-                                                          stats);
+    bwd_pre_bf16_kernel<64><<<kReduceBlocks, 256, 0, s>>>((const uint4*)o, (const uint4*)dO,
+                                                          (const uint4*)v, lse, deltap, lse2p,
+                                                          bh, (int)p.n, npad, stats);
   else
-    bwd_pre_bf16_kernel<128><<<kReduceBlocks, 256, 0, s>>>((const uint2*)o, (const uint2*)dO,
-                                                           lse, deltap, lse2p, prows, (int)p.n,
-                                                           npad, stats);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_vnorm_max(const ra_problem& p, const void* v, uint32_t* vmax,
-                             cudaStream_t s) {
-  const long long rows = p.B * p.H * p.n;
-  if (p.d == 64)
-    vnorm_max_bf16_kernel<64><<<kReduceBlocks, 256, 0, s>>>((const uint2*)v, rows, vmax);
-  else
-    vnorm_max_bf16_kernel<128><<<kReduceBlocks, 256, 0, s>>>((const uint2*)v, rows, vmax);
+    bwd_pre_bf16_kernel<128><<<kReduceBlocks, 256, 0, s>>>((const uint4*)o, (const uint4*)dO,
+                                                           (const uint4*)v, lse, deltap, lse2p,
+                                                           bh, (int)p.n, npad, stats);
   return cudaGetLastError();
 }
 

@@ -44,13 +44,12 @@ struct Sm100Maps {
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
-// Padded per-row vectors for the tensor-core backward: delta and lse * log2(e).
-// ... and max_i |dO_i| into stats[0] (fp32 bits, atomic max; stats zeroed by the caller).
-cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const float* lse,
-                           float* deltap, float* lse2p, uint32_t* stats, cudaStream_t s);
-// max_j |v_j| into *vmax (fp32 bits, atomic max; zeroed by the caller).
-cudaError_t launch_vnorm_max(const ra_problem& p, const void* v, uint32_t* vmax,
-                             cudaStream_t s);
+// Padded per-row vectors for the tensor-core backward, delta and lse * log2(e), plus
+// max_i |dO_i| into stats[0] and max_j |v_j| into stats[1] (fp32 bits, atomic max; stats
+// zeroed by the caller), in one pass over O, dO and V.
+cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, const void* v,
+                           const float* lse, float* deltap, float* lse2p, uint32_t* stats,
+                           cudaStream_t s);
 // stats: [0] max_i |dO_i|, [1] max_j |v_j| (fp32 bits) for the fp16 scale of dS.
 cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,

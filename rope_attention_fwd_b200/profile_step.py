@@ -32,7 +32,7 @@ def main():
     def step():
         o, lse = rb.rope_attn_fwd(q, k, v, alpha, a.base, a.causal, ws=ws)
         L, dO = rb.rope_attn_loss(o, e, ws=ws)
-        return rb.rope_attn_bwd(q, k, v, o, lse, dO, alpha, a.base, a.causal, ws=ws)
+        return rb.rope_attn_bwd_saved(v, o, lse, dO, alpha, a.base, a.causal, ws)
 
     for _ in range(a.warmup):
         step()

@@ -52,6 +52,25 @@ def test_deterministic(dtype):
     assert a["L"] == b["L"]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_saved_matches_bwd(dtype, causal):
+    """rope_attn_bwd_saved after rope_attn_fwd on the same workspace (the saved-for-backward
+    table, Q~ and K~) gives the gradients of rope_attn_bwd bit for bit."""
+    from rope_attention_fwd_b200 import binding as rb
+    wl = small_workload(2, 3, 257, 128 if dtype == "bf16" else 64, dtype, causal, seed=21)
+    inp = make(wl)
+    q, k, v, e, alpha = (getattr(inp, x).cuda() for x in ("q", "k", "v", "e", "alpha"))
+    ws = rb.workspace(rb.problem(wl.B, wl.H, wl.n, wl.d, q.dtype, causal, wl.base), "cuda")
+    o, lse = rb.rope_attn_fwd(q, k, v, alpha, wl.base, causal, ws=ws)
+    _, dO = rb.rope_attn_loss(o, e, ws=ws)
+    saved = rb.rope_attn_bwd_saved(v, o, lse, dO, alpha, wl.base, causal, ws)
+    full = rb.rope_attn_bwd(q, k, v, o, lse, dO, alpha, wl.base, causal, ws=ws)
+    assert rb.rope_attn_device_status(ws)[0] == 0
+    for a, b, name in zip(saved, full, ("dq", "dk", "dv", "dalpha")):
+        assert torch.equal(a, b), name
+
+
 def test_bf16_many_heads_and_batches():
     wl = small_workload(3, 5, 160, 64, "bf16", True, seed=5)
     inp = make(wl)

@@ -34,6 +34,14 @@ M = d/2 frequency bands:
     by every head ("LeRoPE", Escolhas de Design Principais: one set of d/2
     frequencies shared across all layers and heads; log-space parametrisation).
 
+Variants ("LeRoPE", Configuracao Experimental and Ablacao):
+- fixed_bands = f: the f slowest bands (m >= M - f) keep theta_hat_m = 0, i.e. are not
+  rotated -- partial RoPE, the p-RoPE baseline with p = 1 - f/M (p = 0.75 drops the
+  slowest 25% of bands).  Their dalpha is 0: theta_hat_m does not depend on alpha_m.
+- frozen frequencies: alpha given, no dalpha (the backward's step 8 skipped).
+- the optimiser step for alpha ("LeRoPE", Escolhas de Design Principais: no weight decay
+  on the LeRoPE parameters, their gradient clipped separately): :func:`alpha_adam_step`.
+
 A second, independent formula for dalpha -- the derivative of the real part of
 the DTFT of the offset-aggregated gradient signal ("LeRoPE", Analise Teorica)
 -- is :func:`dalpha_offset_dtft`.
@@ -48,12 +56,15 @@ import numpy as np
 # --------------------------------------------------------------------------
 # step 1-2: frequencies, angles, band rotation
 # --------------------------------------------------------------------------
-def frequencies(d, base, alpha):
-    """theta_m = base^(-2m/d) and theta_hat_m = exp(alpha_m) theta_m, m < d/2."""
+def frequencies(d, base, alpha, fixed_bands=0):
+    """theta_m = base^(-2m/d) and theta_hat_m = exp(alpha_m) theta_m, m < d/2; the
+    fixed_bands slowest bands (m >= d/2 - fixed_bands) get theta_hat_m = 0."""
     M = d // 2
     m = np.arange(M, dtype=np.float64)
     theta = np.power(float(base), -2.0 * m / d)
     theta_hat = np.exp(np.asarray(alpha, dtype=np.float64)) * theta
+    if fixed_bands:
+        theta_hat = np.where(m >= M - fixed_bands, 0.0, theta_hat)
     return theta, theta_hat
 
 
@@ -185,10 +196,11 @@ def head_matrices(qt, kt, v, do, causal):
 # --------------------------------------------------------------------------
 # public API over [B, H, n, d]
 # --------------------------------------------------------------------------
-def forward(q, k, v, alpha, base, causal, pairing="interleaved", offset=0, block=512):
+def forward(q, k, v, alpha, base, causal, pairing="interleaved", offset=0, block=512,
+            fixed_bands=0):
     """O [B,H,n,d] and lse [B,H,n] (natural log) in float64."""
     B, H, n, d = q.shape
-    _, th = frequencies(d, base, alpha)
+    _, th = frequencies(d, base, alpha, fixed_bands)
     phi = angles(n, th, offset)
     o = np.empty((B, H, n, d))
     lse = np.empty((B, H, n))
@@ -213,10 +225,10 @@ def band_torque(g, x, pairing="interleaved"):
 
 
 def backward(q, k, v, do, alpha, base, causal, pairing="interleaved", offset=0, block=512,
-             return_rotated=False):
+             return_rotated=False, fixed_bands=0):
     """dQ, dK, dV [B,H,n,d] and dalpha [d/2] in float64 for upstream gradient dO."""
     B, H, n, d = q.shape
-    _, th = frequencies(d, base, alpha)
+    _, th = frequencies(d, base, alpha, fixed_bands)
     phi = angles(n, th, offset)
     pos = np.arange(n, dtype=np.float64) + offset
     dq = np.empty((B, H, n, d))
@@ -286,3 +298,27 @@ def dalpha_offset_dtft(q, k, v, do, alpha, base, causal, pairing="interleaved"):
                 dP = np.real(np.sum(1j * offs * g * np.exp(1j * offs * th[m])))
                 out[m] += th[m] * dP
     return out
+
+
+# --------------------------------------------------------------------------
+# the optimiser step for alpha
+# --------------------------------------------------------------------------
+def alpha_adam_step(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999, eps=1e-8,
+                    clip_norm=1.0):
+    """One Adam step for the LeRoPE log-frequencies with their own gradient clipping and no
+    weight decay ("LeRoPE", Escolhas de Design Principais: Otimizacao).  The page names
+    neither the optimiser nor the clipping rule; this is the plainest reading: dalpha is
+    scaled to L2 norm clip_norm when its norm exceeds it (clip_norm <= 0: no clipping),
+    then the Adam update (first and second moments m1, m2 with bias correction at the
+    1-based step t) is applied with weight decay 0.  Returns (alpha, m1, m2)."""
+    g = np.asarray(dalpha, dtype=np.float64)
+    if clip_norm > 0:
+        nrm = float(np.sqrt(np.sum(g * g)))
+        if nrm > clip_norm:
+            g = g * (clip_norm / nrm)
+    m1 = beta1 * np.asarray(m1, dtype=np.float64) + (1.0 - beta1) * g
+    m2 = beta2 * np.asarray(m2, dtype=np.float64) + (1.0 - beta2) * g * g
+    m_hat = m1 / (1.0 - beta1 ** step)
+    v_hat = m2 / (1.0 - beta2 ** step)
+    alpha = np.asarray(alpha, dtype=np.float64) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return alpha, m1, m2

@@ -311,3 +311,99 @@ def test_row_and_column_restricted_backward(causal):
     ck, cv = ref.head_backward_cols(qt, kt, v[0, 0], do, lse, delta, rows, causal)
     np.testing.assert_allclose(ck, dkt[rows], atol=1e-13)
     np.testing.assert_allclose(cv, dv[rows], atol=1e-13)
+
+
+# ---------------------------------------------------------------- variants: p-RoPE fixed bands
+def test_fixed_bands_all_is_plain_attention():
+    """Every band fixed (no rotation at all) is plain softmax attention: torch's
+    scaled_dot_product_attention on the unrotated q, k; and dalpha is exactly 0."""
+    B, H, n, d = 1, 2, 21, 8
+    q, k, v, e, alpha, base = rand_problem(41, B, H, n, d, alpha_scale=0.5)
+    o, _ = ref.forward(q, k, v, alpha, base, True, fixed_bands=d // 2)
+    sd = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v), is_causal=True).numpy()
+    np.testing.assert_allclose(o, sd, atol=1e-13)
+    _, do = ref.loss(o, e)
+    assert np.all(ref.backward(q, k, v, do, alpha, base, True, fixed_bands=d // 2)[3] == 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fixed_bands_autograd(causal):
+    """p-RoPE (the slowest f bands unrotated) against an independent complex-multiplication
+    forward with those bands' frequency set to zero, differentiated by autograd: the fixed
+    bands get dalpha = 0 (their frequency does not depend on alpha), the others agree."""
+    B, H, n, d, f = 1, 2, 29, 16, 2
+    q, k, v, e, alpha, base = rand_problem(43, B, H, n, d, alpha_scale=0.6, base=300.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal, block=8, fixed_bands=f)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    ta = torch.tensor(alpha, requires_grad=True)
+    m = torch.arange(d // 2, dtype=torch.float64)
+    keep = (m < d // 2 - f).to(torch.float64)
+    th = torch.exp(ta) * base ** (-2.0 * m / d) * keep
+    pos = torch.arange(n, dtype=torch.float64)
+    qr, kr = _torch_rope_complex(tq, pos, th), _torch_rope_complex(tk, pos, th)
+    s = qr @ kr.transpose(-1, -2) / math.sqrt(d)
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ tv
+    L = 0.5 * ((o - torch.tensor(e)) ** 2).sum()
+    L.backward()
+    np.testing.assert_allclose(o.detach().numpy(), r["o"], atol=1e-12)
+    for g, key in ((tq.grad, "dq"), (tk.grad, "dk"), (tv.grad, "dv")):
+        np.testing.assert_allclose(g.numpy(), r[key], atol=1e-11)
+    np.testing.assert_allclose(ta.grad.numpy(), r["dalpha"], rtol=1e-10, atol=1e-11)
+    assert np.all(r["dalpha"][d // 2 - f:] == 0.0)
+
+
+def test_fixed_bands_limit_of_vanishing_frequency():
+    """Fixing a band equals sending its alpha to -inf: O and the other bands' dalpha match
+    alpha_m = -80 (theta_hat ~ 1.8e-35) to rounding."""
+    B, H, n, d, f = 1, 1, 24, 16, 3
+    q, k, v, e, alpha, base = rand_problem(47, B, H, n, d, alpha_scale=0.5)
+    a2 = alpha.copy()
+    a2[d // 2 - f:] = -80.0
+    r1 = ref.forward_backward(q, k, v, e, alpha, base, True, fixed_bands=f)
+    r2 = ref.forward_backward(q, k, v, e, a2, base, True)
+    for key in ("o", "dq", "dk", "dv"):
+        np.testing.assert_allclose(r1[key], r2[key], atol=1e-13)
+    np.testing.assert_allclose(r1["dalpha"][: d // 2 - f], r2["dalpha"][: d // 2 - f],
+                               rtol=1e-10)
+
+
+# ---------------------------------------------------------------- variants: the alpha optimiser step
+def test_alpha_adam_matches_torch_adam_with_own_clipping():
+    """Three steps of the oracle's alpha update against torch.optim.Adam (weight_decay=0)
+    fed the gradient clipped by torch.nn.utils.clip_grad_norm_.  torch clips by
+    max_norm / (norm + 1e-6), the oracle to exactly max_norm; that moves alpha by ~1e-11
+    here, while a wrong moment, sign or bias correction moves it by ~1e-3 (lr = 3e-3)."""
+    M = 32
+    rng = np.random.default_rng(53)
+    alpha = 0.2 * rng.standard_normal(M)
+    p = torch.nn.Parameter(torch.tensor(alpha))
+    opt = torch.optim.Adam([p], lr=3e-3, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.0)
+    m1 = np.zeros(M)
+    m2 = np.zeros(M)
+    a = alpha.copy()
+    for t in (1, 2, 3):
+        g = (2.0 ** t) * rng.standard_normal(M)   # norms above and below the clip
+        a, m1, m2 = ref.alpha_adam_step(a, g, m1, m2, t, 3e-3, 0.9, 0.95, 1e-8, clip_norm=4.0)
+        opt.zero_grad()
+        p.grad = torch.tensor(g)
+        torch.nn.utils.clip_grad_norm_([p], 4.0)
+        opt.step()
+        np.testing.assert_allclose(a, p.detach().numpy(), rtol=0, atol=1e-9)
+
+
+def test_alpha_adam_closed_forms():
+    """First step: the bias-corrected moments are g and g^2, so each alpha_m moves by
+    -lr g_m / (|g_m| + eps); the first moment after clipping is (1 - beta1) g clip / |g|."""
+    M = 16
+    rng = np.random.default_rng(59)
+    g = rng.standard_normal(M) * 10.0
+    a, m1, _ = ref.alpha_adam_step(np.zeros(M), g, np.zeros(M), np.zeros(M), 1, 0.01,
+                                   clip_norm=0.0)
+    np.testing.assert_allclose(a, -0.01 * g / (np.abs(g) + 1e-8), rtol=1e-12)
+    nrm = np.linalg.norm(g)
+    _, m1, _ = ref.alpha_adam_step(np.zeros(M), g, np.zeros(M), np.zeros(M), 1, 0.01,
+                                   clip_norm=1.0)
+    np.testing.assert_allclose(m1, 0.1 * g / nrm, rtol=1e-12)

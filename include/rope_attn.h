@@ -79,6 +79,11 @@ typedef struct {
     int32_t dtype;       /* ra_dtype of Q, K, V, O, E, dO, dQ, dK, dV          */
     int32_t causal;      /* 1: key j is visible to query i only when j <= i     */
     double base;         /* RoPE base b > 0 (theta_m = b^(-2m/d))               */
+    int32_t fixed_bands; /* 0..d/2: the slowest bands m >= d/2 - fixed_bands are not
+                            rotated (theta_hat_m = 0, dalpha_m = 0): partial RoPE, the
+                            p-RoPE baseline of "LeRoPE" (Configuracao Experimental) with
+                            p = 1 - fixed_bands / (d/2); 0 = every band rotates        */
+    int32_t reserved;    /* must be 0                                             */
 } ra_problem;
 
 /* Bytes of workspace the calls below need for problem *p (0 if *p is invalid).
@@ -121,6 +126,24 @@ ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
                               const float* lse, const void* dO, const float* alpha,
                               void* dq, void* dk, void* dv, float* dalpha,
                               void* ws, size_t ws_bytes, void* stream);
+
+/* ---- the optimiser step for the learned frequencies ---------------------------
+ * "LeRoPE" (Escolhas de Design Principais: Otimizacao) trains alpha without weight decay
+ * and clips its gradient separately from the model's.  The page names neither the
+ * optimiser nor the clipping rule; this is Adam with weight decay 0 after scaling dalpha
+ * to L2 norm clip_norm when its norm exceeds it (clip_norm <= 0: no clipping). */
+typedef struct {
+    float lr, beta1, beta2, eps;
+    float clip_norm;     /* L2 norm bound for dalpha; <= 0 disables the clipping        */
+    int32_t step;        /* 1-based step t (bias corrections 1 - beta^t)                 */
+} ra_adam;
+
+/* alpha, m1 (first moment), m2 (second moment): count fp32 each, updated in place from
+ * dalpha (count fp32), on `stream`.  All four device pointers 16-byte aligned; count in
+ * 1..2^20; m1 = m2 = 0 before the first step.  RA_ERR_INVALID_ARG on a bad argument
+ * (nothing launched). */
+ra_status rope_attn_alpha_adam(const ra_adam* opt, int64_t count, float* alpha,
+                               const float* dalpha, float* m1, float* m2, void* stream);
 
 /* Synchronises `stream`, reads and clears the device error word in ws.
  * Returns RA_OK; RA_ERR_TIMEOUT if a kernel gave up on a wait during the most recent

@@ -22,7 +22,13 @@ STATUS = {0: "RA_OK", 1: "RA_ERR_INVALID_ARG", 2: "RA_ERR_UNSUPPORTED", 3: "RA_E
 class RaProblem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("n", ctypes.c_int64),
                 ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
-                ("base", ctypes.c_double)]
+                ("base", ctypes.c_double), ("fixed_bands", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+class RaAdam(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("clip_norm", ctypes.c_float), ("step", ctypes.c_int32)]
 
 
 class RopeAttnError(RuntimeError):
@@ -53,6 +59,9 @@ def lib():
         L.rope_attn_bwd.restype = ctypes.c_int
         L.rope_attn_bwd_saved.argtypes = [P] + [vp] * 10 + [sz, vp]
         L.rope_attn_bwd_saved.restype = ctypes.c_int
+        L.rope_attn_alpha_adam.argtypes = [ctypes.POINTER(RaAdam), ctypes.c_int64, vp, vp, vp, vp,
+                                           vp]
+        L.rope_attn_alpha_adam.restype = ctypes.c_int
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -70,15 +79,17 @@ def lib():
     return _lib
 
 
-def problem(B, H, n, d, dtype, causal, base):
+def problem(B, H, n, d, dtype, causal, base, fixed_bands=0):
+    """fixed_bands: the slowest bands left unrotated (partial RoPE; 0 = all rotate)."""
     if isinstance(dtype, torch.dtype):
         dtype = _DTYPE[dtype]
-    return RaProblem(int(B), int(H), int(n), int(d), int(dtype), int(bool(causal)), float(base))
+    return RaProblem(int(B), int(H), int(n), int(d), int(dtype), int(bool(causal)), float(base),
+                     int(fixed_bands), 0)
 
 
-def _problem_of(q, causal, base):
+def _problem_of(q, causal, base, fixed_bands=0):
     B, H, n, d = q.shape
-    return problem(B, H, n, d, q.dtype, causal, base)
+    return problem(B, H, n, d, q.dtype, causal, base, fixed_bands)
 
 
 def _ptr(t):
@@ -106,9 +117,9 @@ def workspace(prob, device):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None):
+def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None, fixed_bands=0):
     """(o, lse) = softmax(Q~ K~^T / sqrt(d)) V and its row log-sum-exp."""
-    prob = _problem_of(q, causal, base)
+    prob = _problem_of(q, causal, base, fixed_bands)
     B, H, n, d = q.shape
     if ws is None:
         ws = workspace(prob, q.device)
@@ -120,10 +131,10 @@ def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None):
     return o, lse
 
 
-def rope_attn_fwd_noalloc(q, k, v, alpha, base, causal, o=None, lse=None):
+def rope_attn_fwd_noalloc(q, k, v, alpha, base, causal, o=None, lse=None, fixed_bands=0):
     """rope_attn_fwd without a workspace: scratch comes from the library's static
     RA_NOALLOC_SCRATCH_BYTES device array (problems that need more are rejected)."""
-    prob = _problem_of(q, causal, base)
+    prob = _problem_of(q, causal, base, fixed_bands)
     B, H, n, d = q.shape
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -147,15 +158,19 @@ def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
 
 
 def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk=None, dv=None,
-                  dalpha=None):
-    """(dq, dk, dv, dalpha) of L for upstream gradient dO."""
-    prob = _problem_of(q, causal, base)
+                  dalpha=None, fixed_bands=0, frozen_alpha=False):
+    """(dq, dk, dv, dalpha) of L for upstream gradient dO.  frozen_alpha: the frequencies
+    are not trained; no dalpha is computed and None is returned in its place."""
+    prob = _problem_of(q, causal, base, fixed_bands)
     if ws is None:
         ws = workspace(prob, q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    dalpha = torch.empty_like(alpha) if dalpha is None else dalpha
+    if frozen_alpha:
+        dalpha = None
+    elif dalpha is None:
+        dalpha = torch.empty_like(alpha)
     _check("rope_attn_bwd", lib().rope_attn_bwd(
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
         _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(),
@@ -164,18 +179,32 @@ def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk
 
 
 def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None, dv=None,
-                        dalpha=None):
+                        dalpha=None, fixed_bands=0, frozen_alpha=False):
     """rope_attn_bwd from the table, Q~ and K~ the preceding rope_attn_fwd left in ws
     (same problem, q, k and alpha; see include/rope_attn.h)."""
-    prob = _problem_of(v, causal, base)
+    prob = _problem_of(v, causal, base, fixed_bands)
     dq = torch.empty_like(v) if dq is None else dq
     dk = torch.empty_like(v) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    dalpha = torch.empty_like(alpha) if dalpha is None else dalpha
+    if frozen_alpha:
+        dalpha = None
+    elif dalpha is None:
+        dalpha = torch.empty_like(alpha)
     _check("rope_attn_bwd_saved", lib().rope_attn_bwd_saved(
         ctypes.byref(prob), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha), _ptr(dq),
         _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(v.device)))
     return dq, dk, dv, dalpha
+
+
+def rope_attn_alpha_adam(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999, eps=1e-8,
+                         clip_norm=1.0):
+    """One in-place Adam step (weight decay 0) of the fp32 device tensors alpha, m1, m2 from
+    dalpha clipped to L2 norm clip_norm (clip_norm <= 0: no clipping); step is 1-based."""
+    opt = RaAdam(float(lr), float(beta1), float(beta2), float(eps), float(clip_norm), int(step))
+    _check("rope_attn_alpha_adam", lib().rope_attn_alpha_adam(
+        ctypes.byref(opt), alpha.numel(), _ptr(alpha), _ptr(dalpha), _ptr(m1), _ptr(m2),
+        _stream(alpha.device)))
+    return alpha, m1, m2
 
 
 def rope_attn_device_status(ws):

@@ -78,6 +78,8 @@ ra_status check_problem(const ra_problem* p) {
   if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
   if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
   if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
+  if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 || p->reserved != 0)
+    return RA_ERR_INVALID_ARG;
   if (p->d > 128) return RA_ERR_UNSUPPORTED;
   if (p->dtype == RA_BF16 && p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
   return RA_OK;
@@ -234,9 +236,11 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
                    void* stream, bool saved) {
   ra_status st = check_problem(p);
   if (st != RA_OK) return st;
+  // dalpha may be null: frozen frequencies, no frequency gradient (its partials and the
+  // final reduction are skipped)
   if ((!saved && (!aligned16(q) || !aligned16(k))) || !aligned16(v) || !aligned16(o) ||
       !aligned16(lse) || !aligned16(dO) || !aligned16(alpha) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || !aligned16(dalpha))
+      !aligned16(dk) || !aligned16(dv) || (dalpha && !aligned16(dalpha)))
     return RA_ERR_INVALID_ARG;
   if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -248,7 +252,7 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
     return st;
   }
   float* delta = at<float>(ws, L.delta);
-  float* dpart = at<float>(ws, L.dpart);
+  float* dpart = dalpha ? at<float>(ws, L.dpart) : nullptr;
   const float2* table = at<float2>(ws, L.table);
   if (p->dtype == RA_F32) {
     RA_LAUNCH(K_BWD_DELTA, s, launch_delta(*p, o, dO, delta, s));
@@ -279,7 +283,7 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
     RA_LAUNCH(K_BWD_DQ_SM100, s,
               launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
   }
-  RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
+  if (dalpha) RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;
 }
 
@@ -301,6 +305,24 @@ ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
                               void* stream) {
   return bwd_impl(p, nullptr, nullptr, v, o, lse, dO, alpha, dq, dk, dv, dalpha, ws, ws_bytes,
                   stream, true);
+}
+
+ra_status rope_attn_alpha_adam(const ra_adam* opt, int64_t count, float* alpha,
+                               const float* dalpha, float* m1, float* m2, void* stream) {
+  if (!opt || count < 1 || count > (int64_t(1) << 20)) return RA_ERR_INVALID_ARG;
+  if (!aligned16(alpha) || !aligned16(dalpha) || !aligned16(m1) || !aligned16(m2))
+    return RA_ERR_INVALID_ARG;
+  if (!(opt->lr >= 0.f) || !(opt->beta1 >= 0.f && opt->beta1 < 1.f) ||
+      !(opt->beta2 >= 0.f && opt->beta2 < 1.f) || !(opt->eps > 0.f) || opt->step < 1 ||
+      !std::isfinite(opt->clip_norm))
+    return RA_ERR_INVALID_ARG;
+  const float bc1 = (float)(1.0 - std::pow((double)opt->beta1, (double)opt->step));
+  const float bc2 = (float)(1.0 - std::pow((double)opt->beta2, (double)opt->step));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_alpha_adam(alpha, dalpha, m1, m2, count, opt->lr, opt->beta1, opt->beta2, opt->eps,
+                        opt->clip_norm, bc1, bc2, s) != cudaSuccess)
+    return RA_ERR_CUDA;
+  return RA_OK;
 }
 
 ra_status rope_attn_device_status(void* ws, size_t ws_bytes, void* stream, int32_t info[3]) {

@@ -158,7 +158,7 @@ __device__ __forceinline__ void write_partial(const float (&tq)[4], float* red, 
   for (int mb = threadIdx.x; mb < M; mb += blockDim.x) {
     float s = 0.f;
     for (int w = 0; w < kWarps; ++w) s += red[w * M + mb];
-    dst[mb] = s;
+    if (dst) dst[mb] = s;  // null: frozen frequencies, no dalpha
   }
 }
 
@@ -235,8 +235,9 @@ __global__ void __launch_bounds__(256)
                  dq + (bh * n + i) * d, d, lane, tq);
   }
   const long long ntile = (n + kRows - 1) / kRows;
-  write_partial(tq, red, dpart + ((0 * gridDim.y + bh) * ntile + blockIdx.x) * (d / 2), d, warp,
-                lane);
+  write_partial(tq, red,
+                dpart ? dpart + ((0 * gridDim.y + bh) * ntile + blockIdx.x) * (d / 2) : nullptr,
+                d, warp, lane);
 }
 
 __global__ void __launch_bounds__(256)
@@ -326,8 +327,9 @@ __global__ void __launch_bounds__(256)
                  dk + (bh * n + j) * d, d, lane, tq);
   }
   const long long ntile = (n + kRows - 1) / kRows;
-  write_partial(tq, red, dpart + ((1 * gridDim.y + bh) * ntile + blockIdx.x) * (d / 2), d, warp,
-                lane);
+  write_partial(tq, red,
+                dpart ? dpart + ((1 * gridDim.y + bh) * ntile + blockIdx.x) * (d / 2) : nullptr,
+                d, warp, lane);
 }
 
 }  // namespace

@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            half);
       softmax_group_sync();
       const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      if (threadIdx.x < 128)
+      if (dpart != nullptr && threadIdx.x < 128)
         write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
                                  ntile64, t);
     }
@@ -848,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            half);
       softmax_group_sync();
       const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      if (threadIdx.x < 128)
+      if (dpart != nullptr && threadIdx.x < 128)
         write_dalpha_partials<D>(red, dpart + ((size_t)(0 * BH + bh) * ntile64) * (D / 2),
                                  qtile, ntile64, t);
     }

@@ -39,17 +39,20 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-__device__ __forceinline__ double theta_hat(const float* alpha, int m, int d, double base) {
+// theta_hat_m, or 0 for the fixed (unrotated) bands m >= mrot.
+__device__ __forceinline__ double theta_hat(const float* alpha, int m, int d, double base,
+                                            int mrot) {
+  if (m >= mrot) return 0.0;
   return exp((double)alpha[m]) * pow(base, -2.0 * (double)m / (double)d);
 }
 
 // ---------------------------------------------------------------- table
 __global__ void rope_table_kernel(const float* __restrict__ alpha, float2* __restrict__ table,
-                                  int n, int M, int d, double base) {
+                                  int n, int M, int d, double base, int mrot) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)n * M) return;
   const int p = (int)(idx / M), m = (int)(idx % M);
-  const double phi = (double)p * theta_hat(alpha, m, d, base);
+  const double phi = (double)p * theta_hat(alpha, m, d, base, mrot);
   double s, c;
   sincos(phi, &s, &c);
   table[idx] = make_float2((float)c, (float)s);
@@ -360,7 +363,8 @@ __global__ void __launch_bounds__(256)
 // One block per band m: fixed-order fp64 sum of the `count` partials part[i * M + m].
 __global__ void __launch_bounds__(256)
     dalpha_final_kernel(const float* __restrict__ part, const float* __restrict__ alpha,
-                        float* __restrict__ dalpha, long long count, int M, int d, double base) {
+                        float* __restrict__ dalpha, long long count, int M, int d, double base,
+                        int mrot) {
   const int m = blockIdx.x;
   double acc = 0.0;
   for (long long i = threadIdx.x; i < count; i += 256) acc += (double)part[i * M + m];
@@ -371,7 +375,38 @@ __global__ void __launch_bounds__(256)
     if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) dalpha[m] = (float)(theta_hat(alpha, m, d, base) * red[0]);
+  if (threadIdx.x == 0) dalpha[m] = (float)(theta_hat(alpha, m, d, base, mrot) * red[0]);
+}
+
+// ---------------------------------------------------------------- alpha optimiser step
+// One Adam step for the LeRoPE log-frequencies with their own gradient clipping and no
+// weight decay ("LeRoPE", Escolhas de Design Principais: Otimizacao): g = dalpha scaled to
+// L2 norm clip when its norm exceeds clip (the norm is a fixed-order fp64 reduction), then
+// m1 = b1 m1 + (1 - b1) g, m2 = b2 m2 + (1 - b2) g^2 and
+// alpha -= lr (m1 / bc1) / (sqrt(m2 / bc2) + eps), bc = 1 - b^t.  One block.
+__global__ void __launch_bounds__(256)
+    alpha_adam_kernel(float* __restrict__ alpha, const float* __restrict__ dalpha,
+                      float* __restrict__ m1, float* __restrict__ m2, long long count, float lr,
+                      float b1, float b2, float eps, float clip, float bc1, float bc2) {
+  double ss = 0.0;
+  for (long long i = threadIdx.x; i < count; i += 256) ss += (double)dalpha[i] * dalpha[i];
+  __shared__ double red[256];
+  red[threadIdx.x] = ss;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double nrm = sqrt(red[0]);
+  const float scale = (clip > 0.f && nrm > (double)clip) ? (float)((double)clip / nrm) : 1.f;
+  for (long long i = threadIdx.x; i < count; i += 256) {
+    const float g = dalpha[i] * scale;
+    const float a = b1 * m1[i] + (1.f - b1) * g;
+    const float b = b2 * m2[i] + (1.f - b2) * g * g;
+    m1[i] = a;
+    m2[i] = b;
+    alpha[i] -= lr * (a / bc1) / (sqrtf(b / bc2) + eps);
+  }
 }
 
 // ================================================================ launchers
@@ -381,7 +416,7 @@ cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table,
   const long long total = p.n * M;
   const int threads = 256;
   rope_table_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(
-      alpha, table, (int)p.n, M, (int)p.d, p.base);
+      alpha, table, (int)p.n, M, (int)p.d, p.base, M - p.fixed_bands);
   return cudaGetLastError();
 }
 
@@ -467,12 +502,21 @@ cudaError_t launch_bwd_pre(const ra_problem& p, const void* o, const void* dO, c
   return cudaGetLastError();
 }
 
+cudaError_t launch_alpha_adam(float* alpha, const float* dalpha, float* m1, float* m2,
+                              long long count, float lr, float b1, float b2, float eps,
+                              float clip, float bc1, float bc2, cudaStream_t s) {
+  alpha_adam_kernel<<<1, 256, 0, s>>>(alpha, dalpha, m1, m2, count, lr, b1, b2, eps, clip, bc1,
+                                      bc2);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dalpha_final(const ra_problem& p, const float* part, const float* alpha,
                                 float* dalpha, cudaStream_t s) {
   const int M = (int)(p.d / 2);
   const long long ntile = (p.n + kDalphaRows - 1) / kDalphaRows;
   const long long count = 2 * p.B * p.H * ntile;
-  dalpha_final_kernel<<<M, 256, 0, s>>>(part, alpha, dalpha, count, M, (int)p.d, p.base);
+  dalpha_final_kernel<<<M, 256, 0, s>>>(part, alpha, dalpha, count, M, (int)p.d, p.base,
+                                        M - p.fixed_bands);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,10 @@ cudaError_t launch_loss_partial(const ra_problem& p, const void* o, const void* 
 cudaError_t launch_loss_final(const double* part, float* L, cudaStream_t s);
 cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, float* delta,
                          cudaStream_t s);
+// One Adam step for alpha with dalpha clipped to L2 norm clip first (one block).
+cudaError_t launch_alpha_adam(float* alpha, const float* dalpha, float* m1, float* m2,
+                              long long count, float lr, float b1, float b2, float eps,
+                              float clip, float bc1, float bc2, cudaStream_t s);
 cudaError_t launch_dalpha_final(const ra_problem& p, const float* part, const float* alpha,
                                 float* dalpha, cudaStream_t s);
 

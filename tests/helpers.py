@@ -45,19 +45,20 @@ def check_status(ws):
     assert code == 0, (rb.STATUS.get(code, code), info)
 
 
-def gpu_run(inp, device="cuda", ws=None):
+def gpu_run(inp, device="cuda", ws=None, fixed_bands=0):
     """fwd -> loss -> bwd through the C ABI; returns float64 numpy results."""
     wl = inp.wl
     t = gpu_inputs(inp, device)
     if ws is None:
         ws = rb.workspace(rb.problem(wl.B, wl.H, wl.n, wl.d, t["q"].dtype, wl.causal, wl.base),
                           device)
-    o, lse = rb.rope_attn_fwd(t["q"], t["k"], t["v"], t["alpha"], wl.base, wl.causal, ws=ws)
+    o, lse = rb.rope_attn_fwd(t["q"], t["k"], t["v"], t["alpha"], wl.base, wl.causal, ws=ws,
+                              fixed_bands=fixed_bands)
     check_status(ws)
     L, dO = rb.rope_attn_loss(o, t["e"], ws=ws, causal=wl.causal, base=wl.base)
     check_status(ws)
     dq, dk, dv, dalpha = rb.rope_attn_bwd(t["q"], t["k"], t["v"], o, lse, dO, t["alpha"],
-                                          wl.base, wl.causal, ws=ws)
+                                          wl.base, wl.causal, ws=ws, fixed_bands=fixed_bands)
     check_status(ws)
     return dict(o=to64(o), lse=to64(lse), L=float(L.item()), do=to64(dO), dq=to64(dq),
                 dk=to64(dk), dv=to64(dv), dalpha=to64(dalpha))
@@ -71,7 +72,7 @@ def gpu_fwd(inp, device="cuda"):
     return dict(o=to64(o), lse=to64(lse))
 
 
-def oracle_run(inp):
+def oracle_run(inp, fixed_bands=0):
     """Oracle results, plus `dalpha_noise`: the bf16 rounding-noise scale of dalpha.
 
     Each weighted torque term w_p <dX~_pm, J x~_pm> of the dalpha sum is perturbed by
@@ -82,11 +83,11 @@ def oracle_run(inp):
     """
     wl = inp.wl
     q, k, v, e, al = (inp.f64(x) for x in ("q", "k", "v", "e", "alpha"))
-    o, lse = ref.forward(q, k, v, al, wl.base, wl.causal)
+    o, lse = ref.forward(q, k, v, al, wl.base, wl.causal, fixed_bands=fixed_bands)
     L, do = ref.loss(o, e)
     dq, dk, dv, dalpha, extra = ref.backward(q, k, v, do, al, wl.base, wl.causal,
-                                             return_rotated=True)
-    _, th = ref.frequencies(wl.d, wl.base, al)
+                                             return_rotated=True, fixed_bands=fixed_bands)
+    _, th = ref.frequencies(wl.d, wl.base, al, fixed_bands)
     w2 = (np.arange(wl.n) - 0.5 * (wl.n - 1)) ** 2
     rss = np.zeros(wl.d // 2)
     for qt, kt, dqt, dkt in extra:

@@ -101,3 +101,28 @@ def test_kernel_names():
     lib = rb.lib()
     names = {lib.rope_attn_kernel_name(i).decode() for i in range(12)}
     assert {"fwd_sm100", "bwd_dkdv_sm100", "bwd_dq_sm100", "dalpha_final"} <= names
+
+
+def test_fixed_bands_and_reserved_are_validated():
+    """fixed_bands must lie in 0..d/2 and reserved must be 0 (checked before any launch)."""
+    lib = rb.lib()
+    for fb, ok in ((0, True), (64, True), (65, False), (-1, False)):
+        p = rb.problem(1, 1, 256, 128, rb.RA_BF16, True, 1e4, fixed_bands=fb)
+        assert (rb.rope_attn_workspace_bytes(p) > 0) == ok, fb
+    p = rb.problem(1, 1, 256, 128, rb.RA_BF16, True, 1e4)
+    p.reserved = 1
+    assert lib.rope_attn_workspace_bytes(ctypes.byref(p)) == 0
+
+
+def test_alpha_adam_rejects_bad_arguments():
+    """Invalid optimiser arguments return RA_ERR_INVALID_ARG before any launch."""
+    lib = rb.lib()
+    buf = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    for kw in (dict(step=0), dict(beta1=1.0), dict(eps=0.0), dict(lr=float("nan"))):
+        args = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, clip_norm=1.0, step=1)
+        args.update(kw)
+        opt = rb.RaAdam(args["lr"], args["beta1"], args["beta2"], args["eps"], args["clip_norm"],
+                        args["step"])
+        assert lib.rope_attn_alpha_adam(ctypes.byref(opt), 64, buf, buf, buf, buf, None) == 1, kw
+    opt = rb.RaAdam(1e-3, 0.9, 0.999, 1e-8, 1.0, 1)
+    assert lib.rope_attn_alpha_adam(ctypes.byref(opt), 0, buf, buf, buf, buf, None) == 1

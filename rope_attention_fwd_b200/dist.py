@@ -3,9 +3,13 @@
 Every (batch, head) pair is independent except for dalpha: the LeRoPE log-frequencies
 are shared by all heads ("LeRoPE: learnable RoPE frequencies", Escolhas de Design
 Principais), so their gradient is the sum over every head of every rank.  Ranks run
-their own batches (weak scaling); after each backward the d/2 floats of dalpha are
-summed with one all-reduce (NCCL on GPUs, gloo in the CPU tests).
+disjoint (batch, head) units -- their own batches (weak scaling, what bench.py times) or
+contiguous shards of one batch's B*H units (`shard_bh`) -- and after each backward the
+d/2 floats of dalpha are combined by `allreduce_dalpha`: an all-gather of every rank's
+partial and a sum in rank order in fp64, so that every rank holds the same bits whatever
+the collective's internal reduction order (NCCL on GPUs, gloo in the CPU tests).
 """
+import torch
 import torch.distributed as dist
 
 RANK_SEED_STRIDE = 7919
@@ -16,8 +20,30 @@ def rank_seed(base_seed: int, rank: int) -> int:
     return base_seed + RANK_SEED_STRIDE * rank
 
 
+def shard_bh(B: int, H: int, world: int, rank: int):
+    """(start, count) of rank `rank`'s contiguous share of the B*H (batch, head) units,
+    balanced to within one unit.  Rows of a [B, H, n, d] tensor are contiguous per unit,
+    so a shard is the [1, count, n, d] problem starting at unit `start`."""
+    if not (0 <= rank < world):
+        raise ValueError(f"rank {rank} outside world of {world}")
+    units = B * H
+    base, extra = divmod(units, world)
+    start = rank * base + min(rank, extra)
+    return start, base + (1 if rank < extra else 0)
+
+
 def allreduce_dalpha(dalpha, group=None):
-    """In-place sum of every rank's dalpha (shape [d/2], fp32)."""
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(dalpha, op=dist.ReduceOp.SUM, group=group)
+    """dalpha <- the sum of every rank's dalpha (shape [d/2]), deterministic: all-gather,
+    then a fixed rank-order fp64 sum on every rank.  A no-op on one process."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return dalpha
+    world = dist.get_world_size(group)
+    if world == 1:
+        return dalpha
+    parts = [torch.empty_like(dalpha) for _ in range(world)]
+    dist.all_gather(parts, dalpha.contiguous(), group=group)
+    acc = torch.zeros(dalpha.shape, dtype=torch.float64, device=dalpha.device)
+    for p in parts:  # rank order
+        acc += p.to(torch.float64)
+    dalpha.copy_(acc.to(dalpha.dtype))
     return dalpha

@@ -1,6 +1,7 @@
-"""The multi-rank host path on CPU (gloo, world size 2): each rank draws its own batch,
-computes its dalpha (the float64 oracle stands in for the GPU kernels here), and the
-all-reduce must give the dalpha of the union of both ranks' heads."""
+"""The multi-rank host path on CPU (gloo): each rank draws its own batch, computes its
+dalpha (the float64 oracle stands in for the GPU kernels here), and the deterministic
+all-gather reduction must give the dalpha of the union of every rank's heads, bit for bit
+the rank-order sum, on every rank; the (batch, head) sharding covers every unit once."""
 import os
 import socket
 
@@ -10,7 +11,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from rope_attention_fwd_b200.configs import Workload
-from rope_attention_fwd_b200.dist import allreduce_dalpha, rank_seed
+from rope_attention_fwd_b200.dist import allreduce_dalpha, rank_seed, shard_bh
 from rope_attention_fwd_b200.inputs import make_inputs
 
 WL = Workload("dist 1x2x24x8", 1, 2, 24, 8, "f32", True, 100.0, "normal", alpha="normal",
@@ -58,3 +59,44 @@ def test_dalpha_allreduce_two_ranks():
 def test_single_process_is_a_noop():
     da = torch.arange(4, dtype=torch.float32)
     assert torch.equal(allreduce_dalpha(da.clone()), da)
+
+
+def _worker_f32(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(1000 + rank)
+        da = (torch.randn(64, generator=g) * 10 ** (rank % 3)).to(torch.float32)
+        out[("in", rank)] = da.numpy().copy()
+        allreduce_dalpha(da)
+        out[("out", rank)] = da.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dalpha_reduction_is_bitwise_rank_order_sum():
+    """Three ranks of fp32 partials of very different magnitudes: every rank ends with the
+    same bits, the float64 rank-order sum rounded once to fp32."""
+    world = 3
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker_f32, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    acc = np.zeros(64)
+    for r in range(world):
+        acc += res[("in", r)].astype(np.float64)
+    expect = acc.astype(np.float32)
+    for r in range(world):
+        assert np.array_equal(res[("out", r)], expect), r
+
+
+def test_shard_bh_covers_every_unit_once():
+    for B, H, world in ((2, 32, 8), (3, 5, 4), (1, 7, 8), (4, 16, 3)):
+        seen = []
+        counts = []
+        for r in range(world):
+            start, count = shard_bh(B, H, world, r)
+            seen.extend(range(start, start + count))
+            counts.append(count)
+        assert seen == list(range(B * H)), (B, H, world)
+        assert max(counts) - min(counts) <= 1

@@ -127,6 +127,27 @@ ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
                               void* dq, void* dk, void* dv, float* dalpha,
                               void* ws, size_t ws_bytes, void* stream);
 
+/* ---- the projections around the path (plain cuBLAS GEMMs) ---------------------
+ * "RoPE attention can be trained in almost-linear time" (Lemma 4.1) states the loss
+ * gradient with respect to the weights; these two calls carry the path's dQ, dK, dV back
+ * to the projection weights and the layer input.  Row-major layouts: x [B, n, d_model]
+ * (dtype of p); each W [d_model, H*d] (dtype of p) with head h in columns h*d..h*d+d-1;
+ * q, k, v, dq, dk, dv [B, H, n, d] (dtype of p); dW [d_model, H*d] fp32; dx [B, n, d_model]
+ * fp32.  fp32 accumulation (no TF32); fixed GEMM order (deterministic).  Pointers 16-byte
+ * aligned; d_model in 1..2^20.  Only p's B, H, n, d and dtype are used. */
+
+/* q[b,h] = x[b] W_Q[:, h], likewise k, v. */
+ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x,
+                             const void* wq, const void* wk, const void* wv,
+                             void* q, void* k, void* v, void* stream);
+
+/* dW_Q = sum_b x[b]^T dq[b] (dq[b] read as [n, H*d]), likewise dW_K, dW_V, and
+ * dx[b] = sum_h dq[b,h] W_Q[:,h]^T + dk[b,h] W_K[:,h]^T + dv[b,h] W_V[:,h]^T. */
+ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x,
+                             const void* wq, const void* wk, const void* wv,
+                             const void* dq, const void* dk, const void* dv,
+                             float* dwq, float* dwk, float* dwv, float* dx, void* stream);
+
 /* ---- the optimiser step for the learned frequencies ---------------------------
  * "LeRoPE" (Escolhas de Design Principais: Otimizacao) trains alpha without weight decay
  * and clips its gradient separately from the model's.  The page names neither the

@@ -322,3 +322,31 @@ def alpha_adam_step(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999, eps
     v_hat = m2 / (1.0 - beta2 ** step)
     alpha = np.asarray(alpha, dtype=np.float64) - lr * m_hat / (np.sqrt(v_hat) + eps)
     return alpha, m1, m2
+
+
+# --------------------------------------------------------------------------
+# the projections around the path (Lemma 4.1's gradient with respect to the weights)
+# --------------------------------------------------------------------------
+def proj_forward(x, wq, wk, wv, H):
+    """q, k, v [B, H, n, d] = x [B, n, d_model] W [d_model, H d] split into heads."""
+    B, n, _ = x.shape
+    d = wq.shape[1] // H
+    def split(y):
+        return y.reshape(B, n, H, d).transpose(0, 2, 1, 3)
+    x = np.asarray(x, dtype=np.float64)
+    return tuple(split(x @ np.asarray(w, dtype=np.float64)) for w in (wq, wk, wv))
+
+
+def proj_backward(x, wq, wk, wv, dq, dk, dv):
+    """dW = sum_b x_b^T dY_b with dY_b = dq[b] merged to [n, H d] (likewise dW_K, dW_V) and
+    dx = sum over q, k, v of dY W^T ("RoPE attention can be trained in almost-linear time",
+    Lemma 4.1: the gradient with respect to the weights; the chain rule through Y = X W)."""
+    x = np.asarray(x, dtype=np.float64)
+    B, n, dm = x.shape
+    out, dx = [], np.zeros((B, n, dm))
+    for w, g in ((wq, dq), (wk, dk), (wv, dv)):
+        g = np.asarray(g, dtype=np.float64)
+        gm = g.transpose(0, 2, 1, 3).reshape(B, n, -1)          # [B, n, H d]
+        out.append(np.einsum("bnm,bnc->mc", x, gm))
+        dx += gm @ np.asarray(w, dtype=np.float64).T
+    return out[0], out[1], out[2], dx

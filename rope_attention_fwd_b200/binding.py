@@ -62,6 +62,10 @@ def lib():
         L.rope_attn_alpha_adam.argtypes = [ctypes.POINTER(RaAdam), ctypes.c_int64, vp, vp, vp, vp,
                                            vp]
         L.rope_attn_alpha_adam.restype = ctypes.c_int
+        L.rope_attn_proj_fwd.argtypes = [P, ctypes.c_int64] + [vp] * 8
+        L.rope_attn_proj_fwd.restype = ctypes.c_int
+        L.rope_attn_proj_bwd.argtypes = [P, ctypes.c_int64] + [vp] * 12
+        L.rope_attn_proj_bwd.restype = ctypes.c_int
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -194,6 +198,34 @@ def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None
         ctypes.byref(prob), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha), _ptr(dq),
         _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(v.device)))
     return dq, dk, dv, dalpha
+
+
+def rope_attn_proj_fwd(x, wq, wk, wv, H, q=None, k=None, v=None):
+    """q, k, v [B, H, n, d] = x [B, n, d_model] @ W [d_model, H*d], head h in columns h*d.."""
+    B, n, dm = x.shape
+    d = wq.shape[1] // H
+    prob = problem(B, H, n, d, x.dtype, False, 1.0)
+    out = [torch.empty((B, H, n, d), dtype=x.dtype, device=x.device) if t is None else t
+           for t in (q, k, v)]
+    _check("rope_attn_proj_fwd", lib().rope_attn_proj_fwd(
+        ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), *[_ptr(t) for t in out],
+        _stream(x.device)))
+    return tuple(out)
+
+
+def rope_attn_proj_bwd(x, wq, wk, wv, dq, dk, dv):
+    """(dW_Q, dW_K, dW_V [d_model, H*d], dx [B, n, d_model]), all fp32, from the path's
+    dq, dk, dv [B, H, n, d]."""
+    B, H, n, d = dq.shape
+    dm = x.shape[2]
+    prob = problem(B, H, n, d, x.dtype, False, 1.0)
+    f32 = dict(dtype=torch.float32, device=x.device)
+    dws = [torch.empty((dm, H * d), **f32) for _ in range(3)]
+    dx = torch.empty((B, n, dm), **f32)
+    _check("rope_attn_proj_bwd", lib().rope_attn_proj_bwd(
+        ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk),
+        _ptr(dv), *[_ptr(t) for t in dws], _ptr(dx), _stream(x.device)))
+    return dws[0], dws[1], dws[2], dx
 
 
 def rope_attn_alpha_adam(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999, eps=1e-8,

@@ -407,3 +407,36 @@ def test_alpha_adam_closed_forms():
     _, m1, _ = ref.alpha_adam_step(np.zeros(M), g, np.zeros(M), np.zeros(M), 1, 0.01,
                                    clip_norm=1.0)
     np.testing.assert_allclose(m1, 0.1 * g / nrm, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- the projections (Lemma 4.1)
+def test_projection_gradients_match_autograd_of_the_layer():
+    """X -> (Q, K, V) = X W -> LeRoPE attention -> L, differentiated by autograd (the
+    complex-multiplication forward of I4b), against the oracle's chain: forward_backward on
+    the projected q, k, v, then proj_backward for dW_Q, dW_K, dW_V and dX."""
+    B, H, n, d, dm = 2, 2, 17, 8, 12
+    rng = np.random.default_rng(61)
+    x = rng.standard_normal((B, n, dm))
+    wq, wk, wv = (0.3 * rng.standard_normal((dm, H * d)) for _ in range(3))
+    e = rng.standard_normal((B, H, n, d))
+    alpha = 0.4 * rng.standard_normal(d // 2)
+    base = 200.0
+    q, k, v = ref.proj_forward(x, wq, wk, wv, H)
+    r = ref.forward_backward(q, k, v, e, alpha, base, True, block=8)
+    dwq, dwk, dwv, dx = ref.proj_backward(x, wq, wk, wv, r["dq"], r["dk"], r["dv"])
+    tx = torch.tensor(x, requires_grad=True)
+    tw = [torch.tensor(w, requires_grad=True) for w in (wq, wk, wv)]
+    m = torch.arange(d // 2, dtype=torch.float64)
+    th = torch.exp(torch.tensor(alpha)) * base ** (-2.0 * m / d)
+    pos = torch.arange(n, dtype=torch.float64)
+    def heads(y):
+        return y.reshape(B, n, H, d).transpose(1, 2)
+    tq, tk, tv = (heads(tx @ w) for w in tw)
+    qr, kr = _torch_rope_complex(tq, pos, th), _torch_rope_complex(tk, pos, th)
+    s = (qr @ kr.transpose(-1, -2) / math.sqrt(d)).masked_fill(
+        torch.triu(torch.ones(n, n, dtype=torch.bool), 1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ tv
+    (0.5 * ((o - torch.tensor(e)) ** 2).sum()).backward()
+    for g, want in zip(tw, (dwq, dwk, dwv)):
+        np.testing.assert_allclose(g.grad.numpy(), want, atol=1e-11)
+    np.testing.assert_allclose(tx.grad.numpy(), dx, atol=1e-11)

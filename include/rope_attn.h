@@ -141,12 +141,19 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
                              const void* wq, const void* wk, const void* wv,
                              void* q, void* k, void* v, void* stream);
 
+/* Bytes of caller workspace rope_attn_proj_bwd needs: one [B*n, H*d] copy of a gradient in
+ * the dtype (0 if *p is invalid). */
+size_t rope_attn_proj_workspace_bytes(const ra_problem* p);
+
 /* dW_Q = sum_b x[b]^T dq[b] (dq[b] read as [n, H*d]), likewise dW_K, dW_V, and
- * dx[b] = sum_h dq[b,h] W_Q[:,h]^T + dk[b,h] W_K[:,h]^T + dv[b,h] W_V[:,h]^T. */
+ * dx[b] = sum_h dq[b,h] W_Q[:,h]^T + dk[b,h] W_K[:,h]^T + dv[b,h] W_V[:,h]^T.  ws (16-byte
+ * aligned, ws_bytes >= rope_attn_proj_workspace_bytes) holds each gradient merged to
+ * [B*n, H*d] rows, so every product is one GEMM; RA_ERR_WORKSPACE if it is too small. */
 ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x,
                              const void* wq, const void* wk, const void* wv,
                              const void* dq, const void* dk, const void* dv,
-                             float* dwq, float* dwk, float* dwv, float* dx, void* stream);
+                             float* dwq, float* dwk, float* dwv, float* dx,
+                             void* ws, size_t ws_bytes, void* stream);
 
 /* ---- the optimiser step for the learned frequencies ---------------------------
  * "LeRoPE" (Escolhas de Design Principais: Otimizacao) trains alpha without weight decay

@@ -64,8 +64,10 @@ def lib():
         L.rope_attn_alpha_adam.restype = ctypes.c_int
         L.rope_attn_proj_fwd.argtypes = [P, ctypes.c_int64] + [vp] * 8
         L.rope_attn_proj_fwd.restype = ctypes.c_int
-        L.rope_attn_proj_bwd.argtypes = [P, ctypes.c_int64] + [vp] * 12
+        L.rope_attn_proj_bwd.argtypes = [P, ctypes.c_int64] + [vp] * 12 + [sz, vp]
         L.rope_attn_proj_bwd.restype = ctypes.c_int
+        L.rope_attn_proj_workspace_bytes.argtypes = [P]
+        L.rope_attn_proj_workspace_bytes.restype = sz
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -222,9 +224,11 @@ def rope_attn_proj_bwd(x, wq, wk, wv, dq, dk, dv):
     f32 = dict(dtype=torch.float32, device=x.device)
     dws = [torch.empty((dm, H * d), **f32) for _ in range(3)]
     dx = torch.empty((B, n, dm), **f32)
+    ws = torch.empty(int(lib().rope_attn_proj_workspace_bytes(ctypes.byref(prob))),
+                     dtype=torch.uint8, device=x.device)
     _check("rope_attn_proj_bwd", lib().rope_attn_proj_bwd(
         ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk),
-        _ptr(dv), *[_ptr(t) for t in dws], _ptr(dx), _stream(x.device)))
+        _ptr(dv), *[_ptr(t) for t in dws], _ptr(dx), _ptr(ws), ws.numel(), _stream(x.device)))
     return dws[0], dws[1], dws[2], dx
 
 

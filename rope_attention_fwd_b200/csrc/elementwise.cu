@@ -409,6 +409,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------- head merge
+// y[(b n + i) H d + h d + c] = g[((b H + h) n + i) d + c]: a [B, H, n, d] gradient as
+// [B n, H d] rows, 16-byte vectors (d * element size is a multiple of 16).
+__global__ void __launch_bounds__(256)
+    merge_heads_kernel(const uint4* __restrict__ g, uint4* __restrict__ y, long long rows_bhn,
+                       int H, int n, int vec_per_row) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows_bhn * vec_per_row) return;
+  const long long row = idx / vec_per_row;  // (b, h, i)
+  const int c = (int)(idx % vec_per_row);
+  const long long bh = row / n;
+  const int i = (int)(row % n);
+  const long long b = bh / H;
+  const int h = (int)(bh % H);
+  y[((b * n + i) * H + h) * vec_per_row + c] = g[idx];
+}
+
 // ================================================================ launchers
 cudaError_t launch_table(const ra_problem& p, const float* alpha, float2* table,
                          cudaStream_t s) {
@@ -507,6 +524,16 @@ cudaError_t launch_alpha_adam(float* alpha, const float* dalpha, float* m1, floa
                               float clip, float bc1, float bc2, cudaStream_t s) {
   alpha_adam_kernel<<<1, 256, 0, s>>>(alpha, dalpha, m1, m2, count, lr, b1, b2, eps, clip, bc1,
                                       bc2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_heads(const ra_problem& p, const void* g, void* y, cudaStream_t s) {
+  const int es = p.dtype == RA_BF16 ? 2 : 4;
+  const int vec = (int)(p.d * es / 16);
+  const long long rows = p.B * p.H * p.n;
+  const long long total = rows * vec;
+  merge_heads_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+      (const uint4*)g, (uint4*)y, rows, (int)p.H, (int)p.n, vec);
   return cudaGetLastError();
 }
 

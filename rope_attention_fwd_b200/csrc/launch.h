@@ -26,6 +26,8 @@ cudaError_t launch_delta(const ra_problem& p, const void* o, const void* dO, flo
 cudaError_t launch_alpha_adam(float* alpha, const float* dalpha, float* m1, float* m2,
                               long long count, float lr, float b1, float b2, float eps,
                               float clip, float bc1, float bc2, cudaStream_t s);
+// A [B, H, n, d] tensor as [B n, H d] rows (row (b, i) holds every head of position i).
+cudaError_t launch_merge_heads(const ra_problem& p, const void* g, void* y, cudaStream_t s);
 cudaError_t launch_dalpha_final(const ra_problem& p, const float* part, const float* alpha,
                                 float* dalpha, cudaStream_t s);
 

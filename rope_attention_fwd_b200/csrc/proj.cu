@@ -2,22 +2,26 @@
 //   forward:  Q = X W_Q, K = X W_K, V = X W_V, written in the [B, H, n, d] layout the
 //             attention kernels read;
 //   backward: the weight gradients dW_Q = sum_b X_b^T dQ_b (likewise dW_K, dW_V) and the
-//             input gradient dX_b = sum_h dQ_bh W_Q,h^T + dK_bh W_K,h^T + dV_bh W_V,h^T
+//             input gradient dX_b = sum_h dQ_bh W_Q,h^T + dK_bh W_K,h^T + dV_bh W_V,h^T;
+//             each gradient is first merged to [B n, H d] rows (one copy kernel into the
+//             caller's workspace), so that dW = X^T Y and dX += Y W^T are one GEMM each
 // ("RoPE attention can be trained in almost-linear time", Lemma 4.1: the loss gradient with
 // respect to the weights, reached from the gradient of the attention inputs through X).
 //
 // Layouts (row-major): X [B, n, d_model]; W [d_model, H d] with head h in columns
 // h d .. h d + d - 1; Q, K, V, dQ, dK, dV [B, H, n, d]; dW [d_model, H d] fp32;
 // dX [B, n, d_model] fp32.  cuBLAS is column-major, so each row-major matrix is used as
-// its transpose: Q_bh^T = W_h^T X_b^T, dW_h^T = sum_b dQ_bh^T X_b, dX_b^T = sum_h W_h dQ_bh^T.
-// Accumulation is fp32 (CUBLAS_COMPUTE_32F, no TF32); the sums over batches and heads are
-// successive GEMMs with beta = 1 in a fixed order, so the results are deterministic.
+// its transpose: Q_bh^T = W_h^T X_b^T, dW^T = Y^T X, dX^T = sum over Q, K, V of W Y^T.
+// Accumulation is fp32 (CUBLAS_COMPUTE_32F, no TF32); the sums over batches (forward) and
+// over Q, K, V (dX) are successive GEMMs with beta = 1 in a fixed order, and cuBLAS without
+// atomics is bitwise reproducible, so the results are deterministic.
 #include <cublas_v2.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 #include <unordered_map>
 
+#include "launch.h"
 #include "rope_attn.h"
 
 namespace {
@@ -91,55 +95,47 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
   return RA_OK;
 }
 
+size_t rope_attn_proj_workspace_bytes(const ra_problem* p) {
+  if (check(p, 1) != RA_OK) return 0;
+  return (size_t)(p->B * p->n * p->H * p->d) * elem(p);
+}
+
 ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x, const void* wq,
                              const void* wk, const void* wv, const void* dq, const void* dk,
                              const void* dv, float* dwq, float* dwk, float* dwv, float* dx,
-                             void* stream) {
+                             void* ws, size_t ws_bytes, void* stream) {
   ra_status st = check(p, d_model);
   if (st != RA_OK) return st;
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wk) || !aligned16(wv) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(dwq) || !aligned16(dwk) ||
       !aligned16(dwv) || !aligned16(dx))
     return RA_ERR_INVALID_ARG;
+  if (!aligned16(ws) || ws_bytes < rope_attn_proj_workspace_bytes(p)) return RA_ERR_WORKSPACE;
+  // the head merge moves 16-byte vectors: a d-row must be a whole number of them
+  if (p->B * p->n > (int64_t(1) << 31) - 1 || ((size_t)p->d * elem(p)) % 16 != 0)
+    return RA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cublasHandle_t h = cublas_for_current_device();
-  if (!h || cublasSetStream(h, static_cast<cudaStream_t>(stream)) != CUBLAS_STATUS_SUCCESS)
-    return RA_ERR_CUDA;
-  const int n = (int)p->n, d = (int)p->d, H = (int)p->H, dm = (int)d_model;
+  if (!h || cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return RA_ERR_CUDA;
+  const int rows = (int)(p->B * p->n), hd = (int)(p->H * p->d), dm = (int)d_model;
   const cudaDataType_t t = in_type(p);
-  const size_t es = elem(p);
   const float one = 1.f, zero = 0.f;
   const void* W[3] = {wq, wk, wv};
   const void* G[3] = {dq, dk, dv};
   float* DW[3] = {dwq, dwk, dwv};
   for (int which = 0; which < 3; ++which) {
-    // dW_h^T (d x d_model) = sum_b dQ_bh^T (d x n) X_b (n x d_model), every head at once
-    for (int64_t b = 0; b < p->B; ++b) {
-      const char* xb = static_cast<const char*>(x) + (size_t)b * n * dm * es;
-      const char* gb = static_cast<const char*>(G[which]) + (size_t)b * H * n * d * es;
-      if (cublasGemmStridedBatchedEx(h, CUBLAS_OP_N, CUBLAS_OP_T, d, dm, n, &one, gb, t, d,
-                                     (long long)n * d, xb, t, dm, 0LL, b == 0 ? &zero : &one,
-                                     DW[which], CUDA_R_32F, H * d, (long long)d, H,
-                                     CUBLAS_COMPUTE_32F,
-                                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-        return RA_ERR_CUDA;
-    }
-  }
-  // dX_b^T (d_model x n) = sum over Q, K, V and heads h of W_h (d_model x d) dQ_bh^T (d x n)
-  for (int64_t b = 0; b < p->B; ++b) {
-    float* xb = dx + (size_t)b * n * dm;
-    bool first = true;
-    for (int which = 0; which < 3; ++which) {
-      for (int hh = 0; hh < H; ++hh) {
-        const char* wh = static_cast<const char*>(W[which]) + (size_t)hh * d * es;
-        const char* gbh =
-            static_cast<const char*>(G[which]) + ((size_t)b * H + hh) * (size_t)n * d * es;
-        if (cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, dm, n, d, &one, wh, t, H * d, gbh, t, d,
-                         first ? &zero : &one, xb, CUDA_R_32F, dm, CUBLAS_COMPUTE_32F,
-                         CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
-          return RA_ERR_CUDA;
-        first = false;
-      }
-    }
+    // Y = the gradient merged to [B n, H d] rows (row (b, i) holds every head of position i)
+    if (ra::launch_merge_heads(*p, G[which], ws, s) != cudaSuccess) return RA_ERR_CUDA;
+    // dW^T (H d x d_model) = Y^T X: one GEMM over all B n rows
+    if (cublasGemmEx(h, CUBLAS_OP_N, CUBLAS_OP_T, hd, dm, rows, &one, ws, t, hd, x, t, dm, &zero,
+                     DW[which], CUDA_R_32F, hd, CUBLAS_COMPUTE_32F,
+                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+      return RA_ERR_CUDA;
+    // dX^T (d_model x B n) (+)= W Y^T
+    if (cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, dm, rows, hd, &one, W[which], t, hd, ws, t, hd,
+                     which == 0 ? &zero : &one, dx, CUDA_R_32F, dm, CUBLAS_COMPUTE_32F,
+                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+      return RA_ERR_CUDA;
   }
   return RA_OK;
 }

@@ -265,24 +265,20 @@ def forward_backward(q, k, v, e, alpha, base, causal, **kw):
 # --------------------------------------------------------------------------
 # second formula for dalpha: derivative of the DTFT surrogate
 # --------------------------------------------------------------------------
-def dalpha_offset_dtft(q, k, v, do, alpha, base, causal, pairing="interleaved"):
-    """dalpha via the offset-aggregated gradient signal ("LeRoPE", Analise Teorica).
-
-    Band m of a row is read as the complex number z = x0 + i x1, so that a
-    rotation by psi is multiplication by exp(i psi) and the band's share of the
-    score is S_ij^(m) = Re(exp(i (i-j) theta_hat_m) z_q,i conj(z_k,j)) / sqrt(d),
-    built from the UNROTATED q, k.  With g_m(D) = sum_{i-j=D} dS_ij z_q,i
-    conj(z_k,j) / sqrt(d) (the gradient signal aggregated by offset D), the
-    surrogate P_m(theta) = Re sum_D g_m(D) exp(i D theta) is the real part of
-    the DTFT of g_m, and dL/dtheta_hat_m = P_m'(theta_hat_m); dalpha_m =
-    theta_hat_m dL/dtheta_hat_m.  Small n only (builds n x n matrices).
-    """
+def offset_signal(q, k, v, do, alpha, base, causal, pairing="interleaved", fixed_bands=0):
+    """The offset-aggregated gradient signal ("LeRoPE", Analise Teorica), summed over every
+    batch and head: g[m, D + n - 1] = sum_{i - j = D} dS_ij z_q,i conj(z_k,j) / sqrt(d) for
+    offsets D = -(n-1)..n-1, with band m of a row read as z = x0 + i x1 of the UNROTATED
+    q, k (a rotation by psi is multiplication by exp(i psi)).  Then the band's share of the
+    scores is S_ij^(m) = Re(exp(i (i-j) theta_hat_m) z_q,i conj(z_k,j)) / sqrt(d), and
+    P_m(theta) = Re sum_D g_m(D) exp(i D theta), the real part of the DTFT of g_m, is the
+    surrogate whose derivative at theta_hat_m is dL/dtheta_hat_m.  Small n only (n x n)."""
     B, H, n, d = q.shape
-    _, th = frequencies(d, base, alpha)
+    _, th = frequencies(d, base, alpha, fixed_bands)
     phi = angles(n, th)
     i0, i1 = band_index(d, pairing)
     D = np.arange(n)[:, None] - np.arange(n)[None, :]
-    out = np.zeros(d // 2)
+    g = np.zeros((d // 2, 2 * n - 1), dtype=complex)
     for b in range(B):
         for h in range(H):
             qt = rotate(q[b, h], phi, pairing)
@@ -292,12 +288,26 @@ def dalpha_offset_dtft(q, k, v, do, alpha, base, causal, pairing="interleaved"):
             zk = k[b, h][:, i0] + 1j * k[b, h][:, i1]
             for m in range(d // 2):
                 w = ds * np.outer(zq[:, m], np.conj(zk[:, m])) / np.sqrt(d)
-                g = np.zeros(2 * n - 1, dtype=complex)       # offsets -(n-1)..n-1
-                np.add.at(g, (D + n - 1).ravel(), w.ravel())
-                offs = np.arange(-(n - 1), n)
-                dP = np.real(np.sum(1j * offs * g * np.exp(1j * offs * th[m])))
-                out[m] += th[m] * dP
-    return out
+                np.add.at(g[m], (D + n - 1).ravel(), w.ravel())
+    return g
+
+
+def dtft_derivative(g, theta):
+    """P_m'(theta_m) = d/dtheta Re sum_D g_m(D) exp(i D theta) at theta = theta_m, for the
+    signal g [M, 2n - 1] of offsets D = -(n-1)..n-1."""
+    n = (g.shape[1] + 1) // 2
+    offs = np.arange(-(n - 1), n)
+    ph = np.exp(1j * np.outer(np.asarray(theta, dtype=np.float64), offs))
+    return np.real(np.sum(1j * offs[None, :] * g * ph, axis=1))
+
+
+def dalpha_offset_dtft(q, k, v, do, alpha, base, causal, pairing="interleaved", fixed_bands=0):
+    """dalpha via the offset-aggregated gradient signal ("LeRoPE", Analise Teorica):
+    dalpha_m = theta_hat_m P_m'(theta_hat_m) with g_m from :func:`offset_signal`."""
+    d = q.shape[3]
+    _, th = frequencies(d, base, alpha, fixed_bands)
+    g = offset_signal(q, k, v, do, alpha, base, causal, pairing, fixed_bands)
+    return th * dtft_derivative(g, th)
 
 
 # --------------------------------------------------------------------------

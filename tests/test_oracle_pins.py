@@ -440,3 +440,28 @@ def test_projection_gradients_match_autograd_of_the_layer():
     for g, want in zip(tw, (dwq, dwk, dwv)):
         np.testing.assert_allclose(g.grad.numpy(), want, atol=1e-11)
     np.testing.assert_allclose(tx.grad.numpy(), dx, atol=1e-11)
+
+
+# ---------------------------------------------------------------- the spectrum of the gradient signal
+@pytest.mark.parametrize("causal", [False, True])
+def test_offset_signal_surrogate_equals_score_inner_product(causal):
+    """sum over bands of P_m(theta_hat_m) = sum_ij dS_ij S_ij: the surrogate evaluated at the
+    model's own frequencies gives back each band's share of the scores (S from the rotated
+    vectors, dS from the backward's matrices, per head)."""
+    B, H, n, d = 1, 2, 14, 8
+    q, k, v, e, alpha, base = rand_problem(67, B, H, n, d, alpha_scale=0.5, base=50.0)
+    r = ref.forward_backward(q, k, v, e, alpha, base, causal)
+    g = ref.offset_signal(q, k, v, r["do"], alpha, base, causal)
+    _, th = ref.frequencies(d, base, alpha)
+    offs = np.arange(-(n - 1), n)
+    surrogate = np.sum(np.real(g * np.exp(1j * np.outer(th, offs))))
+    phi = ref.angles(n, th)
+    want = 0.0
+    for h in range(H):
+        qt, kt = ref.rotate(q[0, h], phi), ref.rotate(k[0, h], phi)
+        _, ds = ref.head_matrices(qt, kt, v[0, h], r["do"][0, h], causal)
+        s = qt @ kt.T / np.sqrt(d)
+        want += np.sum(np.where(np.isfinite(ds), ds, 0.0) * s)
+    np.testing.assert_allclose(surrogate, want, rtol=1e-11, atol=1e-12)
+    if causal:
+        assert np.all(g[:, : n - 1] == 0)   # no key after its query: no negative offset

@@ -155,6 +155,22 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
                              float* dwq, float* dwk, float* dwv, float* dx,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* ---- the frequency-spectrum diagnostic ----------------------------------------
+ * "LeRoPE" (Analise Teorica): the offset-aggregated gradient signal
+ *   g_m(D) = sum_{b,h} sum_{i-j=D} dS_ij z_q,i conj(z_k,j) / sqrt(d),  D = -(n-1)..n-1,
+ * with band m of a row read as z = x_2m + i x_2m+1 of the unrotated q, k, and the frequency
+ * gradient from the derivative of its DTFT surrogate P_m(theta) = Re sum_D g_m(D) e^{iD theta}:
+ * dalpha_m = theta_hat_m P_m'(theta_hat_m) (the backward's dalpha by a second route).
+ * Inputs as for rope_attn_bwd (o, lse from the forward, dO the upstream gradient).
+ * Outputs: g [d/2][2n-1][2] fp32 (re, im; offset D at index D + n - 1; causal: D < 0 is 0)
+ * and dalpha [d/2] fp32.  A diagnostic: one (batch, head) at a time with n x n fp32 scratch
+ * (workspace from rope_attn_spectrum_workspace_bytes; n <= 32768); deterministic. */
+size_t rope_attn_spectrum_workspace_bytes(const ra_problem* p);
+ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse, const void* dO,
+                             const float* alpha, float* g, float* dalpha,
+                             void* ws, size_t ws_bytes, void* stream);
+
 /* ---- the optimiser step for the learned frequencies ---------------------------
  * "LeRoPE" (Escolhas de Design Principais: Otimizacao) trains alpha without weight decay
  * and clips its gradient separately from the model's.  The page names neither the

@@ -68,6 +68,10 @@ def lib():
         L.rope_attn_proj_bwd.restype = ctypes.c_int
         L.rope_attn_proj_workspace_bytes.argtypes = [P]
         L.rope_attn_proj_workspace_bytes.restype = sz
+        L.rope_attn_spectrum_workspace_bytes.argtypes = [P]
+        L.rope_attn_spectrum_workspace_bytes.restype = sz
+        L.rope_attn_spectrum.argtypes = [P] + [vp] * 10 + [sz, vp]
+        L.rope_attn_spectrum.restype = ctypes.c_int
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
@@ -230,6 +234,21 @@ def rope_attn_proj_bwd(x, wq, wk, wv, dq, dk, dv):
         ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk),
         _ptr(dv), *[_ptr(t) for t in dws], _ptr(dx), _ptr(ws), ws.numel(), _stream(x.device)))
     return dws[0], dws[1], dws[2], dx
+
+
+def rope_attn_spectrum(q, k, v, o, lse, dO, alpha, base, causal, fixed_bands=0):
+    """(g [d/2, 2n-1] complex64, dalpha [d/2] fp32): the offset-aggregated gradient signal of
+    every band and the frequency gradient from its DTFT surrogate (see include/rope_attn.h)."""
+    prob = _problem_of(q, causal, base, fixed_bands)
+    B, H, n, d = q.shape
+    ws = torch.empty(int(lib().rope_attn_spectrum_workspace_bytes(ctypes.byref(prob))),
+                     dtype=torch.uint8, device=q.device)
+    g = torch.empty((d // 2, 2 * n - 1, 2), dtype=torch.float32, device=q.device)
+    dalpha = torch.empty(d // 2, dtype=torch.float32, device=q.device)
+    _check("rope_attn_spectrum", lib().rope_attn_spectrum(
+        ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha),
+        _ptr(g), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(q.device)))
+    return torch.view_as_complex(g), dalpha
 
 
 def rope_attn_alpha_adam(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999, eps=1e-8,

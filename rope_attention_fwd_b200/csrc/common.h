@@ -72,4 +72,13 @@ inline WsLayout ws_layout(const ra_problem& p) {
   return w;
 }
 
+#ifdef __CUDACC__
+// theta_hat_m, or 0 for the fixed (unrotated) bands m >= mrot.
+__device__ __forceinline__ double theta_hat(const float* alpha, int m, int d, double base,
+                                            int mrot) {
+  if (m >= mrot) return 0.0;
+  return exp((double)alpha[m]) * pow(base, -2.0 * (double)m / (double)d);
+}
+#endif
+
 }  // namespace ra

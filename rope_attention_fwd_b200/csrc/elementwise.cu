@@ -39,12 +39,6 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// theta_hat_m, or 0 for the fixed (unrotated) bands m >= mrot.
-__device__ __forceinline__ double theta_hat(const float* alpha, int m, int d, double base,
-                                            int mrot) {
-  if (m >= mrot) return 0.0;
-  return exp((double)alpha[m]) * pow(base, -2.0 * (double)m / (double)d);
-}
 
 // ---------------------------------------------------------------- table
 __global__ void rope_table_kernel(const float* __restrict__ alpha, float2* __restrict__ table,

@@ -21,15 +21,18 @@
 #include <mutex>
 #include <unordered_map>
 
+#include "blas.h"
 #include "launch.h"
 #include "rope_attn.h"
 
-namespace {
+namespace ra {
 
+namespace {
 std::mutex g_cublas_mu;
 std::unordered_map<int, cublasHandle_t> g_cublas;  // one handle per device
+}  // namespace
 
-cublasHandle_t cublas_for_current_device() {
+cublasHandle_t cublas_handle() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
   std::lock_guard<std::mutex> g(g_cublas_mu);
@@ -40,6 +43,10 @@ cublasHandle_t cublas_for_current_device() {
   g_cublas[dev] = h;
   return h;
 }
+
+}  // namespace ra
+
+namespace {
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) % 16) == 0; }
 
@@ -71,7 +78,7 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
   if (!aligned16(x) || !aligned16(wq) || !aligned16(wk) || !aligned16(wv) || !aligned16(q) ||
       !aligned16(k) || !aligned16(v))
     return RA_ERR_INVALID_ARG;
-  cublasHandle_t h = cublas_for_current_device();
+  cublasHandle_t h = ra::cublas_handle();
   if (!h || cublasSetStream(h, static_cast<cudaStream_t>(stream)) != CUBLAS_STATUS_SUCCESS)
     return RA_ERR_CUDA;
   const int n = (int)p->n, d = (int)p->d, H = (int)p->H, dm = (int)d_model;
@@ -115,7 +122,7 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
   if (p->B * p->n > (int64_t(1) << 31) - 1 || ((size_t)p->d * elem(p)) % 16 != 0)
     return RA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cublasHandle_t h = cublas_for_current_device();
+  cublasHandle_t h = ra::cublas_handle();
   if (!h || cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return RA_ERR_CUDA;
   const int rows = (int)(p->B * p->n), hd = (int)(p->H * p->d), dm = (int)d_model;
   const cudaDataType_t t = in_type(p);

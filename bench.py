@@ -343,7 +343,8 @@ def phase_tflops(kernels, share, flops, steps):
 
 
 def traffic_for(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's source (the
+    whole file, or the span of it the record names) is the one the counters were taken on."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -355,7 +356,17 @@ def traffic_for(kernel):
     src = os.path.join(ROOT, "rope_attention_fwd_b200", "csrc", rec["source"])
     if not os.path.exists(src):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    text = open(src, encoding="utf-8").read()
+    # a record may cover only the kernel's own part of a file that holds several kernels
+    if "span_start" in rec:
+        if rec["span_start"] not in text:
+            return None
+        text = text[text.index(rec["span_start"]):]
+    if "span_end" in rec:
+        if rec["span_end"] not in text:
+            return None
+        text = text[:text.index(rec["span_end"])]
+    sha = hashlib.sha256(text.encode("utf-8")).hexdigest()
     return rec["bytes_per_launch"] if sha == rec["source_sha256"] else None
 
 

@@ -814,18 +814,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t dw[16];
 #pragma unroll
         for (int c2 = 0; c2 < 16; ++c2) {
-          float dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = 2 * c2 + e;  // column within this half
-            float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - lse2, 32 * h + c);
-            if (need_mask) {
-              const int key = key0 + 32 * h + c;
-              if (key >= n || (causal && key > row)) p = 0.f;
-            }
-            dsv[e] = p * fmaf(__uint_as_float(dr[c]), dss, -dlt_s);
+          // columns c, c + 1 as one packed pair (f32x2: half the FMA-pipe issue slots)
+          const int c = 2 * c2;
+          const float2 x2 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                  make_float2(scale_log2, scale_log2), make_float2(-lse2, -lse2));
+          float2 p2 = make_float2(exp2_col(x2.x, 32 * h + c), exp2_col(x2.y, 32 * h + c + 1));
+          if (need_mask) {
+            const int key = key0 + 32 * h + c;
+            if (key >= n || (causal && key > row)) p2.x = 0.f;
+            if (key + 1 >= n || (causal && key + 1 > row)) p2.y = 0.f;
           }
-          dw[c2] = pack_f16x2_sat(dsv[0], dsv[1]);
+          const float2 ds2 =
+              fmul2(p2, ffma2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                              make_float2(dss, dss), make_float2(-dlt_s, -dlt_s)));
+          dw[c2] = pack_f16x2_sat(ds2.x, ds2.y);
         }
         tmem_st16(s_base + packed_col(32 * h), dw);
       }

@@ -1,7 +1,7 @@
-// fastmath.cuh -- pipe-balancing replacements for two XU-pipe operations in the
-// softmax loops.  On sm_100 the XU pipe executes both MUFU.EX2 and the f32->bf16x2
-// packing conversion, and in the attention kernels it is the first pipe to saturate
-// while the FMA and integer pipes sit mostly idle.
+// fastmath.cuh -- pipe-balancing replacements for XU-pipe operations in the softmax
+// loops, and packed fp32-pair arithmetic.  On sm_100 the XU pipe executes both MUFU.EX2
+// and the f32->bf16x2 packing conversion, and in the attention kernels it is the first
+// pipe to saturate while the FMA and integer pipes sit mostly idle.
 //
 //  * pack_bf16x2_alu: two fp32 -> two bf16 in one 32-bit word on the integer pipe.
 //    Adding 0x8000 to the bit pattern and keeping the high half rounds the magnitude
@@ -38,6 +38,26 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
   // bits(t) << 23 == rint(x) << 23 (mod 2^32): the magic constant's bits shift out.
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Packed fp32 pairs: sm_100's f32x2 FMA-pipe instructions do two lanes' worth of fp32
+// arithmetic in one issue slot, each lane rounded exactly as the scalar instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 a, b, c, d; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5}; mov.b64 c, {%6, %7};"
+      " fma.rn.f32x2 d, a, b, c; mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 a, b, d; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5};"
+      " mul.rn.f32x2 d, a, b; mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 }  // namespace ra

@@ -299,28 +299,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool need_mask = (key0 + C::BN > n) || (causal && j == qt);
       const int nvalid =
           need_mask ? max(0, min(C::BN, (causal ? min(n, row + 1) : n) - key0)) : C::BN;
-      // pass 1: the row max of the raw scores (masked entries excluded)
+      // the whole row of S in registers (one TMEM read; S_x is free again once P_x is
+      // written over it)
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_base + 32 * c, sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld(sr[c]);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= nvalid) sr[c][i] = __float_as_uint(-CUDART_INF_F);
+      }
+      // the row max of the raw scores (masked entries are -inf)
       float mp[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mp[a] = -CUDART_INF_F;
+      for (int a = 0; a < 8; ++a) mp[a] = __uint_as_float(sr[0][a]);
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(s_base + 64 * c2, r0);
-        tmem_ld32(s_base + 64 * c2 + 32, r1);
-        tmem_wait_ld(r0);
-        tmem_wait_ld(r1);
-        if (need_mask) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (64 * c2 + i >= nvalid) r0[i] = __float_as_uint(-CUDART_INF_F);
-            if (64 * c2 + 32 + i >= nvalid) r1[i] = __float_as_uint(-CUDART_INF_F);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          mp[i & 7] = fmaxf(mp[i & 7], fmaxf(__uint_as_float(r0[i]), __uint_as_float(r1[i])));
-      }
+      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
       const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * scale_log2;
       // lazy rescale: move the reference max only when some row of the warp needs it
@@ -333,19 +331,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_new;
       }
       const float m_use = m == -CUDART_INF_F ? 0.f : m;
-      // pass 2: P = 2^(s scale - m) chunk by chunk, summed and written as bf16 over S.
-      // Chunk c (columns 32c..32c+31) lands in columns 16c..16c+15, inside chunks this
-      // thread has already read.
+      // P = 2^(s scale - m), summed and written as bf16 over S: chunk c (columns
+      // 32c..32c+31) lands in columns 16c..16c+15 (masked entries give 2^-inf = 0)
       float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_base + 32 * c, r);
-        tmem_wait_ld(r);
         float pv[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          pv[i] = exp2_col(fmaf(__uint_as_float(r[i]), scale_log2, -m_use), 32 * c + i);
+          pv[i] = exp2_col(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_use), 32 * c + i);
         if (need_mask) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)

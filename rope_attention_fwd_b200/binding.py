@@ -119,6 +119,14 @@ def rope_attn_workspace_bytes(prob):
     return int(lib().rope_attn_workspace_bytes(ctypes.byref(prob)))
 
 
+def rope_attn_proj_workspace_bytes(prob):
+    return int(lib().rope_attn_proj_workspace_bytes(ctypes.byref(prob)))
+
+
+def rope_attn_spectrum_workspace_bytes(prob):
+    return int(lib().rope_attn_spectrum_workspace_bytes(ctypes.byref(prob)))
+
+
 def workspace(prob, device):
     """A fresh device workspace for `prob` (uint8 tensor)."""
     nbytes = rope_attn_workspace_bytes(prob)

@@ -126,3 +126,48 @@ def test_alpha_adam_rejects_bad_arguments():
         assert lib.rope_attn_alpha_adam(ctypes.byref(opt), 64, buf, buf, buf, buf, None) == 1, kw
     opt = rb.RaAdam(1e-3, 0.9, 0.999, 1e-8, 1.0, 1)
     assert lib.rope_attn_alpha_adam(ctypes.byref(opt), 0, buf, buf, buf, buf, None) == 1
+
+
+def test_projection_validation_before_any_call():
+    """The projection entry points reject bad sizes, pointers and workspaces before they
+    reach cuBLAS or launch anything."""
+    lib = rb.lib()
+    fake = ctypes.c_void_p(4096)
+    p = rb.problem(2, 4, 64, 64, rb.RA_BF16, True, 1e4)
+    need = rb.rope_attn_proj_workspace_bytes(p)
+    assert need == 2 * 64 * 4 * 64 * 2
+    # d_model out of range, a null or misaligned operand
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 0, *[fake] * 7, None) == 1
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, None, *[fake] * 6, None) == 1
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, ctypes.c_void_p(4096 + 8), *[fake] * 6,
+                                  None) == 1
+    # backward: workspace too small or misaligned, then a head row that is not whole
+    # 16-byte vectors (d = 2 in fp32) is unsupported
+    assert lib.rope_attn_proj_bwd(ctypes.byref(p), 256, *[fake] * 11, fake, need - 1, None) == 3
+    assert lib.rope_attn_proj_bwd(ctypes.byref(p), 256, *[fake] * 11,
+                                  ctypes.c_void_p(4096 + 8), need, None) == 3
+    p2 = rb.problem(1, 1, 8, 2, rb.RA_F32, False, 1e4)
+    need2 = rb.rope_attn_proj_workspace_bytes(p2)
+    assert lib.rope_attn_proj_bwd(ctypes.byref(p2), 16, *[fake] * 11, fake, need2, None) == 2
+
+
+def test_spectrum_validation_before_any_call():
+    """The spectrum diagnostic sizes its O(n^2) scratch, caps n and rejects bad pointers and
+    workspaces before any launch."""
+    lib = rb.lib()
+    fake = ctypes.c_void_p(4096)
+    p = rb.problem(1, 2, 96, 64, rb.RA_BF16, True, 1e4)
+    need = rb.rope_attn_spectrum_workspace_bytes(p)
+    assert need >= 2 * 96 * 96 * 4 + 32 * (2 * 96 - 1) * 16
+    too_long = rb.problem(1, 1, 32769, 64, rb.RA_BF16, True, 1e4)
+    assert rb.rope_attn_spectrum_workspace_bytes(too_long) == 0
+    assert rb.rope_attn_spectrum_workspace_bytes(rb.problem(1, 1, 32768, 64, rb.RA_BF16,
+                                                            True, 1e4)) > 0
+    # q, k, v, o, lse, dO, alpha, g, dalpha, then the workspace
+    assert lib.rope_attn_spectrum(ctypes.byref(too_long), *[fake] * 9, fake, 1 << 40,
+                                  None) == 1
+    assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 7, None, fake, fake, need,
+                                  None) == 1
+    assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, fake, need - 1, None) == 3
+    assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, ctypes.c_void_p(4096 + 16),
+                                  need, None) == 3

@@ -171,3 +171,23 @@ def test_spectrum_validation_before_any_call():
     assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, fake, need - 1, None) == 3
     assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, ctypes.c_void_p(4096 + 16),
                                   need, None) == 3
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/rope_attn.h compiles as strict C99 in a C client that links the library and
+    drives its host-side checks (no GPU call)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(rb.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    src = os.path.join(ROOT, "tests", "c_abi", "abi_check.c")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), src, "-L", libdir, "-lrope_attn",
+                        f"-Wl,-rpath,{libdir}", "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "c abi ok" in r.stdout

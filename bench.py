@@ -343,8 +343,9 @@ def phase_tflops(kernels, share, flops, steps):
 
 
 def traffic_for(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's source (the
-    whole file, or the span of it the record names) is the one the counters were taken on."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's code (the whole
+    file, or the span of it the record names; comments aside) is the one the counters were
+    taken on."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
@@ -366,8 +367,15 @@ def traffic_for(kernel):
         if rec["span_end"] not in text:
             return None
         text = text[:text.index(rec["span_end"])]
-    sha = hashlib.sha256(text.encode("utf-8")).hexdigest()
+    sha = hashlib.sha256(code_only(text).encode("utf-8")).hexdigest()
     return rec["bytes_per_launch"] if sha == rec["source_sha256"] else None
+
+
+def code_only(text):
+    """The source without // comments and blank lines: what the counters depend on."""
+    import re
+    lines = (re.sub(r"//.*$", "", line).rstrip() for line in text.split("\n"))
+    return "\n".join(line for line in lines if line)
 
 
 def main():

@@ -30,11 +30,11 @@
 // Two kernels, no atomics (deterministic):
 //   dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
 //         time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
-//         (M = 128 keys, N = 64 queries), the softmax warps form P^T and dS^T in bf16,
+//         (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T (fp16),
 //         then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
 //         accumulated in TMEM for the whole pass.
 //   dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
-//         dP = dO V_j^T (double-buffered in TMEM), dS in bf16, dQ~ += dS K~_j.
+//         dP = dO V_j^T (double-buffered in TMEM), dS in fp16, dQ~ += dS K~_j.
 // Warp roles: two softmax warpgroups (warps 0-7) each own every row (TMEM lane) and half
 // of the 64 streamed columns; warp 8 issues TMA copies; warp 9 allocates TMEM and issues
 // tcgen05.mma.  Every wait is bounded.

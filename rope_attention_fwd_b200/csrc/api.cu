@@ -106,6 +106,12 @@ int starve_block() {
   return s ? std::atoi(s) : -1;
 }
 
+// RA_FWD_SPLIT_S=1 selects the split-half forward (fwd_split_sm100.cu), read per call.
+bool fwd_split_s() {
+  const char* s = std::getenv("RA_FWD_SPLIT_S");
+  return s && std::atoi(s) == 1;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -203,7 +209,9 @@ ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const
       !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128, true) || !make_map(&maps.v, v, *p, 128))
     return RA_ERR_CUDA;
   DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), starve_block()};
-  RA_LAUNCH(K_FWD_SM100, s, launch_fwd_sm100(*p, maps, o, lse, ctl, s));
+  RA_LAUNCH(K_FWD_SM100, s,
+            fwd_split_s() ? launch_fwd_split_sm100(*p, maps, o, lse, ctl, s)
+                          : launch_fwd_sm100(*p, maps, o, lse, ctl, s));
   return RA_OK;
 }
 

@@ -1,0 +1,432 @@
+// fwd_split_sm100.cu -- the forward of fwd_sm100.cu with every 128-key S tile split into
+// two 64-column halves that move through the pipeline on barriers of their own.
+//
+// Same computation, CTA layout, TMA ring and TMEM budget as fwd_sm100.cu ("RoPE attention
+// can be trained in almost-linear time", Metodologia 1: the normalised softmax of the RoPE
+// scores, O and lse; "LeRoPE: learnable RoPE frequencies", Mecanismo Central: the rotated
+// Q~, K~).  What changes is the unit of the S -> P -> P V hand-off.
+//
+// In fwd_sm100.cu, S_x(j+1) overwrites P_x(j) in TMEM, so a query tile's loop is its
+// softmax followed by its own P V and S MMAs: the softmax warps wait for the tensor core
+// once per key tile.  Here half h of tile x (TMEM columns 128x + 64h .. +63, P_x,h written
+// as bf16 pairs over its first 32 columns) has its own S_FULL / P_FULL / PV_DONE barrier.
+// While the softmax warps of tile x turn S_x,1(j) into P_x,1(j), the tensor core runs
+// O_x += P_x,0(j) V_j[0:64] and S_x,0(j+1), and the reverse for the other half, so a
+// tile's MMAs hide behind half a tile of its own softmax.  Each half is one step of the
+// online softmax (its own row max and lazy-rescale vote).
+//
+// Cost: each S MMA is M = 128, N = 64 (twice as many of them, each re-reading its Q~ tile
+// from shared memory); each P V MMA is M = 128, N = d, K = 64.
+//
+// MMA issue order for key tile j (the other tile's MMAs interleave):
+//   PV_a,0(j) S_a,0(j+1) PV_b,0(j) S_b,0(j+1) PV_a,1(j) S_a,1(j+1) PV_b,1(j) S_b,1(j+1)
+// (S_x,h(j+1) overwrites P_x,h(j) after the P V MMA that read it: one thread's tcgen05.mma
+// ops execute in issue order).
+//
+// Every wait is bounded, as in fwd_sm100.cu.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "common.h"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace ra {
+namespace {
+
+template <int D>
+struct SplitCfg {
+  static constexpr int BM = 128, BN = 128, HN = 64;  // query rows per tile, keys per tile, per half
+  static constexpr int NSK = 3, NSV = 2;             // K~ and V ring stages
+  static constexpr int CH = D / 64;                  // 64-column chunks per row
+  static constexpr uint32_t CHUNK = 128u * 128u;     // [128 rows][128 B]
+  static constexpr uint32_t TILE = CHUNK * CH;       // [128][D] 16-bit
+  static constexpr uint32_t HALF_ROWS = HN * 128u;   // byte offset of row 64 inside a chunk
+  static constexpr uint32_t OFF_Q = 0;               // Q~_a, Q~_b
+  static constexpr uint32_t OFF_K = 2 * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + NSK * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + NSV * TILE;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_O = 256;
+};
+
+enum SplitBar {
+  SB_Q_FULL = 0,
+  SB_K_FULL = 1,     // +stage (3)
+  SB_K_EMPTY = 4,    // +stage (3)
+  SB_V_FULL = 7,     // +stage (2)
+  SB_V_EMPTY = 9,    // +stage (2)
+  SB_S_FULL = 11,    // +2x+h: S_x,h(j) computed
+  SB_P_FULL = 15,    // +2x+h: P_x,h(j) written (and O_x rescaled); 4 warp arrivals
+  SB_PV_DONE = 19,   // +2x+h: O_x += P_x,h(j) V_j[64h : 64h+64] has completed
+  SB_O_DONE = 23,
+  SB_DRAIN = 24,
+  SB_COUNT = 25
+};
+static_assert(8 * SB_COUNT + 8 <= 256, "barriers, TMEM slot and abort flag fit the reserve");
+
+#ifndef RA_MMA_BATCH
+#define RA_MMA_BATCH 1
+#endif
+#ifndef RA_FWD_RESCALE_TAU
+#define RA_FWD_RESCALE_TAU 8.0f
+#endif
+constexpr float kSplitTau = RA_FWD_RESCALE_TAU;
+constexpr int kSplitThreads = 320;
+constexpr int kSplitProdWarp = 8, kSplitMmaWarp = 9;
+
+template <int D>
+__global__ void __launch_bounds__(kSplitThreads, 1)
+    fwd_split_sm100_kernel(const __grid_constant__ CUtensorMap map_q,
+                           const __grid_constant__ CUtensorMap map_k,
+                           const __grid_constant__ CUtensorMap map_v,
+                           __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int n, int BH,
+                           int causal, uint32_t* err, uint64_t wait_ns, int starve_block) {
+  using C = SplitCfg<D>;
+  constexpr int KID = K_FWD_SM100;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_s - raw_s);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * SB_COUNT);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * SB_COUNT + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int ntq = (n + C::BM - 1) / C::BM;
+  const int ntp = (ntq + 1) / 2;
+  const int T = ntp - 1 - (int)(blockIdx.x / BH);  // heaviest causal tile pairs first
+  const int bh = (int)(blockIdx.x % BH);
+  const int ntk = (n + C::BN - 1) / C::BN;
+  // key tiles of query tile x (0 when the tile lies past the end of the sequence)
+  auto nkv_of = [&](int x) -> int {
+    const int qt = 2 * T + x;
+    if (qt >= ntq) return 0;
+    return causal ? min(qt + 1, ntk) : ntk;
+  };
+  const int nkv_a = nkv_of(0), nkv_b = nkv_of(1);
+  const int nkv = max(nkv_a, nkv_b);
+  const bool has_b = nkv_b > 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < SB_COUNT; ++i)
+      mbar_init(&bar[i], (i >= SB_P_FULL && i < SB_P_FULL + 4) ? 4 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kSplitMmaWarp) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kSplitProdWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      // starve_block (test hook, -1 = off): that CTA never loads Q~, so its issuer's
+      // bounded wait must expire and report RA_ERR_TIMEOUT instead of hanging.
+      const bool load_q = (int)blockIdx.x != starve_block;
+      if (load_q) {
+        mbar_arrive_expect_tx(&bar[SB_Q_FULL], (has_b ? 2 : 1) * C::TILE);
+        for (int x = 0; x < (has_b ? 2 : 1); ++x)
+          for (int c = 0; c < C::CH; ++c)
+            tma_load_3d(base + C::OFF_Q + x * C::TILE + c * C::CHUNK, &map_q, &bar[SB_Q_FULL],
+                        c * 64, (2 * T + x) * C::BM, bh);
+      }
+      int issued_k = -1, issued_v = -1;
+      auto load_k = [&](int j) -> bool {
+        const int s = j % C::NSK;
+        if (!mbar_wait(&bar[SB_K_EMPTY + s], ((j / C::NSK) & 1) ^ 1, abort_flag, err, KID, 1,
+                       wait_ns))
+          return false;
+        mbar_arrive_expect_tx(&bar[SB_K_FULL + s], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(base + C::OFF_K + s * C::TILE + c * C::CHUNK, &map_k, &bar[SB_K_FULL + s],
+                      c * 64, j * C::BN, bh);
+        issued_k = j;
+        return true;
+      };
+      // K~ runs one tile ahead of V: the S MMAs of tile j + 1 follow the P V MMAs of tile j
+      bool ok = nkv > 0 ? load_k(0) : true;
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv && !load_k(j + 1)) break;
+        const int s = j % C::NSV;
+        if (!mbar_wait(&bar[SB_V_EMPTY + s], ((j / C::NSV) & 1) ^ 1, abort_flag, err, KID, 2,
+                       wait_ns))
+          break;
+        mbar_arrive_expect_tx(&bar[SB_V_FULL + s], C::TILE);
+        for (int c = 0; c < C::CH; ++c)
+          tma_load_3d(base + C::OFF_V + s * C::TILE + c * C::CHUNK, &map_v, &bar[SB_V_FULL + s],
+                      c * 64, j * C::BN, bh);
+        issued_v = j;
+      }
+      if (*abort_flag) {
+        // Let every copy already in flight land before the CTA's shared memory goes away.
+        int dummy = 0;
+        if (load_q) mbar_wait(&bar[SB_Q_FULL], 0, &dummy, err, KID, 20, wait_ns);
+        for (int j = max(0, issued_k - C::NSK + 1); j <= issued_k; ++j)
+          mbar_wait(&bar[SB_K_FULL + j % C::NSK], (j / C::NSK) & 1, &dummy, err, KID, 21, wait_ns);
+        for (int j = max(0, issued_v - C::NSV + 1); j <= issued_v; ++j)
+          mbar_wait(&bar[SB_V_FULL + j % C::NSV], (j / C::NSV) & 1, &dummy, err, KID, 22, wait_ns);
+      }
+    }
+  } else if (warp == kSplitMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idS = idesc_f16_f32(128, C::HN, 0, 0);  // fp16 Q~, K~ half
+    constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);     // bf16 P half, V half
+    const SDesc dkm = sdesc_split(base_s, 16, 1024);        // K-major tiles
+    const SDesc dmn = sdesc_split(base_s, C::CHUNK, 1024);  // V tiles read MN-major
+    bool ok = mbar_wait_warp(&bar[SB_Q_FULL], 0, abort_flag, err, KID, 3, wait_ns);
+    tc_fence_after();
+    const int nkv_x[2] = {nkv_a, nkv_b};
+    // S_x,h(j) = Q~_x K~_j[64h : 64h + 64]^T into TMEM columns 128x + 64h (K~_j waited for)
+    auto issue_s = [&](int x, int h, int j) {
+      const SDesc ks =
+          sdesc_advance(dkm, C::OFF_K + (j % C::NSK) * C::TILE + (uint32_t)h * C::HALF_ROWS);
+      const uint32_t q_off = C::OFF_Q + x * C::TILE;
+      const uint32_t dst = tmem + C::COL_S + x * 128 + h * C::HN;
+      if constexpr (D == 128 && RA_MMA_BATCH) {
+        mma8_kmajor<false, C::CHUNK, C::CHUNK>(dst, sdesc_at(dkm, q_off), sdesc_at(ks, 0), idS,
+                                               0);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss_warp(dst, sdesc_at(dkm, q_off + koff), sdesc_at(ks, koff), idS, kk > 0);
+        }
+      }
+      mma_commit_warp(&bar[SB_S_FULL + 2 * x + h]);
+    };
+    auto wait_k = [&](int j) -> bool {
+      if (!mbar_wait_warp(&bar[SB_K_FULL + j % C::NSK], (j / C::NSK) & 1, abort_flag, err, KID,
+                          4, wait_ns))
+        return false;
+      tc_fence_after();
+      return true;
+    };
+    if (ok && nkv > 0) {
+      ok = wait_k(0);
+      if (ok) {
+        for (int h = 0; h < 2; ++h)
+          for (int x = 0; x < 2; ++x)
+            if (nkv_x[x] > 0) issue_s(x, h, 0);
+        mma_commit_warp(&bar[SB_K_EMPTY + 0]);
+      }
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const bool next = j + 1 < nkv;
+      if (next && !(ok = wait_k(j + 1))) break;
+      if (!(ok = mbar_wait_warp(&bar[SB_V_FULL + j % C::NSV], (j / C::NSV) & 1, abort_flag, err,
+                                KID, 7, wait_ns)))
+        break;
+      for (int h = 0; ok && h < 2; ++h) {
+        for (int x = 0; x < 2; ++x) {
+          if (j >= nkv_x[x]) continue;
+          if (!(ok = mbar_wait_warp(&bar[SB_P_FULL + 2 * x + h], j & 1, abort_flag, err, KID, 6,
+                                    wait_ns)))
+            break;
+          tc_fence_after();
+          // O_x += P_x,h(j) V_j[64h : 64h + 64] with P_x,h read from TMEM
+          const SDesc vs = sdesc_advance(
+              dmn, C::OFF_V + (j % C::NSV) * C::TILE + (uint32_t)h * C::HALF_ROWS);
+          const uint32_t pa = tmem + C::COL_S + x * 128 + h * C::HN;
+          if constexpr (RA_MMA_BATCH) {
+            mma4_ts_mn<8, 16, 24>(tmem + C::COL_O + x * 128, pa, sdesc_at(vs, 0), idO,
+                                  (j > 0 || h > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < C::HN / 16; ++kk)
+              mma_ts_warp(tmem + C::COL_O + x * 128, pa + kk * 8, sdesc_at(vs, kk * 2048), idO,
+                          (j > 0 || h > 0 || kk > 0));
+          }
+          mma_commit_warp(&bar[SB_PV_DONE + 2 * x + h]);
+          if (next && j + 1 < nkv_x[x]) issue_s(x, h, j + 1);
+        }
+      }
+      if (!ok) break;
+      mma_commit_warp(&bar[SB_V_EMPTY + j % C::NSV]);
+      if (next) mma_commit_warp(&bar[SB_K_EMPTY + (j + 1) % C::NSK]);
+    }
+    if (ok) mma_commit_warp(&bar[SB_O_DONE]);
+    // Every MMA issued above has finished once this commit arrives.
+    mma_commit_warp(&bar[SB_DRAIN]);
+    int dummy = 0;
+    mbar_wait_warp(&bar[SB_DRAIN], 0, &dummy, err, KID, 23, wait_ns);
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int x = warp / 4;            // query tile a (0) or b (1)
+    const int t = threadIdx.x % 128;   // row within the tile == TMEM lane
+    const int qt = 2 * T + x;
+    const int row = qt * C::BM + t;
+    const int my_nkv = x == 0 ? nkv_a : nkv_b;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t s_base = lane_base + C::COL_S + x * 128;
+    const uint32_t o_base = lane_base + C::COL_O + x * 128;
+    const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+    float m = -CUDART_INF_F, l = 0.f;  // running max (log2 units, scaled) and row sum
+    bool ok = true;
+    for (int j = 0; ok && j < my_nkv; ++j) {
+      const int key0 = j * C::BN;
+      // columns of this row that hold a key (all of them except on the diagonal tile and
+      // the ragged last tile)
+      const bool need_mask = (key0 + C::BN > n) || (causal && j == qt);
+      const int nvalid =
+          need_mask ? max(0, min(C::BN, (causal ? min(n, row + 1) : n) - key0)) : C::BN;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!mbar_wait_warp(&bar[SB_S_FULL + 2 * x + h], j & 1, abort_flag, err, KID, 8,
+                            wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sh = s_base + h * C::HN;
+        const int nv = min(C::HN, max(0, nvalid - h * C::HN));  // valid columns of this half
+        uint32_t sr[2][32];
+        tmem_ld32(sh, sr[0]);
+        tmem_ld32(sh + 32, sr[1]);
+        tmem_wait_ld(sr[0]);
+        tmem_wait_ld(sr[1]);
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * c + i >= nv) sr[c][i] = __float_as_uint(-CUDART_INF_F);
+        }
+        // the row max of this half's raw scores (masked entries are -inf)
+        float mp[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mp[a] = __uint_as_float(sr[0][a]);
+#pragma unroll
+        for (int i = 8; i < 64; ++i)
+          mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
+        const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * scale_log2;
+        // lazy rescale: move the reference max only when some row of the warp needs it
+        const bool need = mt > m + kSplitTau;
+        const bool warp_rescale = __any_sync(0xffffffffu, need);
+        float corr = 1.f;
+        if (warp_rescale) {
+          const float m_new = fmaxf(m, mt);
+          corr = fast_exp2(m - m_new);  // 0 on the first half-tile (m = -inf)
+          m = m_new;
+        }
+        const float m_use = m == -CUDART_INF_F ? 0.f : m;
+        // P = 2^(s scale - m), summed and written as bf16 over the half: columns 32c..32c+31
+        // of the half land in its columns 16c..16c+15 (masked entries give 2^-inf = 0)
+        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float pv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            pv[i] = fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_use));
+          if (need_mask) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * c + i >= nv) pv[i] = 0.f;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sp[i & 7] += pv[i];
+#pragma unroll
+          for (int i2 = 0; i2 < 16; ++i2) w[i2] = pack_bf16x2(pv[2 * i2], pv[2 * i2 + 1]);
+          tmem_st16(sh + 16 * c, w);
+        }
+        l = l * corr +
+            (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
+        tmem_wait_st();
+        if (warp_rescale && (j > 0 || h > 0)) {
+          // O_x must hold every earlier half's P V before it is rescaled: wait for the P V
+          // MMA of the previous half (half 0 of this tile, or half 1 of the last one)
+          const int ph = h ^ 1, pj = h ? j : j - 1;
+          if (!mbar_wait_warp(&bar[SB_PV_DONE + 2 * x + ph], pj & 1, abort_flag, err, KID, 11,
+                              wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(o_base + 32 * c, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+            tmem_st32(o_base + 32 * c, r);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[SB_P_FULL + 2 * x + h]);
+      }
+    }
+    if (ok && my_nkv > 0 &&
+        mbar_wait_warp(&bar[SB_O_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(o_base + 32 * c, r);
+        tmem_wait_ld(r);
+        if (row < n) {
+          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * n + row) * D + 32 * c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float* f = reinterpret_cast<const float*>(&r[8 * u]);
+            dst[u] = make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv),
+                                pack_bf16x2(f[2] * inv, f[3] * inv),
+                                pack_bf16x2(f[4] * inv, f[5] * inv),
+                                pack_bf16x2(f[6] * inv, f[7] * inv));
+          }
+        }
+      }
+      if (row < n) lse[(size_t)bh * n + row] = (m + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kSplitMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_split_d(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
+                           const DevCtl& ctl, cudaStream_t s) {
+  using C = SplitCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(fwd_split_sm100_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int BH = (int)(p.B * p.H);
+  const long long ntq = (p.n + C::BM - 1) / C::BM;
+  const long long ntp = (ntq + 1) / 2;
+  fwd_split_sm100_kernel<D><<<(unsigned)(ntp * BH), kSplitThreads, C::SMEM, s>>>(
+      maps.qt, maps.kt, maps.v, (__nv_bfloat16*)o, lse, (int)p.n, BH, p.causal, ctl.err,
+      ctl.wait_ns, ctl.starve_block);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_split_sm100(const ra_problem& p, const Sm100Maps& maps, void* o,
+                                   float* lse, const DevCtl& ctl, cudaStream_t s) {
+  if (p.d == 64) return launch_split_d<64>(p, maps, o, lse, ctl, s);
+  return launch_split_d<128>(p, maps, o, lse, ctl, s);
+}
+
+}  // namespace ra

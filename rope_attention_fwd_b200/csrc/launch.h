@@ -50,6 +50,10 @@ struct Sm100Maps {
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
+// The same forward with each 128-key S tile handled as two 64-column halves on their own
+// barriers (fwd_split_sm100.cu); chosen per call by RA_FWD_SPLIT_S=1, off by default.
+cudaError_t launch_fwd_split_sm100(const ra_problem& p, const Sm100Maps& maps, void* o,
+                                   float* lse, const DevCtl& ctl, cudaStream_t s);
 // Padded per-row vectors for the tensor-core backward, delta and lse * log2(e), plus
 // max_i |dO_i| into stats[0] and max_j |v_j| into stats[1] (fp32 bits, atomic max; stats
 // zeroed by the caller), in one pass over O, dO and V.

@@ -1,10 +1,11 @@
-// blas.h -- the library's cuBLAS handle (one per device, created on first use).
+// blas.h -- the library's cuBLAS handles (one per host thread and device, created on
+// first use).
 #pragma once
 #include <cublas_v2.h>
 
 namespace ra {
 
-// The current device's handle, or nullptr if it cannot be created.
+// This thread's handle for the current device, or nullptr if it cannot be created.
 cublasHandle_t cublas_handle();
 
 }  // namespace ra

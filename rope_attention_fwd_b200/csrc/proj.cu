@@ -18,7 +18,6 @@
 #include <cublas_v2.h>
 #include <cuda_runtime.h>
 
-#include <mutex>
 #include <unordered_map>
 
 #include "blas.h"
@@ -27,20 +26,18 @@
 
 namespace ra {
 
-namespace {
-std::mutex g_cublas_mu;
-std::unordered_map<int, cublasHandle_t> g_cublas;  // one handle per device
-}  // namespace
-
+// One handle per host thread and device: every call sets the handle's stream, so two
+// threads must not share one (a handle is not safe for concurrent use).  Handles live until
+// the process exits.
 cublasHandle_t cublas_handle() {
+  thread_local std::unordered_map<int, cublasHandle_t> handles;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  std::lock_guard<std::mutex> g(g_cublas_mu);
-  auto it = g_cublas.find(dev);
-  if (it != g_cublas.end()) return it->second;
+  auto it = handles.find(dev);
+  if (it != handles.end()) return it->second;
   cublasHandle_t h = nullptr;
   if (cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
-  g_cublas[dev] = h;
+  handles[dev] = h;
   return h;
 }
 

@@ -112,6 +112,12 @@ bool fwd_split_s() {
   return s && std::atoi(s) == 1;
 }
 
+// RA_BWD_DKDV_TMEM=1 selects the dK/dV kernel with K~ and V as TMEM operands, read per call.
+bool dkdv_tmem() {
+  const char* s = std::getenv("RA_BWD_DKDV_TMEM");
+  return s && std::atoi(s) == 1;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -286,8 +292,17 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
         !make_map(&maps.v64, v, *p, 64) || !make_map(&maps.dO64, dO, *p, 64))
       return RA_ERR_CUDA;
     DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
-    RA_LAUNCH(K_BWD_DKDV_SM100, s,
-              launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl, s));
+    if (dkdv_tmem()) {
+      if (!make_map(&maps.qt32, qt, *p, 32, true) || !make_map(&maps.dO32, dO, *p, 32))
+        return RA_ERR_CUDA;
+      RA_LAUNCH(K_BWD_DKDV_SM100, s,
+                launch_bwd_dkdv_tmem_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart,
+                                           ctl, s));
+    } else {
+      RA_LAUNCH(K_BWD_DKDV_SM100, s,
+                launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
+                                      s));
+    }
     RA_LAUNCH(K_BWD_DQ_SM100, s,
               launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
   }

@@ -1,6 +1,7 @@
 """Benchmark: RoPE/LeRoPE attention fwd + loss + bwd (incl. dalpha) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+    python bench.py --profile --shape B,H,n,d [--causal] [--steps K] [--warmup W] [--d-model M]
 
 One step = the whole path on one batch: rope_attn_fwd (table, rotation, tcgen05
 forward), rope_attn_loss, rope_attn_bwd_saved (Delta, dK/dV, dQ, dalpha from the table and
@@ -170,7 +171,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     from rope_attention_fwd_b200 import binding as rb
-    from rope_attention_fwd_b200.dist import allreduce_dalpha, rank_seed
+    from rope_attention_fwd_b200.dist import allreduce_sum, rank_seed
     from rope_attention_fwd_b200.inputs import make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -207,7 +208,9 @@ def run_ours(args):
         # the backward takes the table and rotated Q~, K~ the forward just wrote into ws
         rb.rope_attn_bwd_saved(t["v"], o, lse, dO, t["alpha"], wl.base, wl.causal, ws,
                                dq=dq, dk=dk, dv=dvv, dalpha=dalpha)
-        allreduce_dalpha(dalpha)  # sum over every head of every rank (no-op on one GPU)
+        # L and dalpha are sums over every head of every rank (no-ops on one GPU)
+        allreduce_sum(L)
+        allreduce_sum(dalpha)
 
     def barrier():
         if world > 1:
@@ -247,18 +250,20 @@ def run_ours(args):
     value = world * flops / (ms * 1e-3) / 1e12
     launches = sum(c for c, _ in kernels.values())
 
-    # ---------------- end-to-end through host buffers (copies inside the timed region)
+    # ---------------- end-to-end through host buffers (copies inside the timed region):
+    # every step's inputs go host -> device from pinned memory, and every result of the
+    # step (O, lse, L, dO's gradients dQ, dK, dV, and dalpha) comes back device -> host
     h2d = sum(host[x].numel() * host[x].element_size() for x in host)
-    d2h = 4 + 4 * (wl.d // 2)
-    L_host = torch.empty((), dtype=torch.float32).pin_memory()
-    da_host = torch.empty(wl.d // 2, dtype=torch.float32).pin_memory()
+    results = {"o": o, "lse": lse, "L": L, "dq": dq, "dk": dk, "dv": dvv, "dalpha": dalpha}
+    back = {x: torch.empty(t.shape, dtype=t.dtype).pin_memory() for x, t in results.items()}
+    d2h = sum(t.numel() * t.element_size() for t in back.values())
     e2e_steps = max(3, args.steps // 2)
 
     def e2e_step():
         t = {x: host[x].to(dev, non_blocking=True) for x in host}
         step(t)
-        L_host.copy_(L, non_blocking=True)
-        da_host.copy_(dalpha, non_blocking=True)
+        for x, res in results.items():
+            back[x].copy_(res, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -378,6 +383,77 @@ def code_only(text):
     return "\n".join(line for line in lines if line)
 
 
+# ----------------------------------------------------------------- profile mode
+def run_profile(args):
+    """Whole fwd -> loss -> bwd steps on one problem of any shape, for profilers (ncu wraps
+    this): inputs N(0,1) bf16 drawn on the device (the launch sequence matters here, not
+    parity), alpha ~ N(0, 0.3^2).  Prints each kernel's average event time over the timed
+    steps.  With --d-model > 0 each step also runs the projections around the path
+    (q, k, v = x W before; dW and dx after) and prints their times and TFLOP/s."""
+    import torch
+    from rope_attention_fwd_b200 import binding as rb
+    B, H, n, d = args.shape
+    g = torch.Generator(device="cuda").manual_seed(0)
+    shape = (B, H, n, d)
+    q, k, v, e = (torch.randn(shape, device="cuda", generator=g).to(torch.bfloat16)
+                  for _ in range(4))
+    alpha = 0.3 * torch.randn(d // 2, device="cuda", generator=g)
+    ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base), "cuda")
+    proj_ms = {"proj_fwd": 0.0, "proj_bwd": 0.0}
+    if args.d_model > 0:
+        x = torch.randn((B, n, args.d_model), device="cuda", generator=g).to(torch.bfloat16)
+        w = [(torch.randn((args.d_model, H * d), device="cuda", generator=g)
+              * args.d_model ** -0.5).to(torch.bfloat16) for _ in range(3)]
+
+    def timed(name, fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out = fn()
+        e1.record()
+        e1.synchronize()
+        proj_ms[name] += e0.elapsed_time(e1)
+        return out
+
+    def step():
+        qq, kk, vv = (q, k, v) if args.d_model <= 0 else timed(
+            "proj_fwd", lambda: rb.rope_attn_proj_fwd(x, *w, H))
+        o, lse = rb.rope_attn_fwd(qq, kk, vv, alpha, args.base, args.causal, ws=ws)
+        L, dO = rb.rope_attn_loss(o, e, ws=ws)
+        grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws)
+        if args.d_model > 0:
+            timed("proj_bwd", lambda: rb.rope_attn_proj_bwd(x, *w, *grads[:3]))
+        return grads
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    proj_ms = {k2: 0.0 for k2 in proj_ms}
+    rb.rope_attn_timing_read()
+    rb.rope_attn_timing_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    rb.rope_attn_timing_enable(False)
+    f = 0.5 if args.causal else 1.0
+    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0, "bwd_fused_sm100": 10.0}
+    for name, (cnt, ms) in rb.rope_attn_timing_read().items():
+        line = f"{name:16s} {cnt:3d} launches {ms / cnt:8.3f} ms"
+        if name in alg:
+            tf = alg[name] * B * H * n * n * d * f / (ms / cnt * 1e-3) / 1e12
+            line += f"  {tf:7.1f} TFLOP/s algorithmic"
+        print(line)
+    if args.d_model > 0:
+        prod = 2.0 * B * n * args.d_model * H * d  # FLOPs of one x W product
+        for name, nprod in (("proj_fwd", 3), ("proj_bwd", 6)):
+            ms = proj_ms[name] / args.steps
+            print(f"{name:16s}   1 launches {ms:8.3f} ms  "
+                  f"{nprod * prod / (ms * 1e-3) / 1e12:7.1f} TFLOP/s")
+    code, info = rb.rope_attn_device_status(ws)
+    if code != 0:
+        raise SystemExit(f"device status {rb.STATUS.get(code, code)} {info}")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -386,7 +462,18 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=3, choices=[2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="time the kernels of whole steps on --shape (for profilers); no "
+                         "JSON line")
+    ap.add_argument("--shape", type=lambda t: tuple(int(x) for x in t.split(",")),
+                    default=(2, 16, 8192, 128), help="B,H,n,d of --profile")
+    ap.add_argument("--causal", action="store_true", help="causal masking in --profile")
+    ap.add_argument("--base", type=float, default=1e4, help="RoPE base in --profile")
+    ap.add_argument("--d-model", type=int, default=0,
+                    help="--profile: also run the projections with this model width")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be at least 3")
     # the reference arm times a slow CPU program: bound its work per step

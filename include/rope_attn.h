@@ -83,13 +83,23 @@ typedef struct {
                             rotated (theta_hat_m = 0, dalpha_m = 0): partial RoPE, the
                             p-RoPE baseline of "LeRoPE" (Configuracao Experimental) with
                             p = 1 - fixed_bands / (d/2); 0 = every band rotates        */
-    int32_t reserved;    /* must be 0                                             */
+    int32_t flags;       /* 0 or RA_FLAG_DETERMINISTIC                           */
 } ra_problem;
+
+/* ra_problem.flags: the bf16 backward with d = 128 adds the dQ contribution of every
+ * 128-key block into an fp32 accumulator in ws as soon as it is formed (one pass over the
+ * key/query tile pairs), so dQ depends on the order in which blocks add (the last bits of
+ * fp32 sums; in bf16, a one-unit difference in a rare element).  dK, dV and dalpha stay
+ * bitwise reproducible.  RA_FLAG_DETERMINISTIC selects the two-pass backward instead
+ * (dK/dV, then dQ recomputing the scores), bitwise reproducible in every output, at about
+ * 1.4x the backward time.  Other d, and fp32 problems, always take the two-pass form. */
+#define RA_FLAG_DETERMINISTIC 1
 
 /* Bytes of workspace the calls below need for problem *p (0 if *p is invalid).
  * Holds: the fp32 cos/sin table [n, d/2, 2], the rotated Q~ and K~ in the
  * problem dtype, rowsum(dO o O) [B, H, n] fp32, per-tile dalpha partials,
- * loss partials and the device error word. */
+ * loss partials, the device error word and (fused bf16 backward, d = 128) an fp32
+ * [B, H, n, d] dQ accumulator. */
 size_t rope_attn_workspace_bytes(const ra_problem* p);
 
 /* Forward: o = softmax(Q~ K~^T / sqrt(d)) V and lse (natural log) from q, k, v
@@ -105,7 +115,8 @@ ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e,
 
 /* Backward: dq, dk, dv ([B,H,n,d], dtype) and dalpha ([d/2], fp32, summed over
  * every batch and head) from q, k, v, the forward's o and lse, the upstream
- * gradient dO and alpha.  Deterministic: no atomics, fixed-order reductions.
+ * gradient dO and alpha.  dk, dv and dalpha are reduced in a fixed order (bitwise
+ * reproducible); dq too unless the fused form is taken (see ra_problem.flags).
  * Recomputes the table, Q~ and K~ in ws (it does not rely on a previous fwd). */
 ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
                         const void* o, const float* lse, const void* dO, const float* alpha,
@@ -220,12 +231,20 @@ const char* rope_attn_status_string(ra_status s);
  *     contents.  Each call clears the error word and rewrites every region it reads,
  *     but calls that overlap on the GPU (other streams, other host threads) race on
  *     the array: issue them on one stream.
- *   - Device-side wait timeouts are recorded in the array's own error word, which no
- *     entry point reads back; use rope_attn_fwd with a workspace and
- *     rope_attn_device_status when that status is needed. */
+ *   - Device: the tensors must live on the current device (the array used is that
+ *     device's copy).
+ *   - Device-side errors (a wait timeout, RA_ERR_TIMEOUT, or a rotated entry beyond the
+ *     fp16 range, RA_ERR_RANGE) are recorded in the array's own error word; the call's
+ *     return value cannot show them (it returns before the kernels run).  Read them with
+ *     rope_attn_noalloc_status. */
 #define RA_NOALLOC_SCRATCH_BYTES (8u << 20)
 ra_status rope_attn_fwd_noalloc(const ra_problem* p, const void* q, const void* k, const void* v,
                                 const float* alpha, void* o, float* lse, void* stream);
+
+/* Synchronises `stream`, then reads and clears the error word of the current device's
+ * static array: RA_OK, RA_ERR_TIMEOUT (info as for rope_attn_device_status) or RA_ERR_RANGE
+ * from the most recent rope_attn_fwd_noalloc on this device.  Allocates nothing. */
+ra_status rope_attn_noalloc_status(void* stream, int32_t info[3]);
 
 /* ---- optional per-kernel timing (instrumentation, off by default) --------
  * While enabled, every kernel launch made by the calls above is bracketed by

@@ -95,15 +95,6 @@ def rotate(x, phi, pairing="interleaved", sign=1.0):
     return y
 
 
-def j_pair(x, pairing="interleaved"):
-    """J x band-wise: (x0, x1) -> (-x1, x0)."""
-    i0, i1 = band_index(x.shape[-1], pairing)
-    y = np.empty_like(x, dtype=np.float64)
-    y[..., i0] = -x[..., i1]
-    y[..., i1] = x[..., i0]
-    return y
-
-
 # --------------------------------------------------------------------------
 # steps 3-7 for one head, in blocks of full query rows
 # --------------------------------------------------------------------------

@@ -14,6 +14,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "librope_attn.so")
 
 RA_F32, RA_BF16 = 0, 1
+RA_FLAG_DETERMINISTIC = 1
 _DTYPE = {torch.float32: RA_F32, torch.bfloat16: RA_BF16}
 STATUS = {0: "RA_OK", 1: "RA_ERR_INVALID_ARG", 2: "RA_ERR_UNSUPPORTED", 3: "RA_ERR_WORKSPACE",
           4: "RA_ERR_CUDA", 5: "RA_ERR_TIMEOUT", 6: "RA_ERR_RANGE"}
@@ -23,7 +24,7 @@ class RaProblem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("n", ctypes.c_int64),
                 ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
                 ("base", ctypes.c_double), ("fixed_bands", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("flags", ctypes.c_int32)]
 
 
 class RaAdam(ctypes.Structure):
@@ -74,6 +75,8 @@ def lib():
         L.rope_attn_spectrum.restype = ctypes.c_int
         L.rope_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.rope_attn_fwd_noalloc.restype = ctypes.c_int
+        L.rope_attn_noalloc_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+        L.rope_attn_noalloc_status.restype = ctypes.c_int
         L.rope_attn_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)]
         L.rope_attn_device_status.restype = ctypes.c_int
         L.rope_attn_status_string.argtypes = [ctypes.c_int]
@@ -89,17 +92,18 @@ def lib():
     return _lib
 
 
-def problem(B, H, n, d, dtype, causal, base, fixed_bands=0):
-    """fixed_bands: the slowest bands left unrotated (partial RoPE; 0 = all rotate)."""
+def problem(B, H, n, d, dtype, causal, base, fixed_bands=0, deterministic=False):
+    """fixed_bands: the slowest bands left unrotated (partial RoPE; 0 = all rotate).
+    deterministic: the two-pass backward, bitwise reproducible dQ (RA_FLAG_DETERMINISTIC)."""
     if isinstance(dtype, torch.dtype):
         dtype = _DTYPE[dtype]
     return RaProblem(int(B), int(H), int(n), int(d), int(dtype), int(bool(causal)), float(base),
-                     int(fixed_bands), 0)
+                     int(fixed_bands), RA_FLAG_DETERMINISTIC if deterministic else 0)
 
 
-def _problem_of(q, causal, base, fixed_bands=0):
+def _problem_of(q, causal, base, fixed_bands=0, deterministic=False):
     B, H, n, d = q.shape
-    return problem(B, H, n, d, q.dtype, causal, base, fixed_bands)
+    return problem(B, H, n, d, q.dtype, causal, base, fixed_bands, deterministic)
 
 
 def _ptr(t):
@@ -156,10 +160,22 @@ def rope_attn_fwd_noalloc(q, k, v, alpha, base, causal, o=None, lse=None, fixed_
     B, H, n, d = q.shape
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
-    _check("rope_attn_fwd_noalloc", lib().rope_attn_fwd_noalloc(
-        ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
-        _stream(q.device)))
+    # the library uses the static array of the CURRENT device: make it q's
+    with torch.cuda.device(q.device):
+        _check("rope_attn_fwd_noalloc", lib().rope_attn_fwd_noalloc(
+            ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
+            _stream(q.device)))
     return o, lse
+
+
+def rope_attn_noalloc_status(device):
+    """Synchronise the device's current stream and return (status code, [kernel, site,
+    block]) from the static array's error word (read and cleared)."""
+    device = torch.device(device)
+    info = (ctypes.c_int32 * 3)()
+    with torch.cuda.device(device):
+        code = lib().rope_attn_noalloc_status(_stream(device), info)
+    return code, list(info)
 
 
 def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
@@ -176,10 +192,11 @@ def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
 
 
 def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk=None, dv=None,
-                  dalpha=None, fixed_bands=0, frozen_alpha=False):
+                  dalpha=None, fixed_bands=0, frozen_alpha=False, deterministic=False):
     """(dq, dk, dv, dalpha) of L for upstream gradient dO.  frozen_alpha: the frequencies
-    are not trained; no dalpha is computed and None is returned in its place."""
-    prob = _problem_of(q, causal, base, fixed_bands)
+    are not trained; no dalpha is computed and None is returned in its place.
+    deterministic: the two-pass backward (dQ bitwise reproducible too)."""
+    prob = _problem_of(q, causal, base, fixed_bands, deterministic)
     if ws is None:
         ws = workspace(prob, q.device)
     dq = torch.empty_like(q) if dq is None else dq
@@ -197,10 +214,10 @@ def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk
 
 
 def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None, dv=None,
-                        dalpha=None, fixed_bands=0, frozen_alpha=False):
+                        dalpha=None, fixed_bands=0, frozen_alpha=False, deterministic=False):
     """rope_attn_bwd from the table, Q~ and K~ the preceding rope_attn_fwd left in ws
     (same problem, q, k and alpha; see include/rope_attn.h)."""
-    prob = _problem_of(v, causal, base, fixed_bands)
+    prob = _problem_of(v, causal, base, fixed_bands, deterministic)
     dq = torch.empty_like(v) if dq is None else dq
     dk = torch.empty_like(v) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

@@ -78,7 +78,8 @@ ra_status check_problem(const ra_problem* p) {
   if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
   if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
   if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
-  if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 || p->reserved != 0)
+  if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 ||
+      (p->flags & ~RA_FLAG_DETERMINISTIC) != 0)
     return RA_ERR_INVALID_ARG;
   if (p->d > 128) return RA_ERR_UNSUPPORTED;
   if (p->dtype == RA_BF16 && p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
@@ -292,7 +293,16 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
         !make_map(&maps.v64, v, *p, 64) || !make_map(&maps.dO64, dO, *p, 64))
       return RA_ERR_CUDA;
     DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
-    if (dkdv_tmem()) {
+    if (uses_fused_bwd(*p)) {
+      float* dqacc = at<float>(ws, L.dqacc);
+      if (cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)(p->B * p->H * p->n * p->d), s) !=
+          cudaSuccess)
+        return RA_ERR_CUDA;
+      RA_LAUNCH(K_BWD_FUSED_SM100, s,
+                launch_bwd_fused_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dqacc,
+                                       dpart, ctl, s));
+      RA_LAUNCH(K_DQ_FINISH, s, launch_dq_finish(*p, dqacc, table, stats, dq, s));
+    } else if (dkdv_tmem()) {
       if (!make_map(&maps.qt32, qt, *p, 32, true) || !make_map(&maps.dO32, dO, *p, 32))
         return RA_ERR_CUDA;
       RA_LAUNCH(K_BWD_DKDV_SM100, s,
@@ -303,8 +313,9 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
                 launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
                                       s));
     }
-    RA_LAUNCH(K_BWD_DQ_SM100, s,
-              launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
+    if (!uses_fused_bwd(*p))
+      RA_LAUNCH(K_BWD_DQ_SM100, s,
+                launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
   }
   if (dalpha) RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;
@@ -404,7 +415,8 @@ const char* rope_attn_kernel_name(int id) {
   static const char* names[K_COUNT] = {
       "rope_table",       "rotate",       "fwd_f32",      "fwd_sm100",
       "loss_partial",     "loss_final",   "bwd_delta",    "bwd_dq_f32",
-      "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final"};
+      "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final",
+      "bwd_fused_sm100",  "dq_finish"};
   return (id >= 0 && id < K_COUNT) ? names[id] : "unknown";
 }
 

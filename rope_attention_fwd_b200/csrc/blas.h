@@ -1,5 +1,5 @@
 // blas.h -- the library's cuBLAS handles (one per host thread and device, created on
-// first use).
+// first use, destroyed when the thread exits).
 #pragma once
 #include <cublas_v2.h>
 

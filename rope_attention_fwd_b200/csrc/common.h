@@ -21,7 +21,9 @@ enum KernelId : int {
   K_BWD_DQ_SM100 = 9,
   K_BWD_DKDV_SM100 = 10,
   K_DALPHA = 11,
-  K_COUNT = 12
+  K_BWD_FUSED_SM100 = 12,
+  K_DQ_FINISH = 13,
+  K_COUNT = 14
 };
 
 // Rows per dalpha partial (one partial per band per tile of query or key rows).
@@ -41,8 +43,15 @@ struct WsLayout {
   size_t delta;      // float [B*H][npad]   rowsum(dO o O); 0 on rows >= n
   size_t lse2;       // float [B*H][npad]   lse * log2(e); +inf on rows >= n
   size_t dpart;      // float [2][B*H][ceil(n/kDalphaRows)][M]
+  size_t dqacc;      // float [B*H][n][d]: dQ~ accumulator of the fused backward (bf16, d = 128)
   size_t total;
 };
+
+// The bf16 backward with d = 128 runs the fused dK/dV/dQ kernel (an fp32 dQ~ accumulator in
+// the workspace) unless the caller asks for bitwise-reproducible dQ (RA_FLAG_DETERMINISTIC).
+inline bool uses_fused_bwd(const ra_problem& p) {
+  return p.dtype == RA_BF16 && p.d == 128 && (p.flags & RA_FLAG_DETERMINISTIC) == 0;
+}
 
 // Rows of the padded per-row vectors (a whole number of 128-row tiles).
 inline int64_t padded_rows(int64_t n) { return (n + 127) / 128 * 128; }
@@ -68,6 +77,7 @@ inline WsLayout ws_layout(const ra_problem& p) {
   w.delta = take(sizeof(float) * BH * npad);
   w.lse2 = take(sizeof(float) * BH * npad);
   w.dpart = take(sizeof(float) * 2 * BH * ntile * M);
+  w.dqacc = take(uses_fused_bwd(p) ? sizeof(float) * BH * n * d : 0);
   w.total = off;
   return w;
 }

@@ -73,6 +73,14 @@ cudaError_t launch_bwd_dkdv_tmem_sm100(const ra_problem& p, const Sm100Maps& map
                                        const float2* table, const uint32_t* stats, void* dk,
                                        void* dv, float* dpart, const DevCtl& ctl,
                                        cudaStream_t s);
+// Fused dK, dV and dQ~ (into the fp32 accumulator dqacc, zeroed by the caller) in one pass
+// (d = 128); dq_finish turns the accumulator into dQ.
+cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,
+                                   const float* lse2p, const float* deltap, const float2* table,
+                                   const uint32_t* stats, void* dk, void* dv, float* dqacc,
+                                   float* dpart, const DevCtl& ctl, cudaStream_t s);
+cudaError_t launch_dq_finish(const ra_problem& p, const float* dqacc, const float2* table,
+                             const uint32_t* stats, void* dq, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
                                 const float* deltap, const float2* table, const uint32_t* stats,
                                 void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s);

@@ -62,3 +62,11 @@ extern "C" ra_status rope_attn_fwd_noalloc(const ra_problem* p, const void* q, c
   // never leak into this call.
   return rope_attn_fwd(p, q, k, v, alpha, o, lse, scratch, kNoallocScratchBytes, stream);
 }
+
+// The error word at the start of the static array: the same read-and-clear as
+// rope_attn_device_status on a workspace (synchronises the stream first).
+extern "C" ra_status rope_attn_noalloc_status(void* stream, int32_t info[3]) {
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return RA_ERR_CUDA;
+  return rope_attn_device_status(scratch, kNoallocScratchBytes, stream, info);
+}

@@ -27,17 +27,32 @@
 namespace ra {
 
 // One handle per host thread and device: every call sets the handle's stream, so two
-// threads must not share one (a handle is not safe for concurrent use).  Handles live until
-// the process exits.
+// threads must not share one (a handle is not safe for concurrent use).  The holder is
+// thread_local, so a thread's handles (and the device workspace cuBLAS keeps with each) are
+// destroyed when that thread exits, each with its own device current.
+struct HandleSet {
+  std::unordered_map<int, cublasHandle_t> by_dev;
+  ~HandleSet() {
+    // At process exit the runtime may already be unloading (cudaGetDevice fails then): the
+    // process's memory goes with it, so the handles are left alone.
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return;
+    for (auto& kv : by_dev) {
+      if (cudaSetDevice(kv.first) == cudaSuccess) cublasDestroy(kv.second);
+    }
+    cudaSetDevice(cur);
+  }
+};
+
 cublasHandle_t cublas_handle() {
-  thread_local std::unordered_map<int, cublasHandle_t> handles;
+  thread_local HandleSet handles;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  auto it = handles.find(dev);
-  if (it != handles.end()) return it->second;
+  auto it = handles.by_dev.find(dev);
+  if (it != handles.by_dev.end()) return it->second;
   cublasHandle_t h = nullptr;
   if (cublasCreate(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
-  handles[dev] = h;
+  handles.by_dev[dev] = h;
   return h;
 }
 

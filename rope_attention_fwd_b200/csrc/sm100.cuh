@@ -325,6 +325,30 @@ __device__ __forceinline__ void mma8_ts_mn(uint32_t d_tmem, uint32_t a0, uint64_
       : "memory");
 }
 
+// mma8_ss_mn: 8 K-steps of 16 with both operands MN-major in shared memory (each +2048 B =
+// 16 rows of 128 B per step).
+__device__ __forceinline__ void mma8_ss_mn(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+      "add.u64 a1, %1, 128;\n\tadd.u64 a2, %1, 256;\n\tadd.u64 a3, %1, 384;\n\t"
+      "add.u64 a4, %1, 512;\n\tadd.u64 a5, %1, 640;\n\tadd.u64 a6, %1, 768;\n\tadd.u64 a7, %1, 896;\n\t"
+      "add.u64 b1, %2, 128;\n\tadd.u64 b2, %2, 256;\n\tadd.u64 b3, %2, 384;\n\t"
+      "add.u64 b4, %2, 512;\n\tadd.u64 b5, %2, 640;\n\tadd.u64 b6, %2, 768;\n\tadd.u64 b7, %2, 896;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a4, b4, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a5, b5, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a6, b6, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a7, b7, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -495,6 +519,11 @@ __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_
                : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
                : "r"(addr)
                : "memory");
+}
+
+// *addr += v in global memory (a reduction: no value comes back, relaxed, gpu scope).
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
 // Byte offset of 16-byte unit u (0..7) of row r inside a 128B-swizzled chunk.

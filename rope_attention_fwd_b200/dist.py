@@ -7,7 +7,8 @@ disjoint (batch, head) units -- their own batches (weak scaling, what bench.py t
 contiguous shards of one batch's B*H units (`shard_bh`) -- and after each backward the
 d/2 floats of dalpha are combined by `allreduce_dalpha`: an all-gather of every rank's
 partial and a sum in rank order in fp64, so that every rank holds the same bits whatever
-the collective's internal reduction order (NCCL on GPUs, gloo in the CPU tests).
+the collective's internal reduction order (NCCL on GPUs, gloo in the CPU tests).  The loss
+L, a sum over every head as well, is combined the same way.
 """
 import torch
 import torch.distributed as dist
@@ -32,18 +33,24 @@ def shard_bh(B: int, H: int, world: int, rank: int):
     return start, base + (1 if rank < extra else 0)
 
 
-def allreduce_dalpha(dalpha, group=None):
-    """dalpha <- the sum of every rank's dalpha (shape [d/2]), deterministic: all-gather,
-    then a fixed rank-order fp64 sum on every rank.  A no-op on one process."""
+def allreduce_sum(x, group=None):
+    """x <- the sum of every rank's x (any shape, e.g. dalpha [d/2] or the scalar loss L),
+    deterministic: all-gather, then a fixed rank-order fp64 sum on every rank.  A no-op on
+    one process."""
     if not (dist.is_available() and dist.is_initialized()):
-        return dalpha
+        return x
     world = dist.get_world_size(group)
     if world == 1:
-        return dalpha
-    parts = [torch.empty_like(dalpha) for _ in range(world)]
-    dist.all_gather(parts, dalpha.contiguous(), group=group)
-    acc = torch.zeros(dalpha.shape, dtype=torch.float64, device=dalpha.device)
+        return x
+    parts = [torch.empty_like(x) for _ in range(world)]
+    dist.all_gather(parts, x.contiguous(), group=group)
+    acc = torch.zeros(x.shape, dtype=torch.float64, device=x.device)
     for p in parts:  # rank order
         acc += p.to(torch.float64)
-    dalpha.copy_(acc.to(dalpha.dtype))
-    return dalpha
+    x.copy_(acc.to(x.dtype))
+    return x
+
+
+def allreduce_dalpha(dalpha, group=None):
+    """dalpha <- the sum over every rank (see allreduce_sum)."""
+    return allreduce_sum(dalpha, group)

@@ -72,14 +72,25 @@ def gpu_fwd(inp, device="cuda"):
     return dict(o=to64(o), lse=to64(lse))
 
 
-def oracle_run(inp, fixed_bands=0):
-    """Oracle results, plus `dalpha_noise`: the bf16 rounding-noise scale of dalpha.
+def _bf16(x):
+    """Round float64 values to bf16 and back (the storage rounding of a bf16 tensor)."""
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
 
-    Each weighted torque term w_p <dX~_pm, J x~_pm> of the dalpha sum is perturbed by
-    O(u) relative (u = 2^-8, bf16 unit roundoff) when x~ is rounded to bf16 for the
-    tensor cores; the perturbations have random signs, so they add in quadrature.
-    dalpha_noise = 3 u ||theta_hat * sqrt(sum of squared weighted torques)|| / ||dalpha||.
-    (A CPU model of the kernel's roundings puts the actual error at 0.14-1.7 u RSS.)
+
+def oracle_run(inp, fixed_bands=0):
+    """Oracle results, plus `dalpha_noise` for bf16 problems: the relative dalpha error that
+    storage and operand rounding alone produce, derived from the oracle.
+
+    The dalpha sum is a small difference of large Q-side and K-side torque sums (they cancel
+    30-250x on small problems), so roundings that are harmless for dQ, dK, dV show in it.
+    Two are fixed by the path itself, not by kernel error:
+      * O and dO are bf16 tensors at the boundary (rope_attn_loss writes dO = O - E in the
+        problem dtype).  Their effect is measured exactly: the oracle's backward is run a
+        second time with dO_b = bf16(bf16(O) - E), and rel(dalpha_b, dalpha) is taken.
+      * the score operands q~, k~ and dS are fp16 (unit roundoff u = 2^-11).  Each weighted
+        torque term w_p <dX~_pm, J x~_pm> moves by O(u) relative with random sign, so these
+        add in quadrature: 3 u ||theta_hat * sqrt(sum of squared weighted torques)||.
+    dalpha_noise = 2 rel(dalpha_b, dalpha) + 3 u ||theta_hat * RSS|| / ||dalpha||.
     """
     wl = inp.wl
     q, k, v, e, al = (inp.f64(x) for x in ("q", "k", "v", "e", "alpha"))
@@ -87,15 +98,21 @@ def oracle_run(inp, fixed_bands=0):
     L, do = ref.loss(o, e)
     dq, dk, dv, dalpha, extra = ref.backward(q, k, v, do, al, wl.base, wl.causal,
                                              return_rotated=True, fixed_bands=fixed_bands)
-    _, th = ref.frequencies(wl.d, wl.base, al, fixed_bands)
-    w2 = (np.arange(wl.n) - 0.5 * (wl.n - 1)) ** 2
-    rss = np.zeros(wl.d // 2)
-    for qt, kt, dqt, dkt in extra:
-        rss += w2 @ (ref.band_torque(dqt, qt) ** 2 + ref.band_torque(dkt, kt) ** 2)
+    out = dict(o=o, lse=lse, L=L, do=do, dq=dq, dk=dk, dv=dv, dalpha=dalpha)
     nrm = np.linalg.norm(dalpha)
-    noise = 3 * 2.0 ** -8 * np.linalg.norm(th * np.sqrt(rss)) / nrm if nrm > 0 else 0.0
-    return dict(o=o, lse=lse, L=L, do=do, dq=dq, dk=dk, dv=dv, dalpha=dalpha,
-                dalpha_noise=float(noise))
+    if wl.dtype == "bf16" and nrm > 0:
+        _, th = ref.frequencies(wl.d, wl.base, al, fixed_bands)
+        w2 = (np.arange(wl.n) - 0.5 * (wl.n - 1)) ** 2
+        rss = np.zeros(wl.d // 2)
+        for qt, kt, dqt, dkt in extra:
+            rss += w2 @ (ref.band_torque(dqt, qt) ** 2 + ref.band_torque(dkt, kt) ** 2)
+        do_b = _bf16(_bf16(o) - e)
+        dalpha_b = ref.backward(q, k, v, do_b, al, wl.base, wl.causal,
+                                fixed_bands=fixed_bands)[3]
+        storage = np.linalg.norm(dalpha_b - dalpha) / nrm
+        operand = 3 * 2.0 ** -11 * np.linalg.norm(th * np.sqrt(rss)) / nrm
+        out["dalpha_noise"] = float(2 * storage + operand)
+    return out
 
 
 def oracle_fwd(inp):
@@ -105,30 +122,35 @@ def oracle_fwd(inp):
     return dict(o=o, lse=lse)
 
 
-def compare(g, r, dtype, keys=("o", "lse", "L", "dq", "dk", "dv", "dalpha"), small=False):
-    """Assert every result is inside its tolerance; return the measured errors.
+def compare(g, r, dtype, keys=("o", "lse", "L", "dq", "dk", "dv", "dalpha"), small=False,
+            label=""):
+    """Assert every result is inside its tolerance; print and return the measured errors
+    with their bounds.
 
     small=True (problems far below the workload sizes, bf16 only): dalpha may also sit
-    inside the oracle's bf16 rounding-noise scale r["dalpha_noise"] (see oracle_run),
-    since with few positions the cancelling Q/K torque sums leave less signal."""
+    inside the rounding-noise scale r["dalpha_noise"] that oracle_run derives, since with
+    few positions the cancelling Q/K torque sums leave less signal.  On the workloads
+    themselves the target's 1e-2 applies as it stands."""
     tol = dict(TOL[dtype])
     if small and dtype == "bf16" and "dalpha_noise" in r:
         tol["dalpha"] = max(tol["grad"], r["dalpha_noise"])
-    errs = {}
+    errs, bounds = {}, {}
     for key in keys:
         if key == "o":
             errs[key] = float(np.max(np.abs(g["o"] - r["o"]))) if g["o"].size else 0.0
-            assert errs[key] <= tol["o"], (key, errs[key])
+            bounds[key] = tol["o"]
         elif key == "lse":
             errs[key] = float(np.max(np.abs(g["lse"] - r["lse"]))) if g["lse"].size else 0.0
-            assert errs[key] <= tol["lse"], (key, errs[key])
+            bounds[key] = tol["lse"]
         elif key == "L":
             errs[key] = abs(g["L"] - r["L"]) / max(abs(r["L"]), 1e-30)
-            assert errs[key] <= tol["L"], (key, errs[key])
+            bounds[key] = tol["L"]
         else:
             errs[key] = rel_frob(g[key], r[key])
-            bound = tol.get(key, tol["grad"])
-            assert errs[key] <= bound, (key, errs[key], bound)
+            bounds[key] = tol.get(key, tol["grad"])
+    print("parity", label, " ".join(f"{k}={errs[k]:.3e}/{bounds[k]:.1e}" for k in keys))
+    for key in keys:
+        assert errs[key] <= bounds[key], (label, key, errs[key], bounds[key])
     return errs
 
 

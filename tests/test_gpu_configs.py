@@ -1,21 +1,24 @@
 """GPU parity on the five workloads at full size, in the launch configuration the bench
-times (the same kernels and tiles; the whole [B, H, n, d] problem in one call).
+times (rope_attn_fwd, rope_attn_loss, rope_attn_bwd_saved on the whole [B, H, n, d]
+problem in one call each), against the float64 oracle on every element.
 
 * 1x1x256x64 fp32 and 4x16x2048x64 bf16: every output against the full oracle.
-* 2x32x8192x128, 1x8x32768x128, 8x16x4096x128 (bf16): the oracle is too slow for
-  every head, so it checks sampled heads -- O and lse on every row, dQ, dK, dV on
-  sampled rows, and the
-  head's own dalpha (the GPU's per-head dalpha comes from the same kernels run on that
-  head alone) -- plus properties that hold at any size: dalpha of the whole problem is
-  the sum of the per-head dalphas, dO is exactly the bf16 rounding of O - E, and L is
-  1/2 sum (O - E)^2 of the GPU's own O.
+* 2x32x8192x128, 1x8x32768x128, 8x16x4096x128 (bf16): every head is recomputed by the
+  oracle in a spawn process pool (one head per core, see oracle_heads.py).  O and lse are
+  compared on every element; dQ, dK, dV by the relative Frobenius error of the whole
+  tensor; dalpha of the whole problem (summed over every head, "LeRoPE", Escolhas de
+  Design Principais: alpha is shared by all heads) against the oracle's whole-problem
+  dalpha.  All at the target's bounds: 2e-2 max-abs on O, 1e-2 relative Frobenius on
+  dQ, dK, dV, dalpha.  Plus two exact properties of the loss: dO is the bf16 rounding of
+  O - E, and L is 1/2 sum (O - E)^2 of the GPU's own O.
 """
 import numpy as np
 import pytest
 import torch
 
-from helpers import TOL, check_status, compare, gpu_run, oracle_run, rel_frob, to64
+from helpers import TOL, check_status, compare, gpu_run, oracle_run, to64
 from oracle import rope_attn_ref as ref
+from oracle_heads import run_heads
 from rope_attention_fwd_b200 import binding as rb
 from rope_attention_fwd_b200.configs import WORKLOADS
 from rope_attention_fwd_b200.inputs import make_inputs
@@ -26,98 +29,70 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("cfg", [1, 2])
 def test_config_full_oracle(cfg):
     inp = make_inputs(WORKLOADS[cfg])
-    compare(gpu_run(inp), oracle_run(inp), WORKLOADS[cfg].dtype)
+    errs = compare(gpu_run(inp), oracle_run(inp), WORKLOADS[cfg].dtype, label=f"config {cfg}")
+    print(f"config {cfg}", errs)
 
 
-def _head64(t, b, h):
-    return t[b, h].to(torch.float64).numpy()
-
-
-def _sample_rows(n, rng, count=96):
-    fixed = [0, 1, 2, 63, 64, 127, 128, 129, n // 2, n - 2, n - 1]
-    return np.unique(np.concatenate([np.array([r for r in fixed if r < n]),
-                                     rng.choice(n, size=min(count, n), replace=False)]))
-
-
-def _gpu_full(inp, dev="cuda"):
+def _gpu_step(inp, dev="cuda"):
+    """One bench step through the C ABI: forward, loss, backward from the saved operands."""
     wl = inp.wl
     q, k, v, e, alpha = (getattr(inp, x).to(dev) for x in ("q", "k", "v", "e", "alpha"))
     ws = rb.workspace(rb.problem(wl.B, wl.H, wl.n, wl.d, q.dtype, wl.causal, wl.base), dev)
     o, lse = rb.rope_attn_fwd(q, k, v, alpha, wl.base, wl.causal, ws=ws)
-    check_status(ws)
     L, dO = rb.rope_attn_loss(o, e, ws=ws)
+    dq, dk, dv, dalpha = rb.rope_attn_bwd_saved(v, o, lse, dO, alpha, wl.base, wl.causal, ws)
     check_status(ws)
-    dq, dk, dv, dalpha = rb.rope_attn_bwd(q, k, v, o, lse, dO, alpha, wl.base, wl.causal, ws=ws)
-    check_status(ws)
-    return dict(q=q, k=k, v=v, e=e, alpha=alpha, o=o, lse=lse, L=L, dO=dO, dq=dq, dk=dk, dv=dv,
-                dalpha=dalpha)
+    cpu = lambda t: t.cpu()
+    return dict(o=cpu(o), lse=cpu(lse), L=float(L.item()), dO=cpu(dO), dq=cpu(dq), dk=cpu(dk),
+                dv=cpu(dv), dalpha=cpu(dalpha))
 
 
-def _gpu_head_dalpha(g, b, h, wl):
-    """dalpha of head (b, h) alone, from the same kernels on that head's slices."""
-    sl = lambda t: t[b:b + 1, h:h + 1].contiguous()
-    _, _, _, da = rb.rope_attn_bwd(sl(g["q"]), sl(g["k"]), sl(g["v"]), sl(g["o"]), sl(g["lse"]),
-                                   sl(g["dO"]), g["alpha"], wl.base, wl.causal)
-    return da
+def _bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
+@pytest.mark.slow
 @pytest.mark.parametrize("cfg", [3, 4, 5])
-def test_config_sampled(cfg):
+def test_config_every_head(cfg):
     wl = WORKLOADS[cfg]
     inp = make_inputs(wl)
-    g = _gpu_full(inp)
-    torch.cuda.synchronize()
+    g = _gpu_step(inp)
     tol = TOL["bf16"]
 
-    # properties at full size: dO = bf16(O - E) exactly; L = 1/2 sum (O - E)^2 of the GPU's O
-    o_cpu, e_cpu = g["o"].cpu(), inp.e
-    diff = o_cpu.float() - e_cpu.float()
-    assert torch.equal(g["dO"].cpu(), diff.to(torch.bfloat16))
+    # exact properties of the loss: dO = bf16(O - E); L = 1/2 sum (O - E)^2 of the GPU's O
+    diff = g["o"].float() - inp.e.float()
+    assert torch.equal(g["dO"], diff.to(torch.bfloat16))
     L_host = 0.5 * float((diff.double() ** 2).sum())
-    assert abs(g["L"].item() - L_host) <= 1e-6 * L_host
+    assert abs(g["L"] - L_host) <= 1e-6 * L_host
 
-    # dalpha of the whole problem = sum of per-head dalphas (cross-head reduction)
-    BH = wl.B * wl.H
-    per_head = {}
-    acc = torch.zeros(wl.d // 2, dtype=torch.float64, device="cuda")
+    tasks = []
+    alpha = inp.alpha.double().numpy()
     for b in range(wl.B):
         for h in range(wl.H):
-            per_head[(b, h)] = _gpu_head_dalpha(g, b, h, wl)
-            acc += per_head[(b, h)].double()
-    assert rel_frob(to64(g["dalpha"]), to64(acc)) <= 1e-5
+            t = dict(head=(b, h), n=wl.n, d=wl.d, causal=wl.causal, base=wl.base, alpha=alpha)
+            for x in ("q", "k", "v", "e"):
+                t[x] = _bits(getattr(inp, x)[b, h])
+            for x in ("o", "dq", "dk", "dv"):
+                t["g_" + x] = _bits(g[x][b, h])
+            t["g_lse"] = g["lse"][b, h].numpy()
+            tasks.append(t)
+    res = run_heads(tasks)
 
-    # sampled heads against the oracle
-    rng = np.random.default_rng(100 + cfg)
-    heads = [(0, 0), (wl.B - 1, wl.H - 1)] if cfg != 4 else [(0, wl.H // 2)]
-    al = inp.f64("alpha")
-    _, th = ref.frequencies(wl.d, wl.base, al)
-    phi = ref.angles(wl.n, th)
-    for (b, h) in heads:
-        q, k, v, e = (_head64(t, b, h) for t in (inp.q, inp.k, inp.v, inp.e))
-        qt, kt = ref.rotate(q, phi), ref.rotate(k, phi)
-        o, lse = ref.head_forward(qt, kt, v, wl.causal)
-        do = o - e
-        delta = np.sum(do * o, axis=1)
-        rows = _sample_rows(wl.n, rng)
-        # O and lse of every row of the head (the oracle computes them all anyway): rare
-        # elements carry the largest error, so sampled rows alone can miss them
-        go = g["o"][b, h].double().cpu().numpy()
-        assert np.max(np.abs(go - o)) <= tol["o"]
-        assert np.max(np.abs(g["lse"][b, h].double().cpu().numpy() - lse)) <= tol["lse"]
-        dqt = ref.head_backward_rows(qt, kt, v, do[rows], lse[rows], delta[rows], rows,
-                                     wl.causal)
-        dq = ref.rotate(dqt, phi[rows], sign=-1.0)
-        assert rel_frob(g["dq"][b, h].double().cpu().numpy()[rows], dq) <= tol["grad"]
-        dkt, dv = ref.head_backward_cols(qt, kt, v, do, lse, delta, rows, wl.causal)
-        dk = ref.rotate(dkt, phi[rows], sign=-1.0)
-        assert rel_frob(g["dk"][b, h].double().cpu().numpy()[rows], dk) <= tol["grad"]
-        assert rel_frob(g["dv"][b, h].double().cpu().numpy()[rows], dv) <= tol["grad"]
-        # the head's own dalpha: full backward of this one head
-        dqt_all, dkt_all, _ = ref.head_backward(qt, kt, v, do, wl.causal)
-        w = np.arange(wl.n, dtype=np.float64)
-        tq, tk = ref.band_torque(dqt_all, qt), ref.band_torque(dkt_all, kt)
-        da_h = th * (w @ (tq + tk))
-        wc2 = (w - 0.5 * (wl.n - 1)) ** 2
-        noise = 3 * 2.0 ** -8 * np.linalg.norm(th * np.sqrt(wc2 @ (tq ** 2 + tk ** 2)))
-        bound = max(tol["grad"], noise / np.linalg.norm(da_h))
-        assert rel_frob(to64(per_head[(b, h)]), da_h) <= bound
+    errs = {"o": max(r["o_maxabs"] for r in res), "lse": max(r["lse_maxabs"] for r in res)}
+    for name in ("dq", "dk", "dv"):
+        errs[name] = float(np.sqrt(sum(r[name + "_err2"] for r in res) /
+                                   sum(r[name + "_norm2"] for r in res)))
+        errs[name + "_worst_head"] = float(max(np.sqrt(r[name + "_err2"] / r[name + "_norm2"])
+                                               for r in res))
+    _, th = ref.frequencies(wl.d, wl.base, alpha)
+    torque = np.zeros(wl.d // 2)
+    for r in res:  # fixed head order
+        torque += r["torque"]
+    da_ref = th * torque
+    da = g["dalpha"].double().numpy()
+    errs["dalpha"] = float(np.linalg.norm(da - da_ref) / np.linalg.norm(da_ref))
+    print(f"config {cfg} every head:", errs)
+    assert errs["o"] <= tol["o"], errs
+    assert errs["lse"] <= tol["lse"], errs
+    for name in ("dq", "dk", "dv", "dalpha"):
+        assert errs[name] <= tol["grad"], (name, errs)

@@ -32,3 +32,19 @@ def test_forward_wait_expires_and_reports():
     # the status was read and cleared; the context still works and gives correct results
     assert rb.rope_attn_device_status(ws)[0] == 0
     compare(gpu_fwd(inp), oracle_fwd(inp), "bf16", keys=("o", "lse"))
+
+
+def test_range_overflow_is_reported():
+    """A key entry beyond the fp16 range of the score operands is clamped by the rotation
+    and reported as RA_ERR_RANGE through the workspace error word (nothing faults); the
+    following clean call on the same workspace reports nothing."""
+    wl = small_workload(1, 1, 64, 64, "bf16", False, seed=3)
+    inp = make(wl)
+    q, k, v, alpha = (getattr(inp, x).cuda() for x in ("q", "k", "v", "alpha"))
+    ws = rb.workspace(rb.problem(1, 1, 64, 64, torch.bfloat16, False, wl.base), "cuda")
+    big = k.clone()
+    big[0, 0, 0, 1] = -7.0e4  # position 0: the rotation keeps it, |7e4| > 65504
+    rb.rope_attn_fwd(q, big, v, alpha, wl.base, False, ws=ws)
+    assert rb.STATUS[rb.rope_attn_device_status(ws)[0]] == "RA_ERR_RANGE"
+    rb.rope_attn_fwd(q, k, v, alpha, wl.base, False, ws=ws)
+    assert rb.rope_attn_device_status(ws)[0] == 0

@@ -113,12 +113,6 @@ bool fwd_split_s() {
   return s && std::atoi(s) == 1;
 }
 
-// RA_BWD_DKDV_TMEM=1 selects the dK/dV kernel with K~ and V as TMEM operands, read per call.
-bool dkdv_tmem() {
-  const char* s = std::getenv("RA_BWD_DKDV_TMEM");
-  return s && std::atoi(s) == 1;
-}
-
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -302,20 +296,15 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
                 launch_bwd_fused_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dqacc,
                                        dpart, ctl, s));
       RA_LAUNCH(K_DQ_FINISH, s, launch_dq_finish(*p, dqacc, table, stats, dq, s));
-    } else if (dkdv_tmem()) {
-      if (!make_map(&maps.qt32, qt, *p, 32, true) || !make_map(&maps.dO32, dO, *p, 32))
-        return RA_ERR_CUDA;
-      RA_LAUNCH(K_BWD_DKDV_SM100, s,
-                launch_bwd_dkdv_tmem_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart,
-                                           ctl, s));
     } else {
+      // two passes: dK, dV (keys stationary), then dQ (queries stationary, S and dP
+      // recomputed); every output bitwise reproducible
       RA_LAUNCH(K_BWD_DKDV_SM100, s,
                 launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
                                       s));
-    }
-    if (!uses_fused_bwd(*p))
       RA_LAUNCH(K_BWD_DQ_SM100, s,
                 launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
+    }
   }
   if (dalpha) RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;

@@ -27,17 +27,22 @@
 // a CPU model of the roundings (bf16 operands) puts the dalpha error at 1.0e-2 that way,
 // 3.8e-3 this way.
 //
-// Two kernels, no atomics (deterministic):
-//   dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
-//         time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
-//         (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T (fp16),
-//         then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
-//         accumulated in TMEM for the whole pass.
-//   dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
-//         dP = dO V_j^T (double-buffered in TMEM), dS in fp16, dQ~ += dS K~_j.
+// Two forms:
+//   fused (bf16, d = 128; the default): one kernel, 128 keys stationary per CTA, queries
+//         streamed 64 at a time; per step S^T, dP^T, then dV += P^T dO_i, dK~ += dS^T Q~_i
+//         (TMEM accumulators) and dQ~^T = K~^T dS^T, whose partial is added into an fp32
+//         accumulator in global memory; dq_finish_kernel rotates the sum back.
+//   two-pass (d = 64, or RA_FLAG_DETERMINISTIC): no atomics, every output reproducible
+//     dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
+//           time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
+//           (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T
+//           (fp16), then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
+//           accumulated in TMEM for the whole pass.
+//     dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
+//           dP = dO V_j^T (double-buffered in TMEM), dS in fp16, dQ~ += dS K~_j.
 // Warp roles: two softmax warpgroups (warps 0-7) each own every row (TMEM lane) and half
 // of the 64 streamed columns; warp 8 issues TMA copies; warp 9 allocates TMEM and issues
-// tcgen05.mma.  Every wait is bounded.
+// tcgen05.mma; in the fused kernel warps 10-13 drain dQ~.  Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -51,58 +56,16 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-#ifndef RA_DKDV_STAGES
-#define RA_DKDV_STAGES 4
-#endif
-#ifndef RA_BWD_PACK_ALU
-#define RA_BWD_PACK_ALU 0
-#endif
-#ifndef RA_BWD_POLY_EVERY
-#define RA_BWD_POLY_EVERY 0
-#endif
-// exp2 of streamed column c: every RA_BWD_POLY_EVERY-th column on the FMA pipe (exp2_poly),
-// the others on MUFU, to split the load of the XU pipe.
-__device__ __forceinline__ float exp2_col(float x, int c) {
-#if RA_BWD_POLY_EVERY > 0
-  if (c % RA_BWD_POLY_EVERY == RA_BWD_POLY_EVERY - 1) return exp2_poly(x);
-#endif
-  return fast_exp2(x);
-}
-
-#ifndef RA_MMA_BATCH
-#define RA_MMA_BATCH 1
-#endif
-#ifndef RA_BWD_SOFT_WG
-#define RA_BWD_SOFT_WG 2
-#endif
-#ifndef RA_BWD_SPLIT
-#define RA_BWD_SPLIT 1
-#endif
-// Softmax warpgroups per CTA, and how they share the streamed 64-column tiles:
-//  * ping-pong (RA_BWD_SPLIT 0): warpgroup g takes the tiles it = g, g + kSoftWG, ...
-//    (TMEM buffer it & 1), every row (TMEM lane) and all 64 columns, so one warpgroup's
-//    TMEM round trips and barrier hand-offs overlap the other's arithmetic;
-//  * column split (RA_BWD_SPLIT 1, two warpgroups): both take every tile, warpgroup g
-//    its columns 32g .. 32g + 31, which halves the latency from S / dP to dS.
-// The epilogue splits the D output columns between the warpgroups.
-constexpr int kSoftWG = RA_BWD_SOFT_WG;
-constexpr bool kSplit = RA_BWD_SPLIT != 0;
-static_assert(!kSplit || kSoftWG == 2, "the column split takes two warpgroups");
+// Two softmax warpgroups per CTA.  Both take every streamed 64-column tile, warpgroup g its
+// columns 32g .. 32g + 31 (a column split: the S -> dS latency of a tile is half of what one
+// warpgroup over all 64 columns takes); thread t owns row t (TMEM lane t) of the tile.  The
+// epilogue splits the D output columns between the warpgroups.
+constexpr int kSoftWG = 2;
 constexpr int kSoftThreads = 128 * kSoftWG;
 constexpr int kThreads = kSoftThreads + 64;  // + TMA producer warp + MMA warp
-constexpr int kCols = kSplit ? 32 : 64;       // streamed columns per softmax thread and tile
-constexpr int kTileStep = kSplit ? 1 : kSoftWG;   // tiles between one warpgroup's tiles
-constexpr int kHalves = kSplit ? 1 : 2;           // 32-column halves per thread and tile
-constexpr int kDsArrivals = kSplit ? kSoftThreads : 128;
+constexpr int kCols = 32;                     // streamed columns per softmax thread and tile
+constexpr int kDsArrivals = kSoftThreads;
 constexpr int kProdWarp = 4 * kSoftWG, kMmaWarp = 4 * kSoftWG + 1;
-
-__device__ __forceinline__ uint32_t pack_g(float lo, float hi) {
-#if RA_BWD_PACK_ALU
-  return pack_bf16x2_alu(lo, hi);
-#else
-  return pack_bf16x2(lo, hi);
-#endif
-}
 
 __device__ __forceinline__ void softmax_group_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
@@ -246,9 +209,11 @@ __device__ __forceinline__ void write_dalpha_partials(const float* red, float* d
 }
 
 // ======================================================================== dK, dV
+constexpr int kDkdvStages = 4;  // Q~ / dO ring depth
+
 template <int D>
 struct DkdvCfg {
-  static constexpr int BN = 128, BQ = 64, NS = RA_DKDV_STAGES, CH = D / 64;
+  static constexpr int BN = 128, BQ = 64, NS = kDkdvStages, CH = D / 64;
   static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
   static constexpr uint32_t KTILE = KCH * CH;
   static constexpr uint32_t QCH = 64u * 128u;   // chunk of a 64-row tile
@@ -270,8 +235,8 @@ struct DkdvCfg {
 enum DkdvBar {
   KB_KV_FULL = 0,
   KB_Q_FULL = 1,                        // +stage
-  KB_Q_EMPTY = 1 + RA_DKDV_STAGES,      // +stage
-  KB_SDP_FULL = 1 + 2 * RA_DKDV_STAGES, // +buffer: S^T and dP^T of that buffer computed
+  KB_Q_EMPTY = 1 + kDkdvStages,         // +stage
+  KB_SDP_FULL = 1 + 2 * kDkdvStages,    // +buffer: S^T and dP^T of that buffer computed
   KB_DS_FULL = KB_SDP_FULL + 2,         // +buffer: P^T, dS^T written (kDsArrivals arrivals)
   KB_ACC_DONE = KB_DS_FULL + 2,
   KB_DRAIN,
@@ -388,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         tc_fence_after();
         const SDesc qs = sdesc_advance(dkm, C::OFF_ST + s * C::STAGE);
-        if constexpr (D == 128 && RA_MMA_BATCH) {
+        if constexpr (D == 128) {
           mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K),
                                              sdesc_at(qs, 0), idST, 0);
           mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_DPT,
@@ -422,21 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const SDesc qm = sdesc_advance(dmn, C::OFF_ST + s * C::STAGE);
         // dV += P^T dO_i and dK~ += dS^T Q~_i with P^T, dS^T read from TMEM
-        if constexpr (RA_MMA_BATCH) {
-          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
-              tmem + C::COL_DV, tmem + b * 128 + C::COL_ST, sdesc_at(qm, C::QTILE), idDV, it > 0);
-          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
-              tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT, sdesc_at(qm, 0), idDK, it > 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk)
-            mma_ts_warp(tmem + C::COL_DV, tmem + b * 128 + C::COL_ST + packed_col(16 * kk),
-                        sdesc_at(qm, C::QTILE + kk * 2048), idDV, (it > 0 || kk > 0));
-#pragma unroll
-          for (int kk = 0; kk < C::BQ / 16; ++kk)
-            mma_ts_warp(tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT + packed_col(16 * kk),
-                        sdesc_at(qm, kk * 2048), idDK, (it > 0 || kk > 0));
-        }
+        mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+            tmem + C::COL_DV, tmem + b * 128 + C::COL_ST, sdesc_at(qm, C::QTILE), idDV, it > 0);
+        mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+            tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT, sdesc_at(qm, 0), idDK, it > 0);
         mma_commit_warp(&bar[KB_Q_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[KB_ACC_DONE]);
@@ -447,13 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax warpgroups
     const int t = threadIdx.x % 128;      // key row == TMEM lane
-    const int half = threadIdx.x / 128;   // warpgroup: takes query tiles it = half (mod kSoftWG)
+    const int half = threadIdx.x / 128;   // warpgroup: query columns 32 half .. 32 half + 31
     const int key = jt * C::BN + t;
     const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
     const float dss = ds_scale(stats);
     bool ok = true;
-    for (int it = kSplit ? 0 : half; it < nq; it += kTileStep) {
+    for (int it = 0; it < nq; ++it) {
       const int s = it % C::NS, b = it & 1;
       const int i0 = qstart + it * C::BQ;
       if (!mbar_wait_warp(&bar[KB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6, wait_ns) ||
@@ -468,11 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                          2 * C::QTILE);
       const float4* dvv = lv + C::BQ / 4;
       const bool need_mask = causal && (i0 < jt * C::BN + C::BN);
-      // 32 columns at a time: load S^T, dP^T; P^T, dS^T back as bf16 over the first 16
-      // columns of each half (packed_col order), all before this warpgroup's arrival
-#pragma unroll
-      for (int hh = 0; hh < kHalves; ++hh) {
-        const int h = kSplit ? half : hh;
+      // this warpgroup's 32 columns: load S^T, dP^T; P^T, dS^T back as 16-bit pairs over
+      // the first 16 columns of its half (packed_col order), before its arrival
+      {
+        const int h = half;
         uint32_t sr[32], dr[32];
         tmem_ld32(st_base + 32 * h, sr);
         tmem_ld32(dpt_base + 32 * h, dr);
@@ -487,13 +440,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * c4 + e;  // column within this half
-            float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - la[e], 32 * h + c);
+            float p = fast_exp2(__uint_as_float(sr[c]) * scale_log2 - la[e]);
             if (need_mask && (i0 + 32 * h + c < key)) p = 0.f;
             pv[e] = p;
             dsv[e] = p * (__uint_as_float(dr[c]) - da[e]) * dss;
           }
-          pw[2 * c4] = pack_g(pv[0], pv[1]);
-          pw[2 * c4 + 1] = pack_g(pv[2], pv[3]);
+          pw[2 * c4] = pack_bf16x2(pv[0], pv[1]);
+          pw[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
           dw[2 * c4] = pack_f16x2_sat(dsv[0], dsv[1]);
           dw[2 * c4 + 1] = pack_f16x2_sat(dsv[2], dsv[3]);
         }
@@ -552,16 +505,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ======================================================================== dQ
-#ifndef RA_DQ_STAGES
-#define RA_DQ_STAGES 4
-#endif
-#ifndef RA_DQ_BUFS
-#define RA_DQ_BUFS 2
-#endif
+constexpr int kDqStages = 4;  // K~ / V ring depth
 
 template <int D>
 struct DqCfg {
-  static constexpr int BM = 128, BK = 64, NS = RA_DQ_STAGES, CH = D / 64;
+  static constexpr int BM = 128, BK = 64, NS = kDqStages, CH = D / 64;
   static constexpr uint32_t QCH = 128u * 128u;  // chunk of a 128-row tile
   static constexpr uint32_t QTILE = QCH * CH;
   static constexpr uint32_t KCH = 64u * 128u;   // chunk of a 64-row tile
@@ -570,19 +518,15 @@ struct DqCfg {
   static constexpr uint32_t STAGE = 2 * KTILE;  // K~_j, V_j
   static constexpr uint32_t OFF_BAR = OFF_ST + NS * STAGE;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  // TMEM: NB buffers of [S (64 fp32) | dP (64 fp32)] at 128 * b, dS written back as fp16
-  // over the start of each thread's S slice, then the dQ~ accumulator.
-  //  * NB = 3: the issuer runs two key tiles ahead of the softmax, so the S -> dS latency
-  //    of a tile hides behind two tiles of MMAs; Q~ and dO stay in shared memory.
-  //  * NB = 2: only one tile ahead, but the stationary Q~ (fp16) and dO (bf16) tiles sit in
-  //    TMEM (two per column) as the A operands of the S and dP MMAs, which then read only
-  //    their 2 KB B tile from shared memory and run at the tensor rate (from shared memory,
-  //    4 KB more per K-step, an M=128, N=64 MMA is bandwidth-bound).
-  static constexpr int NB = RA_DQ_BUFS;
-  static_assert(NB == 2 || NB == 3, "two or three S/dP buffers");
-  static_assert(NS >= NB, "the K~/V ring holds every key tile whose S, dP are in flight");
+  // TMEM: two buffers of [S (64 fp32) | dP (64 fp32)] at 128 * b, dS written back as fp16
+  // over the start of each thread's S slice; the dQ~ accumulator at 256; the stationary Q~
+  // (fp16) and dO (bf16) rows (two per column) at 256 + D and 256 + 3D/2 as the A operands of
+  // the S and dP MMAs, which then read only their 2 KB B tile from shared memory per K-step
+  // and run at the tensor rate (from shared memory, 4 KB more per K-step, an M = 128, N = 64
+  // MMA is bound by the shared-memory read rate).
+  static constexpr int NB = 2;
   static constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 128 * NB;
-  static constexpr uint32_t COL_QT = 256 + D, COL_DOT = 256 + D + D / 2;  // NB == 2 only
+  static constexpr uint32_t COL_QT = 256 + D, COL_DOT = 256 + D + D / 2;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t RED_BYTES = (128u * (D / 2 + 1) * 4u + 1023u) / 1024u * 1024u;
   static_assert(NS * STAGE >= RED_BYTES + TabStage<D>::BYTES,
@@ -592,10 +536,10 @@ struct DqCfg {
 enum DqBar {
   QB_Q_FULL = 0,
   QB_KV_FULL = 1,                      // +stage
-  QB_KV_EMPTY = 1 + RA_DQ_STAGES,      // +stage
-  QB_SP_FULL = 1 + 2 * RA_DQ_STAGES,   // +buffer
-  QB_DS_FULL = QB_SP_FULL + RA_DQ_BUFS,  // +buffer, kDsArrivals arrivals
-  QB_ACC_DONE = QB_DS_FULL + RA_DQ_BUFS,
+  QB_KV_EMPTY = 1 + kDqStages,         // +stage
+  QB_SP_FULL = 1 + 2 * kDqStages,      // +buffer
+  QB_DS_FULL = QB_SP_FULL + 2,         // +buffer, kDsArrivals arrivals
+  QB_ACC_DONE = QB_DS_FULL + 2,
   QB_DRAIN,
   QB_QT_READY,                         // Q~, dO copied into TMEM (one arrival per softmax warp)
   QB_COUNT
@@ -632,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == kSoftThreads) {
     for (int i = 0; i < QB_COUNT; ++i)
-      mbar_init(&bar[i], (i >= QB_DS_FULL && i < QB_DS_FULL + RA_DQ_BUFS) ? kDsArrivals
+      mbar_init(&bar[i], (i >= QB_DS_FULL && i < QB_DS_FULL + 2) ? kDsArrivals
                          : i == QB_QT_READY                       ? kSoftThreads / 32
                                                                   : 1);
     *abort_flag = 0;
@@ -692,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const SDesc dqd = sdesc_split(base_s, 16, 1024);                   // Q~, dO K-major
       const SDesc dkm = sdesc_split(base_s + C::OFF_ST, 16, 1024);      // K~_j, V_j K-major
       const SDesc dmn = sdesc_split(base_s + C::OFF_ST, C::KCH, 1024);  // K~_j read MN-major
-      bool ok = mbar_wait_warp(&bar[C::NB == 2 ? QB_QT_READY : QB_Q_FULL], 0, abort_flag, err,
+      bool ok = mbar_wait_warp(&bar[QB_QT_READY], 0, abort_flag, err,
                                KID, 2, wait_ns);
       // S / dP of key tile j into TMEM buffer j % NB, which last held dS of tile j - NB;
       // the dQ MMA that read it was issued earlier by this thread (in-order execution).
@@ -702,12 +646,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         tc_fence_after();
         const SDesc ks = sdesc_advance(dkm, s * C::STAGE);
-        if constexpr (C::NB == 2 && D == 128 && RA_MMA_BATCH) {
+        if constexpr (D == 128) {
           mma8_kmajor<true, 0, C::KCH>(tmem + C::COL_S + b * 128, tmem + C::COL_QT,
                                        sdesc_at(ks, 0), idS, 0);
           mma8_kmajor<true, 0, C::KCH>(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT,
                                        sdesc_at(ks, C::KTILE), idDP, 0);
-        } else if constexpr (C::NB == 2) {
+        } else {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
@@ -718,21 +662,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
             mma_ts_warp(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT + 8 * kk,
-                        sdesc_at(ks, C::KTILE + kq), idDP, kk > 0);
-          }
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
-            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-            mma_ss_warp(tmem + C::COL_S + b * 128, sdesc_at(dqd, C::OFF_Q + ka),
-                        sdesc_at(ks, kq), idS, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk / 4) * C::QCH + (kk % 4) * 32;
-            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-            mma_ss_warp(tmem + C::COL_DP + b * 128, sdesc_at(dqd, C::OFF_DO + ka),
                         sdesc_at(ks, C::KTILE + kq), idDP, kk > 0);
           }
         }
@@ -749,15 +678,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const SDesc km = sdesc_advance(dmn, s * C::STAGE);
         // dQ~ += dS K~_j with dS read from TMEM
-        if constexpr (RA_MMA_BATCH) {
-          mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
-              tmem + C::COL_DQ, tmem + C::COL_S + b * 128, sdesc_at(km, 0), idDQ, j > 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)
-            mma_ts_warp(tmem + C::COL_DQ, tmem + C::COL_S + b * 128 + packed_col(16 * kk),
-                        sdesc_at(km, kk * 2048), idDQ, (j > 0 || kk > 0));
-        }
+        mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
+            tmem + C::COL_DQ, tmem + C::COL_S + b * 128, sdesc_at(km, 0), idDQ, j > 0);
         mma_commit_warp(&bar[QB_KV_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[QB_ACC_DONE]);
@@ -768,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax warpgroups
     const int t = threadIdx.x % 128;      // query row == TMEM lane
-    const int half = threadIdx.x / 128;   // warpgroup: takes key tiles j = half (mod kSoftWG)
+    const int half = threadIdx.x / 128;   // warpgroup: key columns 32 half .. 32 half + 31
     const int row = qtile * C::BM + t;
     const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const float scale_log2 = kLog2e / sqrtf((float)D);
@@ -778,20 +700,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dS s = P fma(dP, s, -Delta s) costs one multiply less per element, bit for bit the same
     const float dlt_s = deltap[(size_t)bh * npad + row] * dss;
     bool ok = true;
-    if constexpr (C::NB == 2) {
-      // the stationary Q~ and dO rows into TMEM (warpgroup g copies tiles g, g + kSoftWG, ...)
+    {
+      // the stationary Q~ (warpgroup 0) and dO (warpgroup 1) rows into TMEM
       ok = mbar_wait_warp(&bar[QB_Q_FULL], 0, abort_flag, err, KID, 11, wait_ns);
       if (ok) {
-        for (int src = half; src < 2; src += kSoftWG)
-          tile_row_to_tmem<D>(base_s + (src == 0 ? C::OFF_Q : C::OFF_DO), C::QCH, t,
-                              lane_base + (src == 0 ? C::COL_QT : C::COL_DOT));
+        tile_row_to_tmem<D>(base_s + (half == 0 ? C::OFF_Q : C::OFF_DO), C::QCH, t,
+                            lane_base + (half == 0 ? C::COL_QT : C::COL_DOT));
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[QB_QT_READY]);
     }
-    for (int j = kSplit ? 0 : half; ok && j < nk; j += kTileStep) {
+    for (int j = 0; ok && j < nk; ++j) {
       const int b = j % C::NB;
       if (!mbar_wait_warp(&bar[QB_SP_FULL + b], (j / C::NB) & 1, abort_flag, err, KID, 6,
                           wait_ns)) {
@@ -803,9 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t dp_base = lane_base + C::COL_DP + b * 128;
       const int key0 = j * C::BK;
       const bool need_mask = (causal && key0 + C::BK - 1 > qtile * C::BM) || (key0 + C::BK > n);
-#pragma unroll
-      for (int hh = 0; hh < kHalves; ++hh) {
-        const int h = kSplit ? half : hh;
+      {
+        const int h = half;  // this warpgroup's 32 columns
         uint32_t sr[32], dr[32];
         tmem_ld32(s_base + 32 * h, sr);
         tmem_ld32(dp_base + 32 * h, dr);
@@ -818,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c = 2 * c2;
           const float2 x2 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
                                   make_float2(scale_log2, scale_log2), make_float2(-lse2, -lse2));
-          float2 p2 = make_float2(exp2_col(x2.x, 32 * h + c), exp2_col(x2.y, 32 * h + c + 1));
+          float2 p2 = make_float2(fast_exp2(x2.x), fast_exp2(x2.y));
           if (need_mask) {
             const int key = key0 + 32 * h + c;
             if (key >= n || (causal && key > row)) p2.x = 0.f;
@@ -1311,339 +1231,6 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
   return cudaGetLastError();
 }
 
-// ======================================================================== dK, dV, TMEM A
-// A variant of the dK/dV kernel that keeps the stationary K~ and V in TMEM as the A
-// operands of S^T = K~ Q~_i^T and dP^T = V dO_i^T (TS MMAs), instead of re-reading them
-// from shared memory for every streamed query tile.  Per 64 streamed queries the SS form
-// moves about 160 KB through shared memory (TMA writes plus A and B reads), more than the
-// 1024 cycles of tensor work allow at 128 B/clk; with K~ and V in TMEM it is about 96 KB.
-// The TMEM they take (D/2 columns each) leaves room for two [S^T | dP^T] buffers of 32
-// queries, so queries stream 32 at a time, and the two softmax warpgroups take alternate
-// steps (warpgroup g owns buffer g).  MMAs per step: S^T, dP^T M = 128, N = 32, K = d;
-// dV += P^T dO_i, dK~ += dS^T Q~_i M = 128, N = d, K = 32.  Same arithmetic, epilogue and
-// partials as bwd_dkdv_kernel.  Chosen per call by RA_BWD_DKDV_TMEM=1; off by default.
-template <int D>
-struct DkdvTmCfg {
-  static constexpr int BN = 128, BQ = 32, NS = 8, CH = D / 64;
-  static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
-  static constexpr uint32_t KTILE = KCH * CH;
-  static constexpr uint32_t QCH = 32u * 128u;   // chunk of a 32-row tile
-  static constexpr uint32_t QTILE = QCH * CH;
-  static constexpr uint32_t VEC = BQ * 4;
-  static constexpr uint32_t STAGE = (2 * QTILE + 2 * VEC + 1023) / 1024 * 1024;
-  static constexpr uint32_t OFF_K = 0, OFF_V = KTILE, OFF_ST = 2 * KTILE;
-  static constexpr uint32_t OFF_BAR = OFF_ST + NS * STAGE;
-  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  // TMEM: buffer b of [S^T (32 fp32) | dP^T (32 fp32)] at 64 b, P^T (bf16) and dS^T (fp16)
-  // written back as pairs over the first 16 columns of each; K~ (fp16) and V (bf16) rows as
-  // A operands at 128 and 128 + D/2; the dV and dK~ accumulators at 256 and 256 + D.
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 32, COL_KT = 128, COL_VT = 128 + D / 2;
-  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + D;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t RED_BYTES = (128u * (D / 2 + 1) * 4u + 1023u) / 1024u * 1024u;
-  static_assert(NS * STAGE >= RED_BYTES + TabStage<D>::BYTES,
-                "torque buffer and staged table fit the stages");
-  static_assert(SMEM <= 232448, "fits the shared memory of one CTA");
-};
-
-enum DkdvTmBar {
-  TB_KV_FULL = 0,
-  TB_Q_FULL = 1,     // +stage (8)
-  TB_Q_EMPTY = 9,    // +stage (8)
-  TB_SDP_FULL = 17,  // +buffer: S^T and dP^T of that buffer computed
-  TB_DS_FULL = 19,   // +buffer: P^T, dS^T written (4 warp arrivals: one warpgroup)
-  TB_ACC_DONE = 21,
-  TB_DRAIN = 22,
-  TB_KV_READY = 23,  // K~ and V rows copied into TMEM (one arrival per softmax warp)
-  TB_COUNT = 24
-};
-static_assert(8 * TB_COUNT + 8 <= 256, "barriers, TMEM slot and abort flag fit the reserve");
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dkdv_tmem_kernel(const __grid_constant__ CUtensorMap map_kt,
-                         const __grid_constant__ CUtensorMap map_v,
-                         const __grid_constant__ CUtensorMap map_qt32,
-                         const __grid_constant__ CUtensorMap map_do32,
-                         const float* __restrict__ lse2p, const float* __restrict__ deltap,
-                         const float2* __restrict__ table, const uint32_t* __restrict__ stats,
-                         __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                         float* __restrict__ dpart, int n, int BH, int causal, uint32_t* err,
-                         uint64_t wait_ns) {
-  using C = DkdvTmCfg<D>;
-  static_assert(kSoftWG == 2 && kSoftThreads == 256, "two softmax warpgroups");
-  constexpr int KID = K_BWD_DKDV_SM100;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_s = smem_u32(smem_raw);
-  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
-  uint8_t* base = smem_raw + (base_s - raw_s);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * TB_COUNT);
-  volatile int* abort_flag =
-      reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * TB_COUNT + 4);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int jt = (int)(blockIdx.x / BH);  // key tile; low tiles carry most causal work
-  const int bh = (int)(blockIdx.x % BH);
-  const int npad = (int)((n + 127) / 128 * 128);
-  const int qstart = causal ? jt * C::BN : 0;
-  const int nq = (n - qstart + C::BQ - 1) / C::BQ;
-
-  if (threadIdx.x == kSoftThreads) {
-    for (int i = 0; i < TB_COUNT; ++i)
-      mbar_init(&bar[i], (i == TB_DS_FULL || i == TB_DS_FULL + 1) ? 4
-                         : i == TB_KV_READY                       ? kSoftThreads / 32
-                                                                  : 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == kProdWarp) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&map_kt);
-      tma_prefetch_desc(&map_v);
-      tma_prefetch_desc(&map_qt32);
-      tma_prefetch_desc(&map_do32);
-      mbar_arrive_expect_tx(&bar[TB_KV_FULL], 2 * C::KTILE);
-      for (int c = 0; c < C::CH; ++c) {
-        tma_load_3d(base + C::OFF_K + c * C::KCH, &map_kt, &bar[TB_KV_FULL], c * 64, jt * C::BN,
-                    bh);
-        tma_load_3d(base + C::OFF_V + c * C::KCH, &map_v, &bar[TB_KV_FULL], c * 64, jt * C::BN,
-                    bh);
-      }
-      int issued = -1;
-      for (int it = 0; it < nq; ++it) {
-        const int s = it % C::NS;
-        if (!mbar_wait(&bar[TB_Q_EMPTY + s], ((it / C::NS) & 1) ^ 1, abort_flag, err, KID, 1,
-                       wait_ns))
-          break;
-        const int i0 = qstart + it * C::BQ;
-        uint8_t* st = base + C::OFF_ST + s * C::STAGE;
-        mbar_arrive_expect_tx(&bar[TB_Q_FULL + s], 2 * C::QTILE + 2 * C::VEC);
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_3d(st + c * C::QCH, &map_qt32, &bar[TB_Q_FULL + s], c * 64, i0, bh);
-          tma_load_3d(st + C::QTILE + c * C::QCH, &map_do32, &bar[TB_Q_FULL + s], c * 64, i0,
-                      bh);
-        }
-        bulk_load(st + 2 * C::QTILE, lse2p + (size_t)bh * npad + i0, C::VEC,
-                  &bar[TB_Q_FULL + s]);
-        bulk_load(st + 2 * C::QTILE + C::VEC, deltap + (size_t)bh * npad + i0, C::VEC,
-                  &bar[TB_Q_FULL + s]);
-        issued = it;
-      }
-      if (*abort_flag) {
-        int dummy = 0;
-        mbar_wait(&bar[TB_KV_FULL], 0, &dummy, err, KID, 20, wait_ns);
-        for (int it = max(0, issued - C::NS + 1); it <= issued; ++it)
-          mbar_wait(&bar[TB_Q_FULL + it % C::NS], (it / C::NS) & 1, &dummy, err, KID, 21,
-                    wait_ns);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    {  // the whole warp: converged issue, one elected lane
-      constexpr uint32_t idST = idesc_f16_f32(128, C::BQ, 0, 0);   // fp16 K~ Q~^T
-      constexpr uint32_t idDPT = idesc_bf16_f32(128, C::BQ, 0, 0);  // bf16 V dO^T
-      constexpr uint32_t idDV = idesc_bf16_f32(128, D, 0, 1);       // bf16 P^T dO
-      constexpr uint32_t idDK = idesc_f16_f32(128, D, 0, 1);        // fp16 dS^T Q~
-      const SDesc dkm = sdesc_split(base_s, 16, 1024);       // Q~ / dO tiles, K-major
-      const SDesc dmn = sdesc_split(base_s, C::QCH, 1024);   // Q~ / dO tiles read MN-major
-      bool ok = mbar_wait_warp(&bar[TB_KV_READY], 0, abort_flag, err, KID, 2, wait_ns);
-      // S^T / dP^T of step `it` into TMEM buffer it & 1, which last held P^T / dS^T of step
-      // it - 2, whose dV / dK MMAs were issued earlier by this thread (in order).
-      auto issue_sdp = [&](int it) -> bool {
-        const int s = it % C::NS, b = it & 1;
-        if (!mbar_wait_warp(&bar[TB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3,
-                            wait_ns))
-          return false;
-        tc_fence_after();
-        const SDesc qs = sdesc_advance(dkm, C::OFF_ST + s * C::STAGE);
-        const uint32_t st = tmem + b * 64 + C::COL_ST, dpt = tmem + b * 64 + C::COL_DPT;
-        if constexpr (D == 128 && RA_MMA_BATCH) {
-          mma8_kmajor<true, 0, C::QCH>(st, tmem + C::COL_KT, sdesc_at(qs, 0), idST, 0);
-          mma8_kmajor<true, 0, C::QCH>(dpt, tmem + C::COL_VT, sdesc_at(qs, C::QTILE), idDPT, 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-            mma_ts_warp(st, tmem + C::COL_KT + 8 * kk, sdesc_at(qs, kq), idST, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-            mma_ts_warp(dpt, tmem + C::COL_VT + 8 * kk, sdesc_at(qs, C::QTILE + kq), idDPT,
-                        kk > 0);
-          }
-        }
-        mma_commit_warp(&bar[TB_SDP_FULL + b]);
-        return true;
-      };
-      if (ok) tc_fence_after();
-      if (ok && nq > 0) ok = issue_sdp(0);
-      for (int it = 0; ok && it < nq; ++it) {
-        if (it + 1 < nq && !issue_sdp(it + 1)) break;
-        const int s = it % C::NS, b = it & 1;
-        if (!mbar_wait_warp(&bar[TB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5,
-                            wait_ns))
-          break;
-        tc_fence_after();
-        const SDesc qm = sdesc_advance(dmn, C::OFF_ST + s * C::STAGE);
-        // dV += P^T dO_i and dK~ += dS^T Q~_i, P^T and dS^T read from TMEM (16 queries,
-        // 8 packed columns, per K-step)
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_DV, tmem + b * 64 + C::COL_ST + 8 * kk,
-                      sdesc_at(qm, C::QTILE + kk * 2048), idDV, (it > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          mma_ts_warp(tmem + C::COL_DK, tmem + b * 64 + C::COL_DPT + 8 * kk,
-                      sdesc_at(qm, kk * 2048), idDK, (it > 0 || kk > 0));
-        mma_commit_warp(&bar[TB_Q_EMPTY + s]);
-      }
-      if (ok) mma_commit_warp(&bar[TB_ACC_DONE]);
-      mma_commit_warp(&bar[TB_DRAIN]);
-      int dummy = 0;
-      mbar_wait_warp(&bar[TB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
-    }
-  } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = threadIdx.x % 128;      // key row == TMEM lane
-    const int half = threadIdx.x / 128;   // warpgroup: steps it = half (mod 2), buffer half
-    const int key = jt * C::BN + t;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-    const float scale_log2 = kLog2e / sqrtf((float)D);
-    const float dss = ds_scale(stats);
-    // the stationary K~ (warpgroup 0) and V (warpgroup 1) rows into TMEM
-    bool ok = mbar_wait_warp(&bar[TB_KV_FULL], 0, abort_flag, err, KID, 11, wait_ns);
-    if (ok) {
-      tile_row_to_tmem<D>(base_s + (half == 0 ? C::OFF_K : C::OFF_V), C::KCH, t,
-                          lane_base + (half == 0 ? C::COL_KT : C::COL_VT));
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar[TB_KV_READY]);
-    const uint32_t st_base = lane_base + half * 64 + C::COL_ST;
-    const uint32_t dpt_base = lane_base + half * 64 + C::COL_DPT;
-    for (int it = half; ok && it < nq; it += 2) {
-      const int s = it % C::NS;
-      const int i0 = qstart + it * C::BQ;
-      if (!mbar_wait_warp(&bar[TB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6,
-                          wait_ns) ||
-          !mbar_wait_warp(&bar[TB_SDP_FULL + half], (it >> 1) & 1, abort_flag, err, KID, 7,
-                          wait_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float4* lv = reinterpret_cast<const float4*>(base + C::OFF_ST + s * C::STAGE +
-                                                         2 * C::QTILE);
-      const float4* dvv = lv + C::BQ / 4;
-      const bool need_mask = causal && (i0 < jt * C::BN + C::BN);
-      uint32_t sr[32], dr[32];
-      tmem_ld32(st_base, sr);
-      tmem_ld32(dpt_base, dr);
-      tmem_wait_ld(sr);
-      tmem_wait_ld(dr);
-      uint32_t pw[16], dw[16];
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 l4 = lv[c4], d4 = dvv[c4];
-        const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pv[4], dsv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;  // streamed query i0 + c
-          float p = exp2_col(__uint_as_float(sr[c]) * scale_log2 - la[e], c);
-          if (need_mask && (i0 + c < key)) p = 0.f;
-          pv[e] = p;
-          dsv[e] = p * (__uint_as_float(dr[c]) - da[e]) * dss;
-        }
-        pw[2 * c4] = pack_g(pv[0], pv[1]);
-        pw[2 * c4 + 1] = pack_g(pv[2], pv[3]);
-        dw[2 * c4] = pack_f16x2_sat(dsv[0], dsv[1]);
-        dw[2 * c4 + 1] = pack_f16x2_sat(dsv[2], dsv[3]);
-      }
-      tmem_st16(st_base, pw);
-      tmem_st16(dpt_base, dw);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[TB_DS_FULL + half]);
-    }
-    if (ok && mbar_wait_warp(&bar[TB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
-      tc_fence_after();
-      const bool live = key < n;
-      // every Q~/dO stage has been consumed: the ring holds the torque buffer and the table
-      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
-      uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
-      stage_table<D>(table, jt * C::BN, n, tab);
-      // dV row (this thread's D / 2 columns)
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        const int c = half * (D / 64) + cc;
-        uint32_t r[32];
-        tmem_ld32(lane_base + C::COL_DV + 32 * c, r);
-        tmem_wait_ld(r);
-        if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)bh * n + key) * D + 32 * c);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float* f = reinterpret_cast<const float*>(&r[8 * u]);
-            dst[u] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-          }
-        }
-      }
-      // dK row, its inverse rotation and the K-side torques
-      softmax_group_sync();
-      grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
-                           tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
-                           (float)key - 0.5f * (float)(n - 1), live,
-                           dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
-                           half);
-      softmax_group_sync();
-      const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      if (dpart != nullptr && threadIdx.x < 128)
-        write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
-                                 ntile64, t);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-template <int D>
-cudaError_t launch_dkdv_tmem_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                               const float* deltap, const float2* table, const uint32_t* stats,
-                               void* dk, void* dv, float* dpart, const DevCtl& ctl,
-                               cudaStream_t s) {
-  using C = DkdvTmCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tmem_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  const int BH = (int)(p.B * p.H);
-  const long long ntk = (p.n + C::BN - 1) / C::BN;
-  bwd_dkdv_tmem_kernel<D><<<(unsigned)(ntk * BH), kThreads, C::SMEM, s>>>(
-      maps.kt, maps.v, maps.qt32, maps.dO32, lse2p, deltap, table, stats, (__nv_bfloat16*)dk,
-      (__nv_bfloat16*)dv, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_fused_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
                            const float* deltap, const float2* table, const uint32_t* stats,
                            void* dk, void* dv, float* dqacc, float* dpart, const DevCtl& ctl,
@@ -1725,16 +1312,6 @@ cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, cons
                                 void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s) {
   if (p.d == 64) return launch_dq_d<64>(p, maps, lse2p, deltap, table, stats, dq, dpart, ctl, s);
   return launch_dq_d<128>(p, maps, lse2p, deltap, table, stats, dq, dpart, ctl, s);
-}
-
-cudaError_t launch_bwd_dkdv_tmem_sm100(const ra_problem& p, const Sm100Maps& maps,
-                                       const float* lse2p, const float* deltap,
-                                       const float2* table, const uint32_t* stats, void* dk,
-                                       void* dv, float* dpart, const DevCtl& ctl,
-                                       cudaStream_t s) {
-  if (p.d == 64)
-    return launch_dkdv_tmem_d<64>(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
-  return launch_dkdv_tmem_d<128>(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
 }
 
 }  // namespace ra

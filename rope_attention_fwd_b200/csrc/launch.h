@@ -47,7 +47,6 @@ cudaError_t launch_bwd_dkdv_f32(const ra_problem& p, const float* qt, const floa
 struct Sm100Maps {
   CUtensorMap qt, kt, v, dO;         // boxes of 64 columns x 128 rows
   CUtensorMap qt64, kt64, v64, dO64; // boxes of 64 columns x 64 rows
-  CUtensorMap qt32, dO32;            // boxes of 64 columns x 32 rows (TMEM-operand dK/dV only)
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
@@ -66,13 +65,6 @@ cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,
                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
                                   const DevCtl& ctl, cudaStream_t s);
-// The dK/dV kernel with K~ and V kept in TMEM as MMA operands and queries streamed 32 at a
-// time (needs maps.qt32, maps.dO32); chosen per call by RA_BWD_DKDV_TMEM=1, off by default.
-cudaError_t launch_bwd_dkdv_tmem_sm100(const ra_problem& p, const Sm100Maps& maps,
-                                       const float* lse2p, const float* deltap,
-                                       const float2* table, const uint32_t* stats, void* dk,
-                                       void* dv, float* dpart, const DevCtl& ctl,
-                                       cudaStream_t s);
 // Fused dK, dV and dQ~ (into the fp32 accumulator dqacc, zeroed by the caller) in one pass
 // (d = 128); dq_finish turns the accumulator into dQ.
 cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,

@@ -138,28 +138,35 @@ ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
                               void* dq, void* dk, void* dv, float* dalpha,
                               void* ws, size_t ws_bytes, void* stream);
 
-/* ---- the projections around the path (plain cuBLAS GEMMs) ---------------------
+/* ---- the projections around the path --------------------------------------------
  * "RoPE attention can be trained in almost-linear time" (Lemma 4.1) states the loss
  * gradient with respect to the weights; these two calls carry the path's dQ, dK, dV back
  * to the projection weights and the layer input.  Row-major layouts: x [B, n, d_model]
  * (dtype of p); each W [d_model, H*d] (dtype of p) with head h in columns h*d..h*d+d-1;
  * q, k, v, dq, dk, dv [B, H, n, d] (dtype of p); dW [d_model, H*d] fp32; dx [B, n, d_model]
- * fp32.  fp32 accumulation (no TF32); fixed GEMM order (deterministic).  Pointers 16-byte
- * aligned; d_model in 1..2^20.  Only p's B, H, n, d and dtype are used. */
+ * fp32.  The library's own GEMMs: bf16 on the tcgen05 tensor cores (d in {64, 128},
+ * d_model a multiple of 8, else RA_ERR_UNSUPPORTED), fp32 on CUDA cores (exact fp32
+ * products); fp32 accumulation in a fixed order (deterministic).  Pointers 16-byte
+ * aligned; d_model in 1..2^20.  Only p's B, H, n, d and dtype are used.
+ * ws / ws_bytes (both calls): caller workspace, 256-byte aligned, of at least
+ * rope_attn_proj_workspace_bytes(p) bytes for rope_attn_proj_bwd and at least 1024 bytes
+ * for rope_attn_proj_fwd (RA_ERR_WORKSPACE otherwise).  Its first 64 bytes are the device
+ * error word, read with rope_attn_device_status (a GEMM wait that expires records
+ * RA_ERR_TIMEOUT there). */
 
-/* q[b,h] = x[b] W_Q[:, h], likewise k, v. */
+/* [q | k | v][b, h] = x[b] [W_Q | W_K | W_V][:, h] (one GEMM). */
 ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x,
                              const void* wq, const void* wk, const void* wv,
-                             void* q, void* k, void* v, void* stream);
+                             void* q, void* k, void* v, void* ws, size_t ws_bytes,
+                             void* stream);
 
-/* Bytes of caller workspace rope_attn_proj_bwd needs: one [B*n, H*d] copy of a gradient in
- * the dtype (0 if *p is invalid). */
+/* Bytes of caller workspace rope_attn_proj_bwd needs: the error word and the three
+ * gradients, each merged to [B*n, H*d] rows in the dtype (0 if *p is invalid). */
 size_t rope_attn_proj_workspace_bytes(const ra_problem* p);
 
-/* dW_Q = sum_b x[b]^T dq[b] (dq[b] read as [n, H*d]), likewise dW_K, dW_V, and
- * dx[b] = sum_h dq[b,h] W_Q[:,h]^T + dk[b,h] W_K[:,h]^T + dv[b,h] W_V[:,h]^T.  ws (16-byte
- * aligned, ws_bytes >= rope_attn_proj_workspace_bytes) holds each gradient merged to
- * [B*n, H*d] rows, so every product is one GEMM; RA_ERR_WORKSPACE if it is too small. */
+/* dW_Q = sum_b x[b]^T dq[b] (dq[b] read as [n, H*d]), likewise dW_K, dW_V (one GEMM), and
+ * dx[b] = sum_h dq[b,h] W_Q[:,h]^T + dk[b,h] W_K[:,h]^T + dv[b,h] W_V[:,h]^T (one GEMM over
+ * the three gradients side by side). */
 ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x,
                              const void* wq, const void* wk, const void* wv,
                              const void* dq, const void* dk, const void* dv,
@@ -175,7 +182,8 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
  * Inputs as for rope_attn_bwd (o, lse from the forward, dO the upstream gradient).
  * Outputs: g [d/2][2n-1][2] fp32 (re, im; offset D at index D + n - 1; causal: D < 0 is 0)
  * and dalpha [d/2] fp32.  A diagnostic: one (batch, head) at a time with n x n fp32 scratch
- * (workspace from rope_attn_spectrum_workspace_bytes; n <= 32768); deterministic. */
+ * (workspace from rope_attn_spectrum_workspace_bytes; n <= 32768), its score matrices from
+ * fp32 CUDA-core GEMMs; deterministic. */
 size_t rope_attn_spectrum_workspace_bytes(const ra_problem* p);
 ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, const void* v,
                              const void* o, const float* lse, const void* dO,

@@ -63,7 +63,7 @@ def lib():
         L.rope_attn_alpha_adam.argtypes = [ctypes.POINTER(RaAdam), ctypes.c_int64, vp, vp, vp, vp,
                                            vp]
         L.rope_attn_alpha_adam.restype = ctypes.c_int
-        L.rope_attn_proj_fwd.argtypes = [P, ctypes.c_int64] + [vp] * 8
+        L.rope_attn_proj_fwd.argtypes = [P, ctypes.c_int64] + [vp] * 8 + [sz, vp]
         L.rope_attn_proj_fwd.restype = ctypes.c_int
         L.rope_attn_proj_bwd.argtypes = [P, ctypes.c_int64] + [vp] * 12 + [sz, vp]
         L.rope_attn_proj_bwd.restype = ctypes.c_int
@@ -231,16 +231,19 @@ def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None
     return dq, dk, dv, dalpha
 
 
-def rope_attn_proj_fwd(x, wq, wk, wv, H, q=None, k=None, v=None):
-    """q, k, v [B, H, n, d] = x [B, n, d_model] @ W [d_model, H*d], head h in columns h*d.."""
+def rope_attn_proj_fwd(x, wq, wk, wv, H, q=None, k=None, v=None, ws=None):
+    """q, k, v [B, H, n, d] = x [B, n, d_model] @ W [d_model, H*d], head h in columns h*d..
+    ws: a workspace of at least 1024 bytes (its first 64 bytes are the error word)."""
     B, n, dm = x.shape
     d = wq.shape[1] // H
     prob = problem(B, H, n, d, x.dtype, False, 1.0)
     out = [torch.empty((B, H, n, d), dtype=x.dtype, device=x.device) if t is None else t
            for t in (q, k, v)]
+    if ws is None:
+        ws = torch.empty(1024, dtype=torch.uint8, device=x.device)
     _check("rope_attn_proj_fwd", lib().rope_attn_proj_fwd(
         ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), *[_ptr(t) for t in out],
-        _stream(x.device)))
+        _ptr(ws), ws.numel(), _stream(x.device)))
     return tuple(out)
 
 

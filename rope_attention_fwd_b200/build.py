@@ -61,8 +61,7 @@ def build(force=False, verbose=False):
             if log:
                 sys.stderr.write(log)
     if force or _stale(LIB, objs):
-        cmd = ([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB] + objs
-               + ["-lcublas"])
+        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

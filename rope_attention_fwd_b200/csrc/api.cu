@@ -92,13 +92,6 @@ ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes) {
   return RA_OK;
 }
 
-// Bound on every device-side wait: RA_WAIT_LIMIT_MS (default 2000 ms), read per call.
-uint64_t wait_limit_ns() {
-  const char* s = std::getenv("RA_WAIT_LIMIT_MS");
-  double ms = s ? std::atof(s) : 2000.0;
-  if (!(ms > 0)) ms = 2000.0;
-  return (uint64_t)(ms * 1e6);
-}
 
 // Test hook for the bounded-wait path: RA_DEBUG_STARVE_BLOCK=<cta> makes that CTA of
 // the bf16 forward skip its Q~ load, so its waits expire and it reports RA_ERR_TIMEOUT.
@@ -165,6 +158,31 @@ ra_status prepare(const ra_problem* p, const void* q, const void* k, const float
 }
 
 }  // namespace
+
+namespace ra {
+
+uint64_t wait_limit_ns() {
+  const char* s = std::getenv("RA_WAIT_LIMIT_MS");
+  double ms = s ? std::atof(s) : 2000.0;
+  if (!(ms > 0)) ms = 2000.0;
+  return (uint64_t)(ms * 1e6);
+}
+
+bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace ra
 
 extern "C" {
 
@@ -405,7 +423,7 @@ const char* rope_attn_kernel_name(int id) {
       "rope_table",       "rotate",       "fwd_f32",      "fwd_sm100",
       "loss_partial",     "loss_final",   "bwd_delta",    "bwd_dq_f32",
       "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final",
-      "bwd_fused_sm100",  "dq_finish"};
+      "bwd_fused_sm100",  "dq_finish",    "proj_gemm"};
   return (id >= 0 && id < K_COUNT) ? names[id] : "unknown";
 }
 

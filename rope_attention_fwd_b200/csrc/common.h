@@ -23,7 +23,8 @@ enum KernelId : int {
   K_DALPHA = 11,
   K_BWD_FUSED_SM100 = 12,
   K_DQ_FINISH = 13,
-  K_COUNT = 14
+  K_PROJ_GEMM = 14,
+  K_COUNT = 15
 };
 
 // Rows per dalpha partial (one partial per band per tile of query or key rows).

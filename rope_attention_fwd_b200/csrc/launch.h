@@ -7,6 +7,14 @@
 
 namespace ra {
 
+// Bound on every device-side wait: RA_WAIT_LIMIT_MS (default 2000 ms), read per call.
+uint64_t wait_limit_ns();
+
+// A 2-D row-major tensor map (inner x outer elements, rows row_bytes apart), 128-byte
+// swizzle, box box_inner x box_outer; false if the driver rejects it.
+bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
 struct DevCtl {
   uint32_t* err;        // workspace error word
   uint64_t wait_ns;     // bound on every device-side wait

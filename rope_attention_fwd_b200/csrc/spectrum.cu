@@ -8,17 +8,17 @@
 // P_m'(theta_hat_m) (the backward's dalpha, reached by a second route).
 //
 // A diagnostic, not the hot path: one (batch, head) at a time, S = Q~ K~^T and dP = dO V^T
-// as cuBLAS GEMMs into fp32 n x n scratch, dS = P o (dP - Delta) in place, then one thread
+// as fp32 GEMMs (gemm_sm100.cu, CUDA cores) into fp32 n x n scratch, dS = P o (dP - Delta)
+// in place, then one thread
 // per (band, offset) sums its diagonal of dS z_q conj(z_k) (fp32 per head, fp64 across heads,
 // fixed order: deterministic).
-#include <cublas_v2.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 
-#include "blas.h"
 #include "common.h"
+#include "gemm.h"
 #include "launch.h"
 
 namespace ra {
@@ -184,8 +184,6 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % 256) != 0 || ws_bytes < L.total)
     return RA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cublasHandle_t h = cublas_handle();
-  if (!h || cublasSetStream(h, s) != CUBLAS_STATUS_SUCCESS) return RA_ERR_CUDA;
   uint8_t* w = static_cast<uint8_t*>(ws);
   float2* table = reinterpret_cast<float2*>(w + L.table);
   float* qt = reinterpret_cast<float*>(w + L.qt);
@@ -197,11 +195,14 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
   double2* g64 = reinterpret_cast<double2*>(w + L.g64);
   const int n = (int)p->n, d = (int)p->d, M = d / 2;
   const size_t es = p->dtype == RA_BF16 ? 2 : 4;
-  const cudaDataType_t t = p->dtype == RA_BF16 ? CUDA_R_16BF : CUDA_R_32F;
+  const int in_bf16 = p->dtype == RA_BF16 ? 1 : 0;
+  // S, dP [n][n] fp32 = sum_c A(i, c) B(j, c): both operands K-major [n][d]
+  const GemmSpec sq{n, n, d, 0, 0, 0, 1, 0, 0, 0, 1};
+  const GemmOut os{{S, S, S}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
+  const GemmOut op{{dP, dP, dP}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
   if (launch_table(*p, alpha, table, s) != cudaSuccess) return RA_ERR_CUDA;
   if (cudaMemsetAsync(g64, 0, (size_t)M * (2 * n - 1) * sizeof(double2), s) != cudaSuccess)
     return RA_ERR_CUDA;
-  const float one = 1.f, zero = 0.f;
   const unsigned prep_blocks = (unsigned)(((long long)n * M + 255) / 256);
   const int dmin = p->causal ? 0 : -(n - 1);  // causal: no key after its query
   const dim3 diag_grid((unsigned)((n - 1 - dmin + 1 + 255) / 256), (unsigned)M);
@@ -214,14 +215,13 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
     const char* gh = static_cast<const char*>(dO) + off * es;
     spectrum_prep_kernel<<<prep_blocks, 256, 0, s>>>(qh, table, qt, zq, n, M, p->dtype);
     spectrum_prep_kernel<<<prep_blocks, 256, 0, s>>>(kh, table, kt, zk, n, M, p->dtype);
-    // S_ij (row-major [i][j]) = q~_i . k~_j and dP_ij = dO_i . v_j, as column-major
-    // C = K~ Q~^T and C = V dO^T
-    if (cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, n, n, d, &one, kt, CUDA_R_32F, d, qt,
-                     CUDA_R_32F, d, &zero, S, CUDA_R_32F, n, CUBLAS_COMPUTE_32F,
-                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS ||
-        cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, n, n, d, &one, vh, t, d, gh, t, d, &zero, dP,
-                     CUDA_R_32F, n, CUBLAS_COMPUTE_32F,
-                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+    // S_ij (row-major [i][j]) = q~_i . k~_j and dP_ij = dO_i . v_j
+    const void* qa[1] = {qt};
+    const void* kb[1] = {kt};
+    const void* ga[1] = {gh};
+    const void* vb[1] = {vh};
+    if (launch_gemm_f32(sq, qa, d, 0, kb, d, 0, os, s) != cudaSuccess ||
+        launch_gemm_f32(sq, ga, d, in_bf16, vb, d, in_bf16, op, s) != cudaSuccess)
       return RA_ERR_CUDA;
     spectrum_ds_kernel<<<n, 256, 0, s>>>(S, dP, oh, gh, lse + (size_t)bh * n, n, d, p->causal,
                                          p->dtype);

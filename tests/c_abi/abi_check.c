@@ -29,8 +29,8 @@ int main(void) {
   /* the rotated bf16 Q~ and K~ dominate the workspace */
   expect(ws >= (size_t)2 * 2 * 32 * 8192 * 128 * 2, "headline workspace holds Q~ and K~");
   expect(ws % 1024 == 0, "workspace size is a multiple of 1 KiB");
-  expect(rope_attn_proj_workspace_bytes(&p) == (size_t)2 * 8192 * 32 * 128 * 2,
-         "projection workspace is one merged gradient");
+  expect(rope_attn_proj_workspace_bytes(&p) == (size_t)1024 + 3 * (size_t)2 * 8192 * 32 * 128 * 2,
+         "projection workspace is the error word and three merged gradients");
 
   ra_problem bad = p;
   bad.d = 3;

@@ -141,17 +141,22 @@ def test_alpha_adam_rejects_bad_arguments():
 
 def test_projection_validation_before_any_call():
     """The projection entry points reject bad sizes, pointers and workspaces before they
-    reach cuBLAS or launch anything."""
+    launch anything."""
     lib = rb.lib()
     fake = ctypes.c_void_p(4096)
     p = rb.problem(2, 4, 64, 64, rb.RA_BF16, True, 1e4)
     need = rb.rope_attn_proj_workspace_bytes(p)
-    assert need == 2 * 64 * 4 * 64 * 2
-    # d_model out of range, a null or misaligned operand
-    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 0, *[fake] * 7, None) == 1
-    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, None, *[fake] * 6, None) == 1
-    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, ctypes.c_void_p(4096 + 8), *[fake] * 6,
+    # the error word region and three merged [B n, H d] gradients
+    assert need == 1024 + 3 * 2 * 64 * 4 * 64 * 2
+    # d_model out of range, a null or misaligned operand, a workspace too small
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 0, *[fake] * 7, fake, 1024, None) == 1
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, None, *[fake] * 6, fake, 1024,
                                   None) == 1
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, ctypes.c_void_p(4096 + 8), *[fake] * 6,
+                                  fake, 1024, None) == 1
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 256, *[fake] * 7, fake, 1023, None) == 3
+    # bf16 needs d_model a multiple of 8 (16-byte tensor-map rows)
+    assert lib.rope_attn_proj_fwd(ctypes.byref(p), 100, *[fake] * 7, fake, 1024, None) == 2
     # backward: workspace too small or misaligned, then a head row that is not whole
     # 16-byte vectors (d = 2 in fp32) is unsupported
     assert lib.rope_attn_proj_bwd(ctypes.byref(p), 256, *[fake] * 11, fake, need - 1, None) == 3

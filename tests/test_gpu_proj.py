@@ -1,6 +1,6 @@
 """GPU parity of the projections around the path ("RoPE attention can be trained in
 almost-linear time", Lemma 4.1: the loss gradient with respect to the weights): q, k, v =
-x W through cuBLAS into the path's layout, and dW_Q, dW_K, dW_V, dx back from the path's
+x W through the library's GEMMs (tcgen05 for bf16, CUDA cores for fp32) into the path's layout, and dW_Q, dW_K, dW_V, dx back from the path's
 dq, dk, dv; then the whole layer x -> projections -> attention -> loss -> gradients."""
 import numpy as np
 import pytest

@@ -181,9 +181,10 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
  * dalpha_m = theta_hat_m P_m'(theta_hat_m) (the backward's dalpha by a second route).
  * Inputs as for rope_attn_bwd (o, lse from the forward, dO the upstream gradient).
  * Outputs: g [d/2][2n-1][2] fp32 (re, im; offset D at index D + n - 1; causal: D < 0 is 0)
- * and dalpha [d/2] fp32.  A diagnostic: one (batch, head) at a time with n x n fp32 scratch
- * (workspace from rope_attn_spectrum_workspace_bytes; n <= 32768), its score matrices from
- * fp32 CUDA-core GEMMs; deterministic. */
+ * and dalpha [d/2] fp32.  A diagnostic: one (batch, head) and one block of 64 query rows at
+ * a time, with 64 x n fp32 scratch for the block's score matrices (fp32 CUDA-core GEMMs;
+ * workspace from rope_attn_spectrum_workspace_bytes, O(n d); n <= 32768); sums in a fixed
+ * order (deterministic). */
 size_t rope_attn_spectrum_workspace_bytes(const ra_problem* p);
 ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, const void* v,
                              const void* o, const float* lse, const void* dO,

@@ -7,14 +7,15 @@
 // the model's frequencies, which is the frequency gradient: dalpha_m = theta_hat_m
 // P_m'(theta_hat_m) (the backward's dalpha, reached by a second route).
 //
-// A diagnostic, not the hot path: one (batch, head) at a time, S = Q~ K~^T and dP = dO V^T
-// as fp32 GEMMs (gemm_sm100.cu, CUDA cores) into fp32 n x n scratch, dS = P o (dP - Delta)
-// in place, then one thread
+// A diagnostic, not the hot path: one (batch, head) and one block of 64 query rows at a time,
+// S = Q~ K~^T and dP = dO V^T of the block as fp32 GEMMs (gemm_sm100.cu, CUDA cores) into
+// 64 x n fp32 scratch, dS = P o (dP - Delta) in place, then one thread
 // per (band, offset) sums its diagonal of dS z_q conj(z_k) (fp32 per head, fp64 across heads,
 // fixed order: deterministic).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "common.h"
@@ -45,13 +46,15 @@ __global__ void spectrum_prep_kernel(const void* __restrict__ x, const float2* _
   zb[(long long)m * n + p] = make_float2(x0, x1);
 }
 
-// One block per query row i: Delta_i = sum_c dO_ic O_ic, then in place over row i of s:
-// dS_ij = P_ij (dP_ij - Delta_i), P_ij = exp(S_ij / sqrt(d) - lse_i) (0 for j > i if causal).
+// One block per query row i of the row block starting at row i0: Delta_i =
+// sum_c dO_ic O_ic, then in place over that row of s: dS_ij = P_ij (dP_ij - Delta_i),
+// P_ij = exp(S_ij / sqrt(d) - lse_i) (0 for j > i if causal).
 __global__ void __launch_bounds__(256)
     spectrum_ds_kernel(float* __restrict__ s, const float* __restrict__ dp,
                        const void* __restrict__ o, const void* __restrict__ dO,
-                       const float* __restrict__ lse, int n, int d, int causal, int dtype) {
-  const int i = blockIdx.x;
+                       const float* __restrict__ lse, int i0, int n, int d, int causal,
+                       int dtype) {
+  const int r = blockIdx.x, i = i0 + r;
   float acc = 0.f;
   for (int c = threadIdx.x; c < d; c += blockDim.x)
     acc += load_x(dO, (long long)i * d + c, dtype) * load_x(o, (long long)i * d + c, dtype);
@@ -64,31 +67,32 @@ __global__ void __launch_bounds__(256)
   }
   const float delta = red[0];
   const float scale = rsqrtf((float)d), l = lse[i];
-  float* row = s + (long long)i * n;
-  const float* dprow = dp + (long long)i * n;
+  float* row = s + (long long)r * n;
+  const float* dprow = dp + (long long)r * n;
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
     const float p = (causal && j > i) ? 0.f : expf(row[j] * scale - l);
     row[j] = p * (dprow[j] - delta);
   }
 }
 
-// Thread (m, D) adds sum_{i - j = D} dS_ij zq_i conj(zk_j) / sqrt(d) of this head to
-// g64[m][D + n - 1] (fp64 complex).  Consecutive threads take consecutive offsets, so
-// their dS and zk reads are consecutive.
+// Thread (m, D) adds sum_{i - j = D, i0 <= i < i1} dS_ij zq_i conj(zk_j) / sqrt(d) of this
+// head's row block [i0, i1) (rows of ds relative to i0) to g64[m][D + n - 1] (fp64 complex).
+// Blocks and heads run one after another, so every sum is taken in a fixed order.
+// Consecutive threads take consecutive offsets, so their dS and zk reads are consecutive.
 __global__ void __launch_bounds__(256)
     spectrum_diag_kernel(const float* __restrict__ ds, const float2* __restrict__ zq,
                          const float2* __restrict__ zk, double2* __restrict__ g64, int n, int d,
-                         int dmin) {
+                         int dmin, int i0, int i1) {
   const int m = blockIdx.y;
   const int D = dmin + (int)(blockIdx.x * blockDim.x + threadIdx.x);
   if (D > n - 1) return;
   const float2* q = zq + (long long)m * n;
   const float2* k = zk + (long long)m * n;
   float re = 0.f, im = 0.f;
-  const int i0 = D > 0 ? D : 0, i1 = D < 0 ? n + D : n;
-  for (int i = i0; i < i1; ++i) {
+  const int lo = max(i0, D > 0 ? D : 0), hi = min(i1, D < 0 ? n + D : n);
+  for (int i = lo; i < hi; ++i) {
     const int j = i - D;
-    const float w = ds[(long long)i * n + j];
+    const float w = ds[(long long)(i - i0) * n + j];
     const float2 a = q[i], b = k[j];
     // w * a * conj(b) = w ((a.x b.x + a.y b.y) + i (a.y b.x - a.x b.y))
     re = fmaf(w, fmaf(a.x, b.x, a.y * b.y), re);
@@ -131,6 +135,7 @@ __global__ void __launch_bounds__(256)
 
 struct SpecLayout {
   size_t table, qt, kt, s, dp, zq, zk, g64, total;
+  int rows;  // query rows per block: the S and dP scratch is rows x n fp32 each (O(n))
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -138,13 +143,15 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 SpecLayout spec_layout(const ra_problem& p) {
   const size_t n = (size_t)p.n, d = (size_t)p.d, M = d / 2;
   SpecLayout L{};
+  // one 64-row tile of the fp32 GEMM per block: 64 n fp32 of scratch per matrix
+  L.rows = (int)std::min<size_t>(n, 64);
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
   L.table = take(n * M * sizeof(float2));
   L.qt = take(n * d * 4);
   L.kt = take(n * d * 4);
-  L.s = take(n * n * 4);
-  L.dp = take(n * n * 4);
+  L.s = take((size_t)L.rows * n * 4);
+  L.dp = take((size_t)L.rows * n * 4);
   L.zq = take(M * n * sizeof(float2));
   L.zk = take(M * n * sizeof(float2));
   L.g64 = take(M * (2 * n - 1) * sizeof(double2));
@@ -196,8 +203,8 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
   const int n = (int)p->n, d = (int)p->d, M = d / 2;
   const size_t es = p->dtype == RA_BF16 ? 2 : 4;
   const int in_bf16 = p->dtype == RA_BF16 ? 1 : 0;
-  // S, dP [n][n] fp32 = sum_c A(i, c) B(j, c): both operands K-major [n][d]
-  const GemmSpec sq{n, n, d, 0, 0, 0, 1, 0, 0, 0, 1};
+  // S, dP [rows][n] fp32 for a block of query rows: sum_c A(i, c) B(j, c), both operands
+  // K-major [.][d]
   const GemmOut os{{S, S, S}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
   const GemmOut op{{dP, dP, dP}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
   if (launch_table(*p, alpha, table, s) != cudaSuccess) return RA_ERR_CUDA;
@@ -215,17 +222,21 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
     const char* gh = static_cast<const char*>(dO) + off * es;
     spectrum_prep_kernel<<<prep_blocks, 256, 0, s>>>(qh, table, qt, zq, n, M, p->dtype);
     spectrum_prep_kernel<<<prep_blocks, 256, 0, s>>>(kh, table, kt, zk, n, M, p->dtype);
-    // S_ij (row-major [i][j]) = q~_i . k~_j and dP_ij = dO_i . v_j
-    const void* qa[1] = {qt};
-    const void* kb[1] = {kt};
-    const void* ga[1] = {gh};
-    const void* vb[1] = {vh};
-    if (launch_gemm_f32(sq, qa, d, 0, kb, d, 0, os, s) != cudaSuccess ||
-        launch_gemm_f32(sq, ga, d, in_bf16, vb, d, in_bf16, op, s) != cudaSuccess)
-      return RA_ERR_CUDA;
-    spectrum_ds_kernel<<<n, 256, 0, s>>>(S, dP, oh, gh, lse + (size_t)bh * n, n, d, p->causal,
-                                         p->dtype);
-    spectrum_diag_kernel<<<diag_grid, 256, 0, s>>>(S, zq, zk, g64, n, d, dmin);
+    for (int i0 = 0; i0 < n; i0 += L.rows) {
+      const int rows = std::min(L.rows, n - i0);
+      // S_ij (row-major [i - i0][j]) = q~_i . k~_j and dP_ij = dO_i . v_j
+      const GemmSpec sq{rows, n, d, 0, 0, 0, 1, 0, 0, 0, 1};
+      const void* qa[1] = {qt + (size_t)i0 * d};
+      const void* kb[1] = {kt};
+      const void* ga[1] = {gh + (size_t)i0 * d * es};
+      const void* vb[1] = {vh};
+      if (launch_gemm_f32(sq, qa, d, 0, kb, d, 0, os, s) != cudaSuccess ||
+          launch_gemm_f32(sq, ga, d, in_bf16, vb, d, in_bf16, op, s) != cudaSuccess)
+        return RA_ERR_CUDA;
+      spectrum_ds_kernel<<<rows, 256, 0, s>>>(S, dP, oh, gh, lse + (size_t)bh * n, i0, n, d,
+                                              p->causal, p->dtype);
+      spectrum_diag_kernel<<<diag_grid, 256, 0, s>>>(S, zq, zk, g64, n, d, dmin, i0, i0 + rows);
+    }
   }
   spectrum_final_kernel<<<M, 256, 0, s>>>(g64, alpha, g, dalpha, n, d, p->base,
                                           M - p->fixed_bands);

@@ -1,7 +1,8 @@
 """GPU parity of the projections around the path ("RoPE attention can be trained in
 almost-linear time", Lemma 4.1: the loss gradient with respect to the weights): q, k, v =
-x W through the library's GEMMs (tcgen05 for bf16, CUDA cores for fp32) into the path's layout, and dW_Q, dW_K, dW_V, dx back from the path's
-dq, dk, dv; then the whole layer x -> projections -> attention -> loss -> gradients."""
+x W through the library's GEMMs (tcgen05 for bf16, CUDA cores for fp32) into the path's
+layout, and dW_Q, dW_K, dW_V, dx back from the path's dq, dk, dv; then the whole layer
+x -> projections -> attention -> loss -> gradients."""
 import numpy as np
 import pytest
 import torch
@@ -17,9 +18,13 @@ def _rand(shape, dtype, scale, gen):
     return (torch.randn(shape, generator=gen, dtype=torch.float64) * scale).to(dtype).cuda()
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_proj_fwd_and_bwd_match_oracle(dtype):
-    B, H, n, d, dm = 2, 3, 200, 64, 96
+@pytest.mark.parametrize("dtype,B,H,n,d,dm", [
+    (torch.float32, 2, 3, 200, 64, 96),
+    (torch.bfloat16, 2, 3, 200, 64, 96),      # ragged tiles in M, N and K
+    (torch.bfloat16, 2, 4, 512, 128, 256),    # several 128 x 256 tiles in every direction
+    (torch.bfloat16, 1, 2, 130, 128, 520),    # a K chunk and a d_model tail that are partial
+])
+def test_proj_fwd_and_bwd_match_oracle(dtype, B, H, n, d, dm):
     g = torch.Generator().manual_seed(71)
     x = _rand((B, n, dm), dtype, 1.0, g)
     w = [_rand((dm, H * d), dtype, 0.1, g) for _ in range(3)]

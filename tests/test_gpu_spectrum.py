@@ -13,10 +13,12 @@ from rope_attention_fwd_b200 import binding as rb
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dtype,d", [("f32", 16), ("bf16", 64)])
+@pytest.mark.parametrize("dtype,d,n", [("f32", 16, 96), ("bf16", 64, 96), ("bf16", 128, 300),
+                                       ("f32", 128, 200)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_spectrum_matches_oracle_and_backward(dtype, d, causal):
-    wl = small_workload(1, 2, 96, d, dtype, causal, base=500.0, seed=81)
+def test_spectrum_matches_oracle_and_backward(dtype, d, n, causal):
+    """Several 64-row blocks (the last one ragged), d up to 128."""
+    wl = small_workload(1, 2, n, d, dtype, causal, base=500.0, seed=81)
     inp = make(wl)
     q, k, v, e, alpha = (getattr(inp, x).cuda() for x in ("q", "k", "v", "e", "alpha"))
     ws = rb.workspace(rb.problem(wl.B, wl.H, wl.n, wl.d, q.dtype, causal, wl.base), "cuda")

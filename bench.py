@@ -286,7 +286,9 @@ def run_ours(args):
     # ---------------- roofline of the dominant kernel
     peaks, peak_kind = load_peaks()
     f = 0.5 if wl.causal else 1.0
-    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0}
+    # algorithmic FLOPs per (batch, head) in units of n^2 d (halved when causal)
+    alg = {"fwd_sm100": 4.0, "bwd_fused_sm100": 10.0, "bwd_dkdv_sm100": 8.0,
+           "bwd_dq_sm100": 2.0}
     per_kernel = {name: {"launches": c, "avg_ms": t / c, "share": t / sum(
         tt for _, tt in kernels.values())} for name, (c, t) in kernels.items()}
     dom = max(kernels, key=lambda k: kernels[k][1])
@@ -336,10 +338,11 @@ def run_ours(args):
     return 0
 
 
-# Kernels of each phase; the table and rotation run once in fwd and once in bwd.
+# Kernels of each phase (the step's backward takes the table and rotated Q~, K~ from the
+# forward, so those run in the forward only).
 FWD_KERNELS = {"rope_table": 1.0, "rotate": 1.0, "fwd_sm100": 1.0}
-BWD_KERNELS = {"bwd_delta": 1.0, "bwd_dkdv_sm100": 1.0, "bwd_dq_sm100": 1.0,
-               "dalpha_final": 1.0}
+BWD_KERNELS = {"bwd_delta": 1.0, "bwd_fused_sm100": 1.0, "dq_finish": 1.0,
+               "bwd_dkdv_sm100": 1.0, "bwd_dq_sm100": 1.0, "dalpha_final": 1.0}
 
 
 def phase_tflops(kernels, share, flops, steps):

@@ -100,12 +100,6 @@ int starve_block() {
   return s ? std::atoi(s) : -1;
 }
 
-// RA_FWD_SPLIT_S=1 selects the split-half forward (fwd_split_sm100.cu), read per call.
-bool fwd_split_s() {
-  const char* s = std::getenv("RA_FWD_SPLIT_S");
-  return s && std::atoi(s) == 1;
-}
-
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -143,6 +137,20 @@ bool make_map(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows,
   return fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
             const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 [BH][n][d] tensor viewed as (x = d, y = n, z = BH), box = d columns x `rows` rows, no
+// swizzle (the fused backward's dQ~ accumulator, the target of its bulk reductions).
+bool make_map_f32_rows(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)p.d, (cuuint64_t)p.n, (cuuint64_t)(p.B * p.H)};
+  const cuuint64_t strides[2] = {(cuuint64_t)p.d * 4, (cuuint64_t)p.n * p.d * 4};
+  const cuuint32_t box[3] = {(cuuint32_t)p.d, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -228,9 +236,7 @@ ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const
       !make_map(&maps.kt, at<void>(ws, L.kt), *p, 128, true) || !make_map(&maps.v, v, *p, 128))
     return RA_ERR_CUDA;
   DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), starve_block()};
-  RA_LAUNCH(K_FWD_SM100, s,
-            fwd_split_s() ? launch_fwd_split_sm100(*p, maps, o, lse, ctl, s)
-                          : launch_fwd_sm100(*p, maps, o, lse, ctl, s));
+  RA_LAUNCH(K_FWD_SM100, s, launch_fwd_sm100(*p, maps, o, lse, ctl, s));
   return RA_OK;
 }
 
@@ -310,9 +316,10 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
       if (cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)(p->B * p->H * p->n * p->d), s) !=
           cudaSuccess)
         return RA_ERR_CUDA;
+      if (!make_map_f32_rows(&maps.dqacc, dqacc, *p, 64)) return RA_ERR_CUDA;
       RA_LAUNCH(K_BWD_FUSED_SM100, s,
-                launch_bwd_fused_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dqacc,
-                                       dpart, ctl, s));
+                launch_bwd_fused_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
+                                       s));
       RA_LAUNCH(K_DQ_FINISH, s, launch_dq_finish(*p, dqacc, table, stats, dq, s));
     } else {
       // two passes: dK, dV (keys stationary), then dQ (queries stationary, S and dP

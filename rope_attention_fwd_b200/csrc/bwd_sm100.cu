@@ -789,13 +789,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 // kernel above recomputes S and dP (three MMAs per pair for the one that counts); here each
 // query tile's dS is used three times as soon as it exists: dV += P^T dO, dK~ += dS^T Q~
 // (accumulated in TMEM for the whole pass, as in bwd_dkdv_kernel) and dQ~^T = K~^T dS^T,
-// whose 128 x 64 partial goes straight to an fp32 accumulator in global memory
-// (red.global.add) and is rotated back by dq_finish_kernel once every key block has added
-// its share ("RoPE attention can be trained in almost-linear time", Metodologia 1: gamma(x)
-// is formed once per tile and feeds every gradient).
+// whose 128 x 64 partial is staged in shared memory and added to an fp32 accumulator in
+// global memory with one TMA bulk reduction per step (the L2 adds whole sectors; per-element
+// atomics measured about ten times slower), then rotated back by dq_finish_kernel once every
+// key block has added its share ("RoPE attention can be trained in almost-linear time",
+// Metodologia 1: gamma(x) is formed once per tile and feeds every gradient).
 //
 // CTA: 128 keys (K~, V stationary in shared memory), queries streamed 64 at a time through a
-// 4-stage ring.  14 warps:
+// 3-stage ring.  14 warps:
 //   warps 0-7    softmax: both warpgroups take every tile, warpgroup g its query columns
 //                32g..32g+31, thread t its key row t (TMEM lane); P^T (bf16) and dS^T (fp16)
 //                go back into TMEM over S^T / dP^T, and dS^T also into shared memory as the
@@ -803,8 +804,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warp  8      TMA producer;
 //   warp  9      TMEM allocator and MMA issuer;
 //   warps 10-13  dQ drain: thread c owns TMEM lane c = dimension c of dQ~^T; it reads the
-//                step's 64 query columns, adds them into the fp32 accumulator and forms the
-//                Q-side band torques of the step from them.
+//                step's 64 query columns, writes them into the [64][d] fp32 staging tile
+//                (one thread issues the bulk reduction of the tile) and forms the Q-side
+//                band torques of the step from them.
 // TMEM (512 columns): buffer b in {0, 1}: S^T at 128 b, dP^T at 128 b + 64 (64 queries each);
 // dQ~^T of the step that used buffer b is written over its S^T half once the dV MMA has read
 // P^T there (one thread's MMAs execute in issue order); dV at 256, dK~ at 384.
@@ -822,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 struct FusedCfg {
   static_assert(D == 128, "the fused backward takes d = 128");
-  static constexpr int BN = 128, BQ = 64, NS = 4, CH = D / 64;
+  static constexpr int BN = 128, BQ = 64, NS = 3, CH = D / 64;
   static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
   static constexpr uint32_t KTILE = KCH * CH;
   static constexpr uint32_t QCH = 64u * 128u;   // chunk of a 64-row tile
@@ -832,7 +834,9 @@ struct FusedCfg {
   static constexpr uint32_t DSB = 128u * 128u;  // dS^T [128 keys][64 queries] fp16, SW128
   static constexpr uint32_t OFF_K = 0, OFF_V = KTILE, OFF_ST = 2 * KTILE;
   static constexpr uint32_t OFF_DS = OFF_ST + NS * STAGE;
-  static constexpr uint32_t OFF_BAR = OFF_DS + DSB;
+  static constexpr uint32_t DQS = BQ * D * 4u;  // a step's dQ~ partial, [64 queries][d] fp32
+  static constexpr uint32_t OFF_DQS = OFF_DS + DSB;
+  static constexpr uint32_t OFF_BAR = OFF_DQS + DQS;
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 256, COL_DK = 384;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -844,6 +848,10 @@ struct FusedCfg {
 
 constexpr int kFusedDrainWarp0 = kSoftThreads / 32 + 2;          // warps 10..13
 constexpr int kFusedThreads = kSoftThreads + 64 + 128;            // 448
+
+__device__ __forceinline__ void drain_group_sync() {
+  asm volatile("bar.sync 2, 128;" ::: "memory");
+}
 
 enum FusedBar {
   FB_KV_FULL = 0,
@@ -870,8 +878,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                      const float* __restrict__ lse2p, const float* __restrict__ deltap,
                      const float2* __restrict__ table, const uint32_t* __restrict__ stats,
                      __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                     float* __restrict__ dqacc, float* __restrict__ dpart, int n, int BH,
-                     int causal, uint32_t* err, uint64_t wait_ns) {
+                     const __grid_constant__ CUtensorMap map_dqacc, float* __restrict__ dpart,
+                     int n, int BH, int causal, uint32_t* err, uint64_t wait_ns) {
   using C = FusedCfg<D>;
   constexpr int KID = K_BWD_FUSED_SM100;
   extern __shared__ uint8_t smem_raw[];
@@ -1017,6 +1025,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const uint32_t pair_unit = (uint32_t)((c % 64) / 8);
     const uint32_t pair_byte = (uint32_t)((c % 8) & ~1) * 2u;
     double torque = 0.0;  // sum over the CTA's steps of this lane's query parity
+    float* dqs = reinterpret_cast<float*>(base + C::OFF_DQS);
+    if (threadIdx.x == kFusedDrainWarp0 * 32) tma_prefetch_desc(&map_dqacc);
     for (int it = 0; it < nq; ++it) {
       const int s = it % C::NS, b = it & 1;
       const int i0 = qstart + it * C::BQ;
@@ -1032,15 +1042,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[FB_DQ_FREE + b]);
-      // add this step's partial into the accumulator (rows past n are not written)
-      const int live = min(C::BQ, n - i0);
-      float* dst = dqacc + ((size_t)bh * n + i0) * D + c;
+      // the staging tile is free once the previous step's bulk reduction has read it
+      if (threadIdx.x == kFusedDrainWarp0 * 32) bulk_wait_read();
+      drain_group_sync();
+      // row q = query i0 + q, column c: consecutive lanes write consecutive words
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (q < live) red_add_f32(dst + (size_t)q * D, __uint_as_float(r0[q]));
+      for (int q = 0; q < 32; ++q) dqs[q * D + c] = __uint_as_float(r0[q]);
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (32 + q < live) red_add_f32(dst + (size_t)(32 + q) * D, __uint_as_float(r1[q]));
+      for (int q = 0; q < 32; ++q) dqs[(32 + q) * D + c] = __uint_as_float(r1[q]);
+      fence_proxy_async_smem();
+      drain_group_sync();
+      if (threadIdx.x == kFusedDrainWarp0 * 32) {
+        // accumulator += tile (rows past n fall outside the tensor map and are skipped)
+        tma_reduce_add_3d(&map_dqacc, dqs, 0, i0, bh);
+        bulk_commit();
+      }
       if (dpart != nullptr) {
         // band torque g1 x0 - g0 x1 of band c/2 for the queries of this lane's parity
         const uint8_t* qtile = base + C::OFF_ST + s * C::STAGE + pair_chunk;
@@ -1064,6 +1080,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[FB_Q_EMPTY + s]);
     }
+    // the last reductions complete (and stop reading shared memory) before the CTA exits
+    if (threadIdx.x == kFusedDrainWarp0 * 32) bulk_wait();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[FB_DRAIN_DONE]);
     if (dpart != nullptr) {
@@ -1233,7 +1251,7 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
 
 cudaError_t launch_fused_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
                            const float* deltap, const float2* table, const uint32_t* stats,
-                           void* dk, void* dv, float* dqacc, float* dpart, const DevCtl& ctl,
+                           void* dk, void* dv, float* dpart, const DevCtl& ctl,
                            cudaStream_t s) {
   using C = FusedCfg<128>;
   cudaError_t e = cudaFuncSetAttribute(bwd_fused_kernel<128>,
@@ -1243,7 +1261,7 @@ cudaError_t launch_fused_d(const ra_problem& p, const Sm100Maps& maps, const flo
   const long long ntk = (p.n + C::BN - 1) / C::BN;
   bwd_fused_kernel<128><<<(unsigned)(ntk * BH), kFusedThreads, C::SMEM, s>>>(
       maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, stats, (__nv_bfloat16*)dk,
-      (__nv_bfloat16*)dv, dqacc, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
+      (__nv_bfloat16*)dv, maps.dqacc, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
   return cudaGetLastError();
 }
 
@@ -1281,10 +1299,10 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,
                                    const float* lse2p, const float* deltap, const float2* table,
-                                   const uint32_t* stats, void* dk, void* dv, float* dqacc,
-                                   float* dpart, const DevCtl& ctl, cudaStream_t s) {
+                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
+                                   const DevCtl& ctl, cudaStream_t s) {
   if (p.d != 128) return cudaErrorInvalidValue;
-  return launch_fused_d(p, maps, lse2p, deltap, table, stats, dk, dv, dqacc, dpart, ctl, s);
+  return launch_fused_d(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
 }
 
 cudaError_t launch_dq_finish(const ra_problem& p, const float* dqacc, const float2* table,

@@ -55,13 +55,10 @@ cudaError_t launch_bwd_dkdv_f32(const ra_problem& p, const float* qt, const floa
 struct Sm100Maps {
   CUtensorMap qt, kt, v, dO;         // boxes of 64 columns x 128 rows
   CUtensorMap qt64, kt64, v64, dO64; // boxes of 64 columns x 64 rows
+  CUtensorMap dqacc;                 // fp32 [BH][n][d], box d x 64 rows, no swizzle (fused)
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
-// The same forward with each 128-key S tile handled as two 64-column halves on their own
-// barriers (fwd_split_sm100.cu); chosen per call by RA_FWD_SPLIT_S=1, off by default.
-cudaError_t launch_fwd_split_sm100(const ra_problem& p, const Sm100Maps& maps, void* o,
-                                   float* lse, const DevCtl& ctl, cudaStream_t s);
 // Padded per-row vectors for the tensor-core backward, delta and lse * log2(e), plus
 // max_i |dO_i| into stats[0] and max_j |v_j| into stats[1] (fp32 bits, atomic max; stats
 // zeroed by the caller), in one pass over O, dO and V.
@@ -73,12 +70,12 @@ cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,
                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
                                   const DevCtl& ctl, cudaStream_t s);
-// Fused dK, dV and dQ~ (into the fp32 accumulator dqacc, zeroed by the caller) in one pass
-// (d = 128); dq_finish turns the accumulator into dQ.
+// Fused dK, dV and dQ~ (added into the fp32 accumulator behind maps.dqacc, zeroed by the
+// caller) in one pass (d = 128); dq_finish turns the accumulator into dQ.
 cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,
                                    const float* lse2p, const float* deltap, const float2* table,
-                                   const uint32_t* stats, void* dk, void* dv, float* dqacc,
-                                   float* dpart, const DevCtl& ctl, cudaStream_t s);
+                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
+                                   const DevCtl& ctl, cudaStream_t s);
 cudaError_t launch_dq_finish(const ra_problem& p, const float* dqacc, const float2* table,
                              const uint32_t* stats, void* dq, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,

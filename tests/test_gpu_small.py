@@ -38,7 +38,7 @@ def test_bf16_fwd(n, d, causal):
 def test_bf16_fwd_bwd(n, d, causal):
     wl = small_workload(1, 2, n, d, "bf16", causal, seed=3 * n + d)
     inp = make(wl)
-    compare(gpu_run(inp), oracle_run(inp), "bf16", small=True, label=wl.name)
+    compare(gpu_run(inp), oracle_run(inp), "bf16", label=wl.name)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -111,7 +111,7 @@ def test_bwd_saved_matches_bwd(dtype, causal):
 def test_bf16_many_heads_and_batches():
     wl = small_workload(3, 5, 160, 64, "bf16", True, seed=5)
     inp = make(wl)
-    compare(gpu_run(inp), oracle_run(inp), "bf16", small=True, label=wl.name)
+    compare(gpu_run(inp), oracle_run(inp), "bf16", label=wl.name)
 
 
 def test_bf16_large_entries():
@@ -120,7 +120,7 @@ def test_bf16_large_entries():
     wl = small_workload(1, 2, 300, 128, "bf16", False, base=5e5, seed=4, qkve="uniform")
     wl = wl.with_(lo=-3.0, hi=3.0)
     inp = make(wl)
-    compare(gpu_run(inp), oracle_run(inp), "bf16", small=True, label=wl.name)
+    compare(gpu_run(inp), oracle_run(inp), "bf16", label=wl.name)
 
 
 def test_bf16_spread_frequencies():
@@ -128,7 +128,7 @@ def test_bf16_spread_frequencies():
     wl = small_workload(1, 2, 256, 128, "bf16", True, base=5e5, seed=6)
     wl = wl.with_(alpha="uniform", alpha_a=float(np.log(1e-3)), alpha_b=float(np.log(4.0)))
     inp = make(wl)
-    compare(gpu_run(inp), oracle_run(inp), "bf16", small=True, label=wl.name)
+    compare(gpu_run(inp), oracle_run(inp), "bf16", label=wl.name)
 
 
 def test_guard_bands_untouched():

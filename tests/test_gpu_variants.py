@@ -21,7 +21,7 @@ def test_fixed_bands_match_oracle(dtype, d, causal):
     inp = make(wl)
     f = d // 8  # a quarter of the d/2 bands
     g = gpu_run(inp, fixed_bands=f)
-    compare(g, oracle_run(inp, fixed_bands=f), dtype, small=True)
+    compare(g, oracle_run(inp, fixed_bands=f), dtype)
     assert np.all(g["dalpha"][d // 2 - f:] == 0.0)
 
 

@@ -102,8 +102,14 @@ typedef struct {
  * [B, H, n, d] dQ accumulator. */
 size_t rope_attn_workspace_bytes(const ra_problem* p);
 
+/* Bytes of workspace rope_attn_fwd alone needs (a prefix of the full layout: error word,
+ * loss partials, table, Q~, K~); 0 if *p is invalid. */
+size_t rope_attn_fwd_workspace_bytes(const ra_problem* p);
+
 /* Forward: o = softmax(Q~ K~^T / sqrt(d)) V and lse (natural log) from q, k, v
- * and alpha.  Overwrites the table, Q~ and K~ regions of ws. */
+ * and alpha.  ws needs at least rope_attn_fwd_workspace_bytes(p) bytes (a workspace of
+ * rope_attn_workspace_bytes(p) bytes serves every call).  Overwrites the table, Q~ and K~
+ * regions of ws. */
 ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const void* v,
                         const float* alpha, void* o, float* lse,
                         void* ws, size_t ws_bytes, void* stream);
@@ -230,7 +236,7 @@ const char* rope_attn_status_string(ra_status s);
  * RA_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads the
  * library holds until the process exits.  The call itself allocates nothing: no
  * cudaMalloc, no cudaFree, no allocating library routine.
- *   - Limit: a problem with rope_attn_workspace_bytes(p) > RA_NOALLOC_SCRATCH_BYTES
+ *   - Limit: a problem with rope_attn_fwd_workspace_bytes(p) > RA_NOALLOC_SCRATCH_BYTES
  *     (e.g. more than about 1.9M elements per [B,H,n,d] tensor in bf16) is rejected
  *     with RA_ERR_UNSUPPORTED before anything is launched.
  *   - Set-up: the first call on each device looks up the array's device address

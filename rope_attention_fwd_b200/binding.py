@@ -52,6 +52,8 @@ def lib():
         P, vp, sz = ctypes.POINTER(RaProblem), ctypes.c_void_p, ctypes.c_size_t
         L.rope_attn_workspace_bytes.argtypes = [P]
         L.rope_attn_workspace_bytes.restype = sz
+        L.rope_attn_fwd_workspace_bytes.argtypes = [P]
+        L.rope_attn_fwd_workspace_bytes.restype = sz
         L.rope_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.rope_attn_fwd.restype = ctypes.c_int
         L.rope_attn_loss.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]

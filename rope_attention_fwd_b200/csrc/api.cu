@@ -86,9 +86,12 @@ ra_status check_problem(const ra_problem* p) {
   return RA_OK;
 }
 
-ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes) {
+// fwd_only: the forward needs only the leading regions of the layout (error word, loss
+// partials, table, Q~, K~), so a smaller workspace is enough for it.
+ra_status check_ws(const ra_problem* p, void* ws, size_t ws_bytes, bool fwd_only = false) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) % 256) != 0) return RA_ERR_WORKSPACE;
-  if (ws_bytes < ws_layout(*p).total) return RA_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*p);
+  if (ws_bytes < (fwd_only ? L.fwd_total : L.total)) return RA_ERR_WORKSPACE;
   return RA_OK;
 }
 
@@ -199,6 +202,11 @@ size_t rope_attn_workspace_bytes(const ra_problem* p) {
   return ws_layout(*p).total;
 }
 
+size_t rope_attn_fwd_workspace_bytes(const ra_problem* p) {
+  if (check_problem(p) != RA_OK) return 0;
+  return ws_layout(*p).fwd_total;
+}
+
 const char* rope_attn_status_string(ra_status s) {
   switch (s) {
     case RA_OK: return "ok";
@@ -220,7 +228,7 @@ ra_status rope_attn_fwd(const ra_problem* p, const void* q, const void* k, const
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(o) ||
       !aligned16(lse))
     return RA_ERR_INVALID_ARG;
-  if ((st = check_ws(p, ws, ws_bytes)) != RA_OK) return st;
+  if ((st = check_ws(p, ws, ws_bytes, true)) != RA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(*p);
   if ((st = prepare(p, q, k, alpha, ws, L, s)) != RA_OK) return st;

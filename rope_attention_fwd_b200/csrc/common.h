@@ -46,6 +46,7 @@ struct WsLayout {
   size_t dpart;      // float [2][B*H][ceil(n/kDalphaRows)][M]
   size_t dqacc;      // float [B*H][n][d]: dQ~ accumulator of the fused backward (bf16, d = 128)
   size_t total;
+  size_t fwd_total;  // the regions the forward touches (error word .. K~): a prefix of total
 };
 
 // The bf16 backward with d = 128 runs the fused dK/dV/dQ kernel (an fp32 dQ~ accumulator in
@@ -74,6 +75,7 @@ inline WsLayout ws_layout(const ra_problem& p) {
   w.table = take(sizeof(float) * 2 * n * M);
   w.qt = take(elem * BH * n * d);
   w.kt = take(elem * BH * n * d);
+  w.fwd_total = off;
   const size_t npad = (size_t)padded_rows(p.n);
   w.delta = take(sizeof(float) * BH * npad);
   w.lse2 = take(sizeof(float) * BH * npad);

@@ -50,7 +50,7 @@ cudaError_t noalloc_scratch(void** out) {
 extern "C" ra_status rope_attn_fwd_noalloc(const ra_problem* p, const void* q, const void* k,
                                            const void* v, const float* alpha, void* o,
                                            float* lse, void* stream) {
-  const size_t need = rope_attn_workspace_bytes(p);
+  const size_t need = rope_attn_fwd_workspace_bytes(p);
   // An invalid or unsupported problem: let the regular validation name the error
   // (it returns before launching anything, and before it looks at the workspace).
   if (need == 0) return rope_attn_fwd(p, q, k, v, alpha, o, lse, nullptr, 0, stream);

@@ -90,10 +90,13 @@ def test_null_pointers_rejected_before_launch():
 
 
 def test_workspace_checks_before_launch():
+    """The forward needs the leading part of the layout (rope_attn_fwd_workspace_bytes);
+    one byte less, a misaligned or a null workspace is rejected before any launch."""
     lib = rb.lib()
     p = rb.problem(1, 1, 16, 64, rb.RA_F32, False, 1e4)
     fake = ctypes.c_void_p(4096)
-    need = rb.rope_attn_workspace_bytes(p)
+    need = rb.lib().rope_attn_fwd_workspace_bytes(ctypes.byref(p))
+    assert 0 < need <= rb.rope_attn_workspace_bytes(p)
     assert lib.rope_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake,
                              need - 1, None) == 3
     assert lib.rope_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake,

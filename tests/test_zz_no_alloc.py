@@ -45,7 +45,7 @@ def test_noalloc_matches_workspace_forward_on_two_calls():
         inp = make(wl)
         q, k, v, alpha = (getattr(inp, x).cuda() for x in ("q", "k", "v", "alpha"))
         prob = rb.problem(wl.B, wl.H, wl.n, wl.d, q.dtype, wl.causal, wl.base)
-        assert rb.rope_attn_workspace_bytes(prob) <= (8 << 20)
+        assert rb.lib().rope_attn_fwd_workspace_bytes(ctypes.byref(prob)) <= (8 << 20)
         o_ref, lse_ref = rb.rope_attn_fwd(q, k, v, alpha, wl.base, wl.causal)
         o = torch.full_like(q, float("nan"))
         lse = torch.full((wl.B, wl.H, wl.n), float("nan"), device="cuda")
@@ -77,7 +77,7 @@ def test_noalloc_reports_range_overflow():
 
 def test_noalloc_rejects_problems_beyond_the_scratch():
     prob = rb.problem(2, 32, 8192, 128, torch.bfloat16, True, 1e4)
-    assert rb.rope_attn_workspace_bytes(prob) > (8 << 20)
+    assert rb.lib().rope_attn_fwd_workspace_bytes(ctypes.byref(prob)) > (8 << 20)
     null = ctypes.c_void_p(0)
     r = rb.lib().rope_attn_fwd_noalloc(ctypes.byref(prob), null, null, null, null, null, null,
                                        null)

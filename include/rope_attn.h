@@ -83,22 +83,23 @@ typedef struct {
                             rotated (theta_hat_m = 0, dalpha_m = 0): partial RoPE, the
                             p-RoPE baseline of "LeRoPE" (Configuracao Experimental) with
                             p = 1 - fixed_bands / (d/2); 0 = every band rotates        */
-    int32_t flags;       /* 0 or RA_FLAG_DETERMINISTIC                           */
+    int32_t flags;       /* 0 or RA_FLAG_FUSED_BWD                               */
 } ra_problem;
 
-/* ra_problem.flags: the bf16 backward with d = 128 adds the dQ contribution of every
- * 128-key block into an fp32 accumulator in ws as soon as it is formed (one pass over the
- * key/query tile pairs), so dQ depends on the order in which blocks add (the last bits of
- * fp32 sums; in bf16, a one-unit difference in a rare element).  dK, dV and dalpha stay
- * bitwise reproducible.  RA_FLAG_DETERMINISTIC selects the two-pass backward instead
- * (dK/dV, then dQ recomputing the scores), bitwise reproducible in every output, at about
- * 1.4x the backward time.  Other d, and fp32 problems, always take the two-pass form. */
-#define RA_FLAG_DETERMINISTIC 1
+/* ra_problem.flags: by default the backward takes two passes (dK/dV with keys stationary,
+ * then dQ with queries stationary recomputing the scores), every output bitwise
+ * reproducible.  RA_FLAG_FUSED_BWD (bf16, d = 128) selects one pass instead: each 128-key
+ * block adds its dQ contribution into an fp32 accumulator in ws as soon as it is formed, so
+ * dQ depends on the order in which blocks add (the last bits of fp32 sums; in bf16, a
+ * one-unit difference in a rare element); dK, dV and dalpha stay bitwise reproducible.
+ * On a B200 the one pass is the slower of the two at the headline size (its fp32
+ * reductions into L2 bound it); other d, and fp32 problems, always take two passes. */
+#define RA_FLAG_FUSED_BWD 1
 
 /* Bytes of workspace the calls below need for problem *p (0 if *p is invalid).
  * Holds: the fp32 cos/sin table [n, d/2, 2], the rotated Q~ and K~ in the
  * problem dtype, rowsum(dO o O) [B, H, n] fp32, per-tile dalpha partials,
- * loss partials, the device error word and (fused bf16 backward, d = 128) an fp32
+ * loss partials, the device error word and (with RA_FLAG_FUSED_BWD) an fp32
  * [B, H, n, d] dQ accumulator. */
 size_t rope_attn_workspace_bytes(const ra_problem* p);
 
@@ -122,7 +123,7 @@ ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e,
 /* Backward: dq, dk, dv ([B,H,n,d], dtype) and dalpha ([d/2], fp32, summed over
  * every batch and head) from q, k, v, the forward's o and lse, the upstream
  * gradient dO and alpha.  dk, dv and dalpha are reduced in a fixed order (bitwise
- * reproducible); dq too unless the fused form is taken (see ra_problem.flags).
+ * reproducible); dq too unless the one-pass form is asked for (see ra_problem.flags).
  * Recomputes the table, Q~ and K~ in ws (it does not rely on a previous fwd). */
 ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
                         const void* o, const float* lse, const void* dO, const float* alpha,

@@ -79,7 +79,7 @@ ra_status check_problem(const ra_problem* p) {
   if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
   if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
   if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 ||
-      (p->flags & ~RA_FLAG_DETERMINISTIC) != 0)
+      (p->flags & ~RA_FLAG_FUSED_BWD) != 0)
     return RA_ERR_INVALID_ARG;
   if (p->d > 128) return RA_ERR_UNSUPPORTED;
   if (p->dtype == RA_BF16 && p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
@@ -330,8 +330,8 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
                                        s));
       RA_LAUNCH(K_DQ_FINISH, s, launch_dq_finish(*p, dqacc, table, stats, dq, s));
     } else {
-      // two passes: dK, dV (keys stationary), then dQ (queries stationary, S and dP
-      // recomputed); every output bitwise reproducible
+      // two passes (the default): dK, dV (keys stationary), then dQ (queries stationary, S
+      // and dP recomputed); every output bitwise reproducible
       RA_LAUNCH(K_BWD_DKDV_SM100, s,
                 launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
                                       s));

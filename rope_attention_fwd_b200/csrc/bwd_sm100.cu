@@ -28,11 +28,11 @@
 // 3.8e-3 this way.
 //
 // Two forms:
-//   fused (bf16, d = 128; the default): one kernel, 128 keys stationary per CTA, queries
+//   fused (bf16, d = 128, RA_FLAG_FUSED_BWD): one kernel, 128 keys stationary per CTA, queries
 //         streamed 64 at a time; per step S^T, dP^T, then dV += P^T dO_i, dK~ += dS^T Q~_i
 //         (TMEM accumulators) and dQ~^T = K~^T dS^T, whose partial is added into an fp32
 //         accumulator in global memory; dq_finish_kernel rotates the sum back.
-//   two-pass (d = 64, or RA_FLAG_DETERMINISTIC): no atomics, every output reproducible
+//   two-pass (the default): no atomics, every output reproducible
 //     dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
 //           time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
 //           (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T

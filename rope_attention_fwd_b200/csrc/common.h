@@ -49,10 +49,10 @@ struct WsLayout {
   size_t fwd_total;  // the regions the forward touches (error word .. K~): a prefix of total
 };
 
-// The bf16 backward with d = 128 runs the fused dK/dV/dQ kernel (an fp32 dQ~ accumulator in
-// the workspace) unless the caller asks for bitwise-reproducible dQ (RA_FLAG_DETERMINISTIC).
+// The one-pass backward (fused dK/dV/dQ kernel, an fp32 dQ~ accumulator in the workspace):
+// bf16 with d = 128 when the caller asks for it (RA_FLAG_FUSED_BWD).
 inline bool uses_fused_bwd(const ra_problem& p) {
-  return p.dtype == RA_BF16 && p.d == 128 && (p.flags & RA_FLAG_DETERMINISTIC) == 0;
+  return p.dtype == RA_BF16 && p.d == 128 && (p.flags & RA_FLAG_FUSED_BWD) != 0;
 }
 
 // Rows of the padded per-row vectors (a whole number of 128-row tiles).

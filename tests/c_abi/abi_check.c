@@ -38,8 +38,8 @@ int main(void) {
   bad = p;
   bad.flags = 2;
   expect(rope_attn_workspace_bytes(&bad) == 0, "unknown flag bits are rejected");
-  bad.flags = RA_FLAG_DETERMINISTIC;
-  expect(rope_attn_workspace_bytes(&bad) > 0, "the deterministic flag is accepted");
+  bad.flags = RA_FLAG_FUSED_BWD;
+  expect(rope_attn_workspace_bytes(&bad) > 0, "the one-pass backward flag is accepted");
 
   expect(strcmp(rope_attn_status_string(RA_OK), "ok") == 0, "status string of RA_OK");
   expect(rope_attn_status_string(RA_ERR_TIMEOUT) != NULL, "status string of RA_ERR_TIMEOUT");

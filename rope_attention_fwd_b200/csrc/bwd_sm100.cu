@@ -272,8 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * KB_COUNT + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int jt = (int)(blockIdx.x / BH);  // key tile; low tiles carry most causal work
-  const int bh = (int)(blockIdx.x % BH);
+  // head-major grid: the CTAs resident at one time share a few heads' Q~ / dO stream in L2;
+  // key tile 0 (the most causal work) first within a head
+  const int ntk_grid = (n + C::BN - 1) / C::BN;
+  const int jt = (int)(blockIdx.x % ntk_grid);
+  const int bh = (int)(blockIdx.x / ntk_grid);
   const int npad = (int)((n + 127) / 128 * 128);
   const int qstart = causal ? jt * C::BN : 0;
   const int nq = (n - qstart + C::BQ - 1) / C::BQ;
@@ -568,8 +571,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
-  const int qtile = ntq - 1 - (int)(blockIdx.x / BH);  // heaviest causal tiles first
-  const int bh = (int)(blockIdx.x % BH);
+  // head-major grid (the resident CTAs share a few heads' K~ / V stream in L2), heaviest
+  // causal tiles first within a head
+  const int qtile = ntq - 1 - (int)(blockIdx.x % ntq);
+  const int bh = (int)(blockIdx.x / ntq);
   const int npad = (int)((n + 127) / 128 * 128);
   const int kend = causal ? min(n, (qtile + 1) * C::BM) : n;
   const int nk = (kend + C::BK - 1) / C::BK;
@@ -892,8 +897,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * FB_COUNT + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int jt = (int)(blockIdx.x / BH);  // key tile; low tiles carry most causal work
-  const int bh = (int)(blockIdx.x % BH);
+  // head-major grid: the CTAs resident at one time share a few heads' Q~ / dO stream in L2;
+  // key tile 0 (the most causal work) first within a head
+  const int ntk_grid = (n + C::BN - 1) / C::BN;
+  const int jt = (int)(blockIdx.x % ntk_grid);
+  const int bh = (int)(blockIdx.x / ntk_grid);
   const int npad = (int)((n + 127) / 128 * 128);
   const int qstart = causal ? jt * C::BN : 0;
   const int nq = (n - qstart + C::BQ - 1) / C::BQ;

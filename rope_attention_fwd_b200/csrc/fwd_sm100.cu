@@ -118,8 +118,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
   const int ntp = (ntq + 1) / 2;
-  const int T = ntp - 1 - (int)(blockIdx.x / BH);  // heaviest causal tile pairs first
-  const int bh = (int)(blockIdx.x % BH);
+  // head-major grid: the CTAs resident at one time share a few heads' K~ / V stream in L2
+  // (all heads at once do not fit); heaviest causal tile pairs first within a head
+  const int T = ntp - 1 - (int)(blockIdx.x % ntp);
+  const int bh = (int)(blockIdx.x / ntp);
   const int ntk = (n + C::BN - 1) / C::BN;
   // key tiles of query tile x (0 when the tile lies past the end of the sequence)
   auto nkv_of = [&](int x) -> int {

@@ -401,7 +401,8 @@ def run_profile(args):
     q, k, v, e = (torch.randn(shape, device="cuda", generator=g).to(torch.bfloat16)
                   for _ in range(4))
     alpha = 0.3 * torch.randn(d // 2, device="cuda", generator=g)
-    ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base), "cuda")
+    ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base,
+                                 fused=args.fused), "cuda")
     proj_ms = {"proj_fwd": 0.0, "proj_bwd": 0.0}
     if args.d_model > 0:
         x = torch.randn((B, n, args.d_model), device="cuda", generator=g).to(torch.bfloat16)
@@ -422,7 +423,8 @@ def run_profile(args):
             "proj_fwd", lambda: rb.rope_attn_proj_fwd(x, *w, H))
         o, lse = rb.rope_attn_fwd(qq, kk, vv, alpha, args.base, args.causal, ws=ws)
         L, dO = rb.rope_attn_loss(o, e, ws=ws)
-        grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws)
+        grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws,
+                                       fused=args.fused)
         if args.d_model > 0:
             timed("proj_bwd", lambda: rb.rope_attn_proj_bwd(x, *w, *grads[:3]))
         return grads
@@ -474,6 +476,8 @@ def main():
     ap.add_argument("--base", type=float, default=1e4, help="RoPE base in --profile")
     ap.add_argument("--d-model", type=int, default=0,
                     help="--profile: also run the projections with this model width")
+    ap.add_argument("--fused", action="store_true",
+                    help="--profile: the one-pass backward (RA_FLAG_FUSED_BWD)")
     args = ap.parse_args()
     if args.profile:
         return run_profile(args)

@@ -14,12 +14,18 @@
 // tile per CTA on 2 x 32 x 8192 x 128) runs into the on-chip L2 -> SM bandwidth before
 // the tensor cores are busy.  With 256 rows per CTA the traffic halves.
 //
-// CTA = 10 warps, query tiles a = 2T, b = 2T + 1, 1 CTA per SM:
-//   warps 0-3 / 4-7  softmax of tile a / b: thread t owns row t (TMEM lane t) of S and O
-//   warp  8          TMA producer: Q~_a, Q~_b once, then K~_j (3-stage ring), V_j (2 stages)
-//   warp  9          TMEM allocator + tcgen05.mma issuer (converged warp, one elected lane)
-// TMEM (512 columns): S_x at 128 x with P_x (bf16, two per column) written over its first
-// 64 columns, O_x at 256 + 128 x.  One S buffer per tile: the MMAs alternate between the
+// CTA = 18 warps, query tiles a = 2T, b = 2T + 1, 1 CTA per SM:
+//   warps 0-7 / 8-15   softmax of tile a / b, two warpgroups per tile: warpgroup h takes the
+//                      score columns 64h .. 64h + 63 of every row, thread t row t (TMEM lane
+//                      t); the pair exchanges its partial row maxima (and, at the end, row
+//                      sums) through two TMEM columns and a bounded-wait barrier
+//   warp  16           TMA producer: Q~_a, Q~_b once, then K~_j (3-stage ring), V_j (2 stages)
+//   warp  17           TMEM allocator + tcgen05.mma issuer (converged warp, one elected lane)
+// Splitting each row over two warpgroups halves the softmax latency that sits between a
+// tile's S and P V MMAs.
+// TMEM (512 columns): S_x at 128 x; warpgroup h writes P_x (bf16, two per column) for its 64
+// keys over S columns 64h .. 64h + 31, which it has itself read, and the P V MMA reads them
+// as two halves; O_x at 256 + 128 x.  One S buffer per tile: the MMAs alternate between the
 // tiles, S_a(j+1) running on the tensor core while the softmax of tile b turns S_b(j) into
 // P_b(j) and the reverse, in the issue order
 //   S_a(0) S_b(0) | PV_a(0) S_a(1) PV_b(0) S_b(1) | PV_a(1) S_a(2) PV_b(1) S_b(2) | ...
@@ -69,33 +75,34 @@ enum FwdBar {
   B_V_FULL = 7,               // +stage (2)
   B_V_EMPTY = 9,              // +stage (2)
   B_S_FULL = 11,              // +tile: S_x(j) computed
-  B_P_FULL = 13,              // +tile: P_x(j) written (and O_x rescaled); 4 warp arrivals
+  B_P_FULL = 13,              // +tile: P_x(j) written (and O_x rescaled); 8 warp arrivals
   B_PV_DONE = 15,             // +tile: O_x += P_x(j) V_j has completed
   B_O_DONE = 17,
   B_DRAIN = 18,
-  B_COUNT = 19
+  B_XCH = 19,                 // +tile: both warpgroups have written their partial row max
+                              // (or, after the loop, row sum); 8 warp arrivals
+  B_COUNT = 21
 };
 
-#ifndef RA_FWD_RESCALE_TAU
-#define RA_FWD_RESCALE_TAU 8.0f
-#endif
-#ifndef RA_MMA_BATCH
-#define RA_MMA_BATCH 1
-#endif
-#ifndef RA_FWD_POLY_EVERY
-#define RA_FWD_POLY_EVERY 0
-#endif
-constexpr float kRescaleTau = RA_FWD_RESCALE_TAU;
-constexpr int kFwdThreads = 320;
-constexpr int kFwdProdWarp = 8, kFwdMmaWarp = 9;
+constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold, log2 units
+// 16 softmax warps: two warpgroups per query tile, warpgroup h of a tile taking its score
+// columns 64h .. 64h + 63 of every row; then the TMA warp and the MMA warp.
+constexpr int kFwdThreads = 576;
+constexpr int kFwdProdWarp = 16, kFwdMmaWarp = 17;
 
-// 2^x of column c: every RA_FWD_POLY_EVERY-th column on the FMA pipe (exp2_poly), the
-// others on MUFU, to split the exponential load off the XU pipe.
-__device__ __forceinline__ float exp2_col(float x, int c) {
-#if RA_FWD_POLY_EVERY > 0
-  if (c % RA_FWD_POLY_EVERY == RA_FWD_POLY_EVERY - 1) return exp2_poly(x);
-#endif
-  return fast_exp2(x);
+// One 32-bit TMEM column of this thread's lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, const uint32_t (&r)[1]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0])
+               : "memory");
+}
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(v)
+               : "r"(taddr)
+               : "memory");
+  return v;
 }
 
 template <int D>
@@ -118,8 +125,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
   const int ntp = (ntq + 1) / 2;
-  // head-major grid: the CTAs resident at one time share a few heads' K~ / V stream in L2
-  // (all heads at once do not fit); heaviest causal tile pairs first within a head
   const int T = ntp - 1 - (int)(blockIdx.x % ntp);
   const int bh = (int)(blockIdx.x / ntp);
   const int ntk = (n + C::BN - 1) / C::BN;
@@ -135,7 +140,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i)
-      mbar_init(&bar[i], (i == B_P_FULL || i == B_P_FULL + 1) ? 4 : 1);
+      mbar_init(&bar[i],
+                (i == B_P_FULL || i == B_P_FULL + 1 || i == B_XCH || i == B_XCH + 1) ? 8 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -214,7 +220,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     auto issue_s = [&](int x, int j) {
       const SDesc ks = sdesc_advance(dkm, C::OFF_K + (j % C::NSK) * C::TILE);
       const uint32_t q_off = C::OFF_Q + x * C::TILE;
-      if constexpr (D == 128 && RA_MMA_BATCH) {
+      if constexpr (D == 128) {
         mma8_kmajor<false, C::CHUNK, C::CHUNK>(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off),
                                                sdesc_at(ks, 0), idS, 0);
       } else {
@@ -255,13 +261,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         // O_x += P_x(j) V_j with P_x(j) read from TMEM buffer x
         const SDesc vs = sdesc_advance(dmn, C::OFF_V + (j % C::NSV) * C::TILE);
-        if constexpr (C::BN == 128 && RA_MMA_BATCH) {
-          mma8_ts_mn(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128, sdesc_at(vs, 0), idO,
-                     j > 0);
+        if constexpr (C::BN == 128) {
+          // P of keys 0..63 sits in S columns 0..31 (warpgroup 0), of keys 64..127 in 64..95
+          mma4_ts_mn<8, 16, 24>(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128,
+                                sdesc_at(vs, 0), idO, j > 0);
+          mma4_ts_mn<8, 16, 24>(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128 + 64,
+                                sdesc_at(vs, 4 * 2048), idO, 1);
         } else {
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk)
-            mma_ts_warp(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128 + kk * 8,
+            mma_ts_warp(tmem + C::COL_O + x * 128, tmem + C::COL_S + x * 128 + (kk / 4) * 64 +
+                            (kk % 4) * 8,
                         sdesc_at(vs, kk * 2048), idO, (j > 0 || kk > 0));
         }
         mma_commit_warp(&bar[B_PV_DONE + x]);
@@ -278,7 +288,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_wait_warp(&bar[B_DRAIN], 0, &dummy, err, KID, 23, wait_ns);
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int x = warp / 4;            // query tile a (0) or b (1)
+    const int x = warp / 8;            // query tile a (0) or b (1)
+    const int h = (warp / 4) % 2;      // column half: S columns 64h .. 64h + 63
     const int t = threadIdx.x % 128;   // row within the tile == TMEM lane
     const int qt = 2 * T + x;
     const int row = qt * C::BM + t;
@@ -286,8 +297,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     const uint32_t s_base = lane_base + C::COL_S + x * 128;
     const uint32_t o_base = lane_base + C::COL_O + x * 128;
+    // exchange columns: each warpgroup writes its partial row max / sum into a column of its
+    // own S half that it has already read, and reads the other's
+    const uint32_t x_mine = s_base + 64 * h + 32, x_other = s_base + 64 * (1 - h) + 32;
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    float m = -CUDART_INF_F, l = 0.f;  // running max (log2 units, scaled) and row sum
+    float m = -CUDART_INF_F, l = 0.f;  // running max (log2 units, scaled), this half's sum
     bool ok = true;
     for (int j = 0; j < my_nkv; ++j) {
       if (!mbar_wait_warp(&bar[B_S_FULL + x], j & 1, abort_flag, err, KID, 8, wait_ns)) {
@@ -295,35 +309,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         break;
       }
       tc_fence_after();
-      const int key0 = j * C::BN;
-      // columns of this row that hold a key (all of them except on the diagonal tile and
-      // the ragged last tile)
-      const bool need_mask = (key0 + C::BN > n) || (causal && j == qt);
+      const int key0 = j * C::BN + 64 * h;
+      const bool need_mask = (j * C::BN + C::BN > n) || (causal && j == qt);
       const int nvalid =
-          need_mask ? max(0, min(C::BN, (causal ? min(n, row + 1) : n) - key0)) : C::BN;
-      // the whole row of S in registers (one TMEM read; S_x is free again once P_x is
-      // written over it)
-      uint32_t sr[4][32];
+          need_mask ? max(0, min(64, (causal ? min(n, row + 1) : n) - key0)) : 64;
+      // this half of the row of S in registers (two TMEM reads)
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(s_base + 32 * c, sr[c]);
+      for (int c = 0; c < 2; ++c) tmem_ld32(s_base + 64 * h + 32 * c, sr[c]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_wait_ld(sr[c]);
+      for (int c = 0; c < 2; ++c) tmem_wait_ld(sr[c]);
       if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= nvalid) sr[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // the row max of the raw scores (masked entries are -inf)
       float mp[8];
 #pragma unroll
       for (int a = 0; a < 8; ++a) mp[a] = __uint_as_float(sr[0][a]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
-      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7]))) * scale_log2;
-      // lazy rescale: move the reference max only when some row of the warp needs it
+      for (int i = 8; i < 64; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
+      float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      // the row max over both halves, through TMEM columns and the tile's exchange barrier
+      // (phase j; a bounded wait, like every other)
+      {
+        uint32_t w1[1] = {__float_as_uint(mh)};
+        tmem_st1(x_mine, w1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_XCH + x]);
+        if (!mbar_wait_warp(&bar[B_XCH + x], j & 1, abort_flag, err, KID, 12, wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t o1 = tmem_ld1(x_other);
+        mh = fmaxf(mh, __uint_as_float(o1));
+      }
+      const float mt = mh * scale_log2;
+      // lazy rescale: move the reference max only when some row of the warp needs it (both
+      // warpgroups of a tile see the same row maxima, so they decide alike)
       const bool need = mt > m + kRescaleTau;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
       float corr = 1.f;
@@ -333,15 +362,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m = m_new;
       }
       const float m_use = m == -CUDART_INF_F ? 0.f : m;
-      // P = 2^(s scale - m), summed and written as bf16 over S: chunk c (columns
-      // 32c..32c+31) lands in columns 16c..16c+15 (masked entries give 2^-inf = 0)
+      // P = 2^(s scale - m), summed and written as bf16 pairs: columns 64h + 32c .. + 31 land
+      // in S columns 64h + 16c .. + 15 (masked entries give 2^-inf = 0)
       float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float pv[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          pv[i] = exp2_col(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_use), 32 * c + i);
+          pv[i] = fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_use));
         if (need_mask) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -352,12 +381,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < 32; ++i) sp[i & 7] += pv[i];
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) w[i2] = pack_bf16x2(pv[2 * i2], pv[2 * i2 + 1]);
-        tmem_st16(s_base + 16 * c, w);
+        tmem_st16(s_base + 64 * h + 16 * c, w);
       }
       l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
       tmem_wait_st();
       if (warp_rescale && j > 0) {
-        // O_x must hold every P_x(j') V_j' with j' < j: wait for the PV MMA of step j-1
+        // O_x must hold every P_x(j') V_j' with j' < j: wait for the PV MMA of step j-1;
+        // this warpgroup rescales its half of the O columns
         if (!mbar_wait_warp(&bar[B_PV_DONE + x], (j - 1) & 1, abort_flag, err, KID, 11,
                             wait_ns)) {
           ok = false;
@@ -365,13 +395,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
-          tmem_ld32(o_base + 32 * c, r);
+          tmem_ld32(o_base + (D / 2) * h + 32 * c, r);
           tmem_wait_ld(r);
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-          tmem_st32(o_base + 32 * c, r);
+          tmem_st32(o_base + (D / 2) * h + 32 * c, r);
         }
         tmem_wait_st();
       }
@@ -382,14 +412,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (ok && my_nkv > 0 &&
         mbar_wait_warp(&bar[B_O_DONE], 0, abort_flag, err, KID, 10, wait_ns)) {
       tc_fence_after();
+      // the row sum over both halves (every MMA is done: the S columns are free); exchange
+      // phase my_nkv
+      bool have_l = true;
+      {
+        uint32_t w1[1] = {__float_as_uint(l)};
+        tmem_st1(x_mine, w1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_XCH + x]);
+        have_l = mbar_wait_warp(&bar[B_XCH + x], my_nkv & 1, abort_flag, err, KID, 13, wait_ns);
+        tc_fence_after();
+        if (have_l) l += __uint_as_float(tmem_ld1(x_other));
+      }
       const float inv = 1.f / l;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(o_base + 32 * c, r);
+        tmem_ld32(o_base + (D / 2) * h + 32 * c, r);
         tmem_wait_ld(r);
-        if (row < n) {
-          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * n + row) * D + 32 * c);
+        if (have_l && row < n) {
+          uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)bh * n + row) * D + (D / 2) * h +
+                                                32 * c);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const float* f = reinterpret_cast<const float*>(&r[8 * u]);
@@ -400,7 +445,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      if (row < n) lse[(size_t)bh * n + row] = (m + __log2f(l)) * 0.6931471805599453f;
+      if (have_l && row < n && h == 0)
+        lse[(size_t)bh * n + row] = (m + __log2f(l)) * 0.6931471805599453f;
     }
   }
 

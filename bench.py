@@ -287,8 +287,7 @@ def run_ours(args):
     peaks, peak_kind = load_peaks()
     f = 0.5 if wl.causal else 1.0
     # algorithmic FLOPs per (batch, head) in units of n^2 d (halved when causal)
-    alg = {"fwd_sm100": 4.0, "bwd_fused_sm100": 10.0, "bwd_dkdv_sm100": 8.0,
-           "bwd_dq_sm100": 2.0}
+    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0}
     per_kernel = {name: {"launches": c, "avg_ms": t / c, "share": t / sum(
         tt for _, tt in kernels.values())} for name, (c, t) in kernels.items()}
     dom = max(kernels, key=lambda k: kernels[k][1])
@@ -341,8 +340,8 @@ def run_ours(args):
 # Kernels of each phase (the step's backward takes the table and rotated Q~, K~ from the
 # forward, so those run in the forward only).
 FWD_KERNELS = {"rope_table": 1.0, "rotate": 1.0, "fwd_sm100": 1.0}
-BWD_KERNELS = {"bwd_delta": 1.0, "bwd_fused_sm100": 1.0, "dq_finish": 1.0,
-               "bwd_dkdv_sm100": 1.0, "bwd_dq_sm100": 1.0, "dalpha_final": 1.0}
+BWD_KERNELS = {"bwd_delta": 1.0, "bwd_dkdv_sm100": 1.0, "bwd_dq_sm100": 1.0,
+               "dalpha_final": 1.0}
 
 
 def phase_tflops(kernels, share, flops, steps):
@@ -401,8 +400,7 @@ def run_profile(args):
     q, k, v, e = (torch.randn(shape, device="cuda", generator=g).to(torch.bfloat16)
                   for _ in range(4))
     alpha = 0.3 * torch.randn(d // 2, device="cuda", generator=g)
-    ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base,
-                                 fused=args.fused), "cuda")
+    ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base), "cuda")
     proj_ms = {"proj_fwd": 0.0, "proj_bwd": 0.0}
     if args.d_model > 0:
         x = torch.randn((B, n, args.d_model), device="cuda", generator=g).to(torch.bfloat16)
@@ -423,8 +421,7 @@ def run_profile(args):
             "proj_fwd", lambda: rb.rope_attn_proj_fwd(x, *w, H))
         o, lse = rb.rope_attn_fwd(qq, kk, vv, alpha, args.base, args.causal, ws=ws)
         L, dO = rb.rope_attn_loss(o, e, ws=ws)
-        grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws,
-                                       fused=args.fused)
+        grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws)
         if args.d_model > 0:
             timed("proj_bwd", lambda: rb.rope_attn_proj_bwd(x, *w, *grads[:3]))
         return grads
@@ -440,7 +437,7 @@ def run_profile(args):
     torch.cuda.synchronize()
     rb.rope_attn_timing_enable(False)
     f = 0.5 if args.causal else 1.0
-    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0, "bwd_fused_sm100": 10.0}
+    alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0}
     for name, (cnt, ms) in rb.rope_attn_timing_read().items():
         line = f"{name:16s} {cnt:3d} launches {ms / cnt:8.3f} ms"
         if name in alg:
@@ -476,8 +473,6 @@ def main():
     ap.add_argument("--base", type=float, default=1e4, help="RoPE base in --profile")
     ap.add_argument("--d-model", type=int, default=0,
                     help="--profile: also run the projections with this model width")
-    ap.add_argument("--fused", action="store_true",
-                    help="--profile: the one-pass backward (RA_FLAG_FUSED_BWD)")
     args = ap.parse_args()
     if args.profile:
         return run_profile(args)

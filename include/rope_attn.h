@@ -83,24 +83,13 @@ typedef struct {
                             rotated (theta_hat_m = 0, dalpha_m = 0): partial RoPE, the
                             p-RoPE baseline of "LeRoPE" (Configuracao Experimental) with
                             p = 1 - fixed_bands / (d/2); 0 = every band rotates        */
-    int32_t flags;       /* 0 or RA_FLAG_FUSED_BWD                               */
+    int32_t reserved;    /* must be 0                                             */
 } ra_problem;
-
-/* ra_problem.flags: by default the backward takes two passes (dK/dV with keys stationary,
- * then dQ with queries stationary recomputing the scores), every output bitwise
- * reproducible.  RA_FLAG_FUSED_BWD (bf16, d = 128) selects one pass instead: each 128-key
- * block adds its dQ contribution into an fp32 accumulator in ws as soon as it is formed, so
- * dQ depends on the order in which blocks add (the last bits of fp32 sums; in bf16, a
- * one-unit difference in a rare element); dK, dV and dalpha stay bitwise reproducible.
- * On a B200 the one pass is the slower of the two at the headline size (its fp32
- * reductions into L2 bound it); other d, and fp32 problems, always take two passes. */
-#define RA_FLAG_FUSED_BWD 1
 
 /* Bytes of workspace the calls below need for problem *p (0 if *p is invalid).
  * Holds: the fp32 cos/sin table [n, d/2, 2], the rotated Q~ and K~ in the
  * problem dtype, rowsum(dO o O) [B, H, n] fp32, per-tile dalpha partials,
- * loss partials, the device error word and (with RA_FLAG_FUSED_BWD) an fp32
- * [B, H, n, d] dQ accumulator. */
+ * loss partials and the device error word. */
 size_t rope_attn_workspace_bytes(const ra_problem* p);
 
 /* Bytes of workspace rope_attn_fwd alone needs (a prefix of the full layout: error word,
@@ -122,8 +111,8 @@ ra_status rope_attn_loss(const ra_problem* p, const void* o, const void* e,
 
 /* Backward: dq, dk, dv ([B,H,n,d], dtype) and dalpha ([d/2], fp32, summed over
  * every batch and head) from q, k, v, the forward's o and lse, the upstream
- * gradient dO and alpha.  dk, dv and dalpha are reduced in a fixed order (bitwise
- * reproducible); dq too unless the one-pass form is asked for (see ra_problem.flags).
+ * gradient dO and alpha.  Deterministic: no atomics, fixed-order reductions (every output
+ * bitwise reproducible).
  * Recomputes the table, Q~ and K~ in ws (it does not rely on a previous fwd). */
 ra_status rope_attn_bwd(const ra_problem* p, const void* q, const void* k, const void* v,
                         const void* o, const float* lse, const void* dO, const float* alpha,

@@ -14,7 +14,6 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "librope_attn.so")
 
 RA_F32, RA_BF16 = 0, 1
-RA_FLAG_FUSED_BWD = 1
 _DTYPE = {torch.float32: RA_F32, torch.bfloat16: RA_BF16}
 STATUS = {0: "RA_OK", 1: "RA_ERR_INVALID_ARG", 2: "RA_ERR_UNSUPPORTED", 3: "RA_ERR_WORKSPACE",
           4: "RA_ERR_CUDA", 5: "RA_ERR_TIMEOUT", 6: "RA_ERR_RANGE"}
@@ -24,7 +23,7 @@ class RaProblem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("n", ctypes.c_int64),
                 ("d", ctypes.c_int64), ("dtype", ctypes.c_int32), ("causal", ctypes.c_int32),
                 ("base", ctypes.c_double), ("fixed_bands", ctypes.c_int32),
-                ("flags", ctypes.c_int32)]
+                ("reserved", ctypes.c_int32)]
 
 
 class RaAdam(ctypes.Structure):
@@ -94,18 +93,17 @@ def lib():
     return _lib
 
 
-def problem(B, H, n, d, dtype, causal, base, fixed_bands=0, fused=False):
-    """fixed_bands: the slowest bands left unrotated (partial RoPE; 0 = all rotate).
-    fused: the one-pass backward (RA_FLAG_FUSED_BWD; bf16, d = 128)."""
+def problem(B, H, n, d, dtype, causal, base, fixed_bands=0):
+    """fixed_bands: the slowest bands left unrotated (partial RoPE; 0 = all rotate)."""
     if isinstance(dtype, torch.dtype):
         dtype = _DTYPE[dtype]
     return RaProblem(int(B), int(H), int(n), int(d), int(dtype), int(bool(causal)), float(base),
-                     int(fixed_bands), RA_FLAG_FUSED_BWD if fused else 0)
+                     int(fixed_bands), 0)
 
 
-def _problem_of(q, causal, base, fixed_bands=0, fused=False):
+def _problem_of(q, causal, base, fixed_bands=0):
     B, H, n, d = q.shape
-    return problem(B, H, n, d, q.dtype, causal, base, fixed_bands, fused)
+    return problem(B, H, n, d, q.dtype, causal, base, fixed_bands)
 
 
 def _ptr(t):
@@ -194,11 +192,10 @@ def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
 
 
 def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk=None, dv=None,
-                  dalpha=None, fixed_bands=0, frozen_alpha=False, fused=False):
+                  dalpha=None, fixed_bands=0, frozen_alpha=False):
     """(dq, dk, dv, dalpha) of L for upstream gradient dO.  frozen_alpha: the frequencies
-    are not trained; no dalpha is computed and None is returned in its place.
-    fused: the one-pass backward (dQ summed over key blocks in arrival order)."""
-    prob = _problem_of(q, causal, base, fixed_bands, fused)
+    are not trained; no dalpha is computed and None is returned in its place."""
+    prob = _problem_of(q, causal, base, fixed_bands)
     if ws is None:
         ws = workspace(prob, q.device)
     dq = torch.empty_like(q) if dq is None else dq
@@ -216,10 +213,10 @@ def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk
 
 
 def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None, dv=None,
-                        dalpha=None, fixed_bands=0, frozen_alpha=False, fused=False):
+                        dalpha=None, fixed_bands=0, frozen_alpha=False):
     """rope_attn_bwd from the table, Q~ and K~ the preceding rope_attn_fwd left in ws
     (same problem, q, k and alpha; see include/rope_attn.h)."""
-    prob = _problem_of(v, causal, base, fixed_bands, fused)
+    prob = _problem_of(v, causal, base, fixed_bands)
     dq = torch.empty_like(v) if dq is None else dq
     dk = torch.empty_like(v) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv

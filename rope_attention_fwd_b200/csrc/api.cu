@@ -78,8 +78,7 @@ ra_status check_problem(const ra_problem* p) {
   if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
   if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
   if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
-  if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 ||
-      (p->flags & ~RA_FLAG_FUSED_BWD) != 0)
+  if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 || p->reserved != 0)
     return RA_ERR_INVALID_ARG;
   if (p->d > 128) return RA_ERR_UNSUPPORTED;
   if (p->dtype == RA_BF16 && p->d != 64 && p->d != 128) return RA_ERR_UNSUPPORTED;
@@ -140,20 +139,6 @@ bool make_map(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows,
   return fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
             const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// fp32 [BH][n][d] tensor viewed as (x = d, y = n, z = BH), box = d columns x `rows` rows, no
-// swizzle (the fused backward's dQ~ accumulator, the target of its bulk reductions).
-bool make_map_f32_rows(CUtensorMap* map, const void* ptr, const ra_problem& p, int rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)p.d, (cuuint64_t)p.n, (cuuint64_t)(p.B * p.H)};
-  const cuuint64_t strides[2] = {(cuuint64_t)p.d * 4, (cuuint64_t)p.n * p.d * 4};
-  const cuuint32_t box[3] = {(cuuint32_t)p.d, (cuuint32_t)rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -319,25 +304,12 @@ ra_status bwd_impl(const ra_problem* p, const void* q, const void* k, const void
         !make_map(&maps.v64, v, *p, 64) || !make_map(&maps.dO64, dO, *p, 64))
       return RA_ERR_CUDA;
     DevCtl ctl{at<uint32_t>(ws, L.err), wait_limit_ns(), -1};
-    if (uses_fused_bwd(*p)) {
-      float* dqacc = at<float>(ws, L.dqacc);
-      if (cudaMemsetAsync(dqacc, 0, sizeof(float) * (size_t)(p->B * p->H * p->n * p->d), s) !=
-          cudaSuccess)
-        return RA_ERR_CUDA;
-      if (!make_map_f32_rows(&maps.dqacc, dqacc, *p, 64)) return RA_ERR_CUDA;
-      RA_LAUNCH(K_BWD_FUSED_SM100, s,
-                launch_bwd_fused_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
-                                       s));
-      RA_LAUNCH(K_DQ_FINISH, s, launch_dq_finish(*p, dqacc, table, stats, dq, s));
-    } else {
-      // two passes (the default): dK, dV (keys stationary), then dQ (queries stationary, S
-      // and dP recomputed); every output bitwise reproducible
-      RA_LAUNCH(K_BWD_DKDV_SM100, s,
-                launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl,
-                                      s));
-      RA_LAUNCH(K_BWD_DQ_SM100, s,
-                launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
-    }
+    // two passes: dK, dV (keys stationary), then dQ (queries stationary, S and dP
+    // recomputed); every output bitwise reproducible
+    RA_LAUNCH(K_BWD_DKDV_SM100, s,
+              launch_bwd_dkdv_sm100(*p, maps, lse2, delta, table, stats, dk, dv, dpart, ctl, s));
+    RA_LAUNCH(K_BWD_DQ_SM100, s,
+              launch_bwd_dq_sm100(*p, maps, lse2, delta, table, stats, dq, dpart, ctl, s));
   }
   if (dalpha) RA_LAUNCH(K_DALPHA, s, launch_dalpha_final(*p, dpart, alpha, dalpha, s));
   return RA_OK;
@@ -438,7 +410,7 @@ const char* rope_attn_kernel_name(int id) {
       "rope_table",       "rotate",       "fwd_f32",      "fwd_sm100",
       "loss_partial",     "loss_final",   "bwd_delta",    "bwd_dq_f32",
       "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final",
-      "bwd_fused_sm100",  "dq_finish",    "proj_gemm"};
+      "proj_gemm"};
   return (id >= 0 && id < K_COUNT) ? names[id] : "unknown";
 }
 

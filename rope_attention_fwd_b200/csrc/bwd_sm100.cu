@@ -27,22 +27,20 @@
 // a CPU model of the roundings (bf16 operands) puts the dalpha error at 1.0e-2 that way,
 // 3.8e-3 this way.
 //
-// Two forms:
-//   fused (bf16, d = 128, RA_FLAG_FUSED_BWD): one kernel, 128 keys stationary per CTA, queries
-//         streamed 64 at a time; per step S^T, dP^T, then dV += P^T dO_i, dK~ += dS^T Q~_i
-//         (TMEM accumulators) and dQ~^T = K~^T dS^T, whose partial is added into an fp32
-//         accumulator in global memory; dq_finish_kernel rotates the sum back.
-//   two-pass (the default): no atomics, every output reproducible
-//     dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
-//           time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
-//           (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T
-//           (fp16), then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
-//           accumulated in TMEM for the whole pass.
-//     dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
-//           dP = dO V_j^T (double-buffered in TMEM), dS in fp16, dQ~ += dS K~_j.
+// Two kernels, no atomics (every output bitwise reproducible):
+//   dkdv: 128 keys stationary per CTA (K~, V in shared memory), queries stream 64 at a
+//         time.  Per step: S^T = K~ Q~_i^T and dP^T = V dO_i^T on the tensor core
+//         (M = 128 keys, N = 64 queries), the softmax warps form P^T (bf16) and dS^T (fp16),
+//         then dV += P^T dO_i and dK~ += dS^T Q~_i (M = 128, N = d, K = 64), both
+//         accumulated in TMEM for the whole pass.
+//   dq:   128 queries stationary (Q~, dO), keys stream 64 at a time.  S = Q~ K~_j^T and
+//         dP = dO V_j^T (double-buffered in TMEM), dS in fp16, dQ~ += dS K~_j.
+// A single pass that adds each key block's dQ~ partial into an fp32 accumulator was built
+// and measured slower on the B200 (its per-step dQ~ hand-off cost more issue slots than the
+// softmax, and the L2's fp32 reduction rate bounds such a pass near the two kernels' time).
 // Warp roles: two softmax warpgroups (warps 0-7) each own every row (TMEM lane) and half
 // of the 64 streamed columns; warp 8 issues TMA copies; warp 9 allocates TMEM and issues
-// tcgen05.mma; in the fused kernel warps 10-13 drain dQ~.  Every wait is bounded.
+// tcgen05.mma.  Every wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -789,441 +787,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ======================================================================== fused dK, dV, dQ
-// One pass over every (key block, query tile) pair computes all three gradients.  The dQ
-// kernel above recomputes S and dP (three MMAs per pair for the one that counts); here each
-// query tile's dS is used three times as soon as it exists: dV += P^T dO, dK~ += dS^T Q~
-// (accumulated in TMEM for the whole pass, as in bwd_dkdv_kernel) and dQ~^T = K~^T dS^T,
-// whose 128 x 64 partial is staged in shared memory and added to an fp32 accumulator in
-// global memory with one TMA bulk reduction per step (the L2 adds whole sectors; per-element
-// atomics measured about ten times slower), then rotated back by dq_finish_kernel once every
-// key block has added its share ("RoPE attention can be trained in almost-linear time",
-// Metodologia 1: gamma(x) is formed once per tile and feeds every gradient).
-//
-// CTA: 128 keys (K~, V stationary in shared memory), queries streamed 64 at a time through a
-// 3-stage ring.  14 warps:
-//   warps 0-7    softmax: both warpgroups take every tile, warpgroup g its query columns
-//                32g..32g+31, thread t its key row t (TMEM lane); P^T (bf16) and dS^T (fp16)
-//                go back into TMEM over S^T / dP^T, and dS^T also into shared memory as the
-//                MN-major B operand of the dQ~^T MMA;
-//   warp  8      TMA producer;
-//   warp  9      TMEM allocator and MMA issuer;
-//   warps 10-13  dQ drain: thread c owns TMEM lane c = dimension c of dQ~^T; it reads the
-//                step's 64 query columns, writes them into the [64][d] fp32 staging tile
-//                (one thread issues the bulk reduction of the tile) and forms the Q-side
-//                band torques of the step from them.
-// TMEM (512 columns): buffer b in {0, 1}: S^T at 128 b, dP^T at 128 b + 64 (64 queries each);
-// dQ~^T of the step that used buffer b is written over its S^T half once the dV MMA has read
-// P^T there (one thread's MMAs execute in issue order); dV at 256, dK~ at 384.
-// Per step t (buffer b = t & 1):
-//   MMA:     S^T, dP^T(t+1) [after the drain has read dQ~^T(t-1) out of that buffer];
-//            dV(t), dK~(t), dQ~^T(t) [after the softmax of t]
-//   softmax: P^T, dS^T(t) from S^T, dP^T(t)
-//   drain:   dQ~^T(t) -> registers -> global accumulator, torques
-//
-// dalpha stays bitwise deterministic although the dQ~ sums are not: the Q-side torque
-// sum_p (p - c) <dQ~_pm, J q~_pm> is linear in dQ~, so each CTA forms it from its own
-// partial dQ~^(j) (fixed order within the CTA) and writes one partial per key block; the
-// final reduction adds the partials in a fixed order.  dQ itself depends on the order in
-// which key blocks add into the accumulator (last fp32 bits, seldom visible in bf16).
-template <int D>
-struct FusedCfg {
-  static_assert(D == 128, "the fused backward takes d = 128");
-  static constexpr int BN = 128, BQ = 64, NS = 3, CH = D / 64;
-  static constexpr uint32_t KCH = 128u * 128u;  // chunk of a 128-row tile
-  static constexpr uint32_t KTILE = KCH * CH;
-  static constexpr uint32_t QCH = 64u * 128u;   // chunk of a 64-row tile
-  static constexpr uint32_t QTILE = QCH * CH;
-  static constexpr uint32_t VEC = BQ * 4;
-  static constexpr uint32_t STAGE = (2 * QTILE + 2 * VEC + 1023) / 1024 * 1024;
-  static constexpr uint32_t DSB = 128u * 128u;  // dS^T [128 keys][64 queries] fp16, SW128
-  static constexpr uint32_t OFF_K = 0, OFF_V = KTILE, OFF_ST = 2 * KTILE;
-  static constexpr uint32_t OFF_DS = OFF_ST + NS * STAGE;
-  static constexpr uint32_t DQS = BQ * D * 4u;  // a step's dQ~ partial, [64 queries][d] fp32
-  static constexpr uint32_t OFF_DQS = OFF_DS + DSB;
-  static constexpr uint32_t OFF_BAR = OFF_DQS + DQS;
-  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DV = 256, COL_DK = 384;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t RED_BYTES = (128u * (D / 2 + 1) * 4u + 1023u) / 1024u * 1024u;
-  static_assert(NS * STAGE >= RED_BYTES + TabStage<D>::BYTES,
-                "torque buffer and staged table fit the stages");
-  static_assert(SMEM <= 232448, "fits the shared memory of one CTA");
-};
-
-constexpr int kFusedDrainWarp0 = kSoftThreads / 32 + 2;          // warps 10..13
-constexpr int kFusedThreads = kSoftThreads + 64 + 128;            // 448
-
-__device__ __forceinline__ void drain_group_sync() {
-  asm volatile("bar.sync 2, 128;" ::: "memory");
-}
-
-enum FusedBar {
-  FB_KV_FULL = 0,
-  FB_Q_FULL = 1,      // +stage (4)
-  FB_Q_EMPTY = 5,     // +stage (4): MMA commit + one arrival per drain warp
-  FB_SDP_FULL = 9,    // +buffer: S^T, dP^T computed
-  FB_DS_FULL = 11,    // +buffer: P^T, dS^T written (TMEM and shared memory)
-  FB_DQ_FULL = 13,    // +buffer: dQ~^T of the buffer's step computed
-  FB_DQ_FREE = 15,    // +buffer: dQ~^T read out by the drain warps
-  FB_DSM_FREE = 17,   // the dQ~^T MMA of the last step has read dS^T from shared memory
-  FB_ACC_DONE = 18,
-  FB_DRAIN = 19,
-  FB_DRAIN_DONE = 20, // the drain warps have left their loop (one arrival per warp)
-  FB_COUNT = 21
-};
-static_assert(8 * FB_COUNT + 8 <= 256, "barriers, TMEM slot and abort flag fit the reserve");
-
-template <int D>
-__global__ void __launch_bounds__(kFusedThreads, 1)
-    bwd_fused_kernel(const __grid_constant__ CUtensorMap map_kt,
-                     const __grid_constant__ CUtensorMap map_v,
-                     const __grid_constant__ CUtensorMap map_qt64,
-                     const __grid_constant__ CUtensorMap map_do64,
-                     const float* __restrict__ lse2p, const float* __restrict__ deltap,
-                     const float2* __restrict__ table, const uint32_t* __restrict__ stats,
-                     __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                     const __grid_constant__ CUtensorMap map_dqacc, float* __restrict__ dpart,
-                     int n, int BH, int causal, uint32_t* err, uint64_t wait_ns) {
-  using C = FusedCfg<D>;
-  constexpr int KID = K_BWD_FUSED_SM100;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_s = smem_u32(smem_raw);
-  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
-  uint8_t* base = smem_raw + (base_s - raw_s);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * FB_COUNT);
-  volatile int* abort_flag =
-      reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * FB_COUNT + 4);
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // head-major grid: the CTAs resident at one time share a few heads' Q~ / dO stream in L2;
-  // key tile 0 (the most causal work) first within a head
-  const int ntk_grid = (n + C::BN - 1) / C::BN;
-  const int jt = (int)(blockIdx.x % ntk_grid);
-  const int bh = (int)(blockIdx.x / ntk_grid);
-  const int npad = (int)((n + 127) / 128 * 128);
-  const int qstart = causal ? jt * C::BN : 0;
-  const int nq = (n - qstart + C::BQ - 1) / C::BQ;
-
-  if (threadIdx.x == kSoftThreads) {
-    for (int i = 0; i < FB_COUNT; ++i) {
-      uint32_t cnt = 1;
-      if (i >= FB_Q_EMPTY && i < FB_Q_EMPTY + C::NS) cnt = 1 + 4;
-      if (i == FB_DS_FULL || i == FB_DS_FULL + 1) cnt = kSoftThreads / 32;
-      if (i == FB_DQ_FREE || i == FB_DQ_FREE + 1 || i == FB_DRAIN_DONE) cnt = 4;
-      mbar_init(&bar[i], cnt);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == kProdWarp) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&map_kt);
-      tma_prefetch_desc(&map_v);
-      tma_prefetch_desc(&map_qt64);
-      tma_prefetch_desc(&map_do64);
-      mbar_arrive_expect_tx(&bar[FB_KV_FULL], 2 * C::KTILE);
-      for (int c = 0; c < C::CH; ++c) {
-        tma_load_3d(base + C::OFF_K + c * C::KCH, &map_kt, &bar[FB_KV_FULL], c * 64, jt * C::BN,
-                    bh);
-        tma_load_3d(base + C::OFF_V + c * C::KCH, &map_v, &bar[FB_KV_FULL], c * 64, jt * C::BN,
-                    bh);
-      }
-      int issued = -1;
-      for (int it = 0; it < nq; ++it) {
-        const int s = it % C::NS;
-        if (!mbar_wait(&bar[FB_Q_EMPTY + s], ((it / C::NS) & 1) ^ 1, abort_flag, err, KID, 1,
-                       wait_ns))
-          break;
-        const int i0 = qstart + it * C::BQ;
-        uint8_t* st = base + C::OFF_ST + s * C::STAGE;
-        mbar_arrive_expect_tx(&bar[FB_Q_FULL + s], 2 * C::QTILE + 2 * C::VEC);
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_3d(st + c * C::QCH, &map_qt64, &bar[FB_Q_FULL + s], c * 64, i0, bh);
-          tma_load_3d(st + C::QTILE + c * C::QCH, &map_do64, &bar[FB_Q_FULL + s], c * 64, i0,
-                      bh);
-        }
-        bulk_load(st + 2 * C::QTILE, lse2p + (size_t)bh * npad + i0, C::VEC,
-                  &bar[FB_Q_FULL + s]);
-        bulk_load(st + 2 * C::QTILE + C::VEC, deltap + (size_t)bh * npad + i0, C::VEC,
-                  &bar[FB_Q_FULL + s]);
-        issued = it;
-      }
-      if (*abort_flag) {
-        int dummy = 0;
-        mbar_wait(&bar[FB_KV_FULL], 0, &dummy, err, KID, 20, wait_ns);
-        for (int it = max(0, issued - C::NS + 1); it <= issued; ++it)
-          mbar_wait(&bar[FB_Q_FULL + it % C::NS], (it / C::NS) & 1, &dummy, err, KID, 21,
-                    wait_ns);
-      }
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idST = idesc_f16_f32(128, C::BQ, 0, 0);   // fp16 K~ Q~^T
-    constexpr uint32_t idDPT = idesc_bf16_f32(128, C::BQ, 0, 0);  // bf16 V dO^T
-    constexpr uint32_t idDV = idesc_bf16_f32(128, D, 0, 1);       // bf16 P^T dO
-    constexpr uint32_t idDK = idesc_f16_f32(128, D, 0, 1);        // fp16 dS^T Q~
-    constexpr uint32_t idDQ = idesc_f16_f32(D, C::BQ, 1, 1);      // fp16 K~^T dS^T
-    const SDesc dkm = sdesc_split(base_s, 16, 1024);        // K-major tiles
-    const SDesc dmn = sdesc_split(base_s, C::QCH, 1024);    // Q~ / dO tiles read MN-major
-    const SDesc kmn = sdesc_split(base_s, C::KCH, 1024);    // K~ read MN-major (A = K~^T)
-    const SDesc dsd = sdesc_split(base_s, C::DSB, 1024);    // dS^T, MN-major B (one chunk)
-    bool ok = mbar_wait_warp(&bar[FB_KV_FULL], 0, abort_flag, err, KID, 2, wait_ns);
-    auto issue_sdp = [&](int it) -> bool {
-      const int s = it % C::NS, b = it & 1;
-      if (!mbar_wait_warp(&bar[FB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 3,
-                          wait_ns))
-        return false;
-      // buffer b last held dQ~^T of step it - 2: wait until the drain has read it
-      if (it >= 2 && !mbar_wait_warp(&bar[FB_DQ_FREE + b], ((it - 2) >> 1) & 1, abort_flag, err,
-                                     KID, 4, wait_ns))
-        return false;
-      tc_fence_after();
-      const SDesc qs = sdesc_advance(dkm, C::OFF_ST + s * C::STAGE);
-      mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K),
-                                         sdesc_at(qs, 0), idST, 0);
-      mma8_kmajor<false, C::KCH, C::QCH>(tmem + b * 128 + C::COL_DPT, sdesc_at(dkm, C::OFF_V),
-                                         sdesc_at(qs, C::QTILE), idDPT, 0);
-      mma_commit_warp(&bar[FB_SDP_FULL + b]);
-      return true;
-    };
-    if (ok && nq > 0) ok = issue_sdp(0);
-    for (int it = 0; ok && it < nq; ++it) {
-      if (it + 1 < nq && !issue_sdp(it + 1)) break;
-      const int s = it % C::NS, b = it & 1;
-      if (!mbar_wait_warp(&bar[FB_DS_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 5, wait_ns))
-        break;
-      tc_fence_after();
-      const SDesc qm = sdesc_advance(dmn, C::OFF_ST + s * C::STAGE);
-      // dV += P^T dO_i and dK~ += dS^T Q~_i with P^T, dS^T read from TMEM
-      mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
-          tmem + C::COL_DV, tmem + b * 128 + C::COL_ST, sdesc_at(qm, C::QTILE), idDV, it > 0);
-      mma4_ts_mn<packed_col(16), packed_col(32), packed_col(48)>(
-          tmem + C::COL_DK, tmem + b * 128 + C::COL_DPT, sdesc_at(qm, 0), idDK, it > 0);
-      // dQ~^T (d x 64) = K~^T dS^T over the CTA's 128 keys, into the S^T half of buffer b
-      // (after the dV MMA above has read P^T there)
-      mma8_ss_mn(tmem + b * 128 + C::COL_ST, sdesc_at(kmn, C::OFF_K), sdesc_at(dsd, C::OFF_DS),
-                 idDQ, 0);
-      mma_commit_warp(&bar[FB_DQ_FULL + b]);
-      mma_commit_warp(&bar[FB_DSM_FREE]);
-      mma_commit_warp(&bar[FB_Q_EMPTY + s]);
-    }
-    if (ok) mma_commit_warp(&bar[FB_ACC_DONE]);
-    mma_commit_warp(&bar[FB_DRAIN]);
-    int dummy = 0;
-    mbar_wait_warp(&bar[FB_DRAIN], 0, &dummy, err, KID, 22, wait_ns);
-  } else if (warp >= kFusedDrainWarp0) {
-    // ------------------------------------------------------------ dQ drain
-    const int c = (warp % 4) * 32 + lane;  // dimension == TMEM lane
-    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-    const float center = 0.5f * (float)(n - 1);
-    // this lane's fp16 pair (x~_2m, x~_2m+1) inside a Q~ tile row: chunk, 16-byte unit, byte
-    const uint32_t pair_chunk = (uint32_t)(c / 64) * C::QCH;
-    const uint32_t pair_unit = (uint32_t)((c % 64) / 8);
-    const uint32_t pair_byte = (uint32_t)((c % 8) & ~1) * 2u;
-    double torque = 0.0;  // sum over the CTA's steps of this lane's query parity
-    float* dqs = reinterpret_cast<float*>(base + C::OFF_DQS);
-    if (threadIdx.x == kFusedDrainWarp0 * 32) tma_prefetch_desc(&map_dqacc);
-    for (int it = 0; it < nq; ++it) {
-      const int s = it % C::NS, b = it & 1;
-      const int i0 = qstart + it * C::BQ;
-      if (!mbar_wait_warp(&bar[FB_DQ_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 12,
-                          wait_ns))
-        break;
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(lane_base + b * 128 + C::COL_ST, r0);
-      tmem_ld32(lane_base + b * 128 + C::COL_ST + 32, r1);
-      tmem_wait_ld(r0);
-      tmem_wait_ld(r1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[FB_DQ_FREE + b]);
-      // the staging tile is free once the previous step's bulk reduction has read it
-      if (threadIdx.x == kFusedDrainWarp0 * 32) bulk_wait_read();
-      drain_group_sync();
-      // row q = query i0 + q, column c: consecutive lanes write consecutive words
-#pragma unroll
-      for (int q = 0; q < 32; ++q) dqs[q * D + c] = __uint_as_float(r0[q]);
-#pragma unroll
-      for (int q = 0; q < 32; ++q) dqs[(32 + q) * D + c] = __uint_as_float(r1[q]);
-      fence_proxy_async_smem();
-      drain_group_sync();
-      if (threadIdx.x == kFusedDrainWarp0 * 32) {
-        // accumulator += tile (rows past n fall outside the tensor map and are skipped)
-        tma_reduce_add_3d(&map_dqacc, dqs, 0, i0, bh);
-        bulk_commit();
-      }
-      if (dpart != nullptr) {
-        // band torque g1 x0 - g0 x1 of band c/2 for the queries of this lane's parity
-        const uint8_t* qtile = base + C::OFF_ST + s * C::STAGE + pair_chunk;
-        const bool odd = (c & 1) != 0;
-        float acc = 0.f;
-#pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          const float mine = __uint_as_float(q < 32 ? r0[q] : r1[q - 32]);
-          const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-          if ((q & 1) == (int)odd) {
-            const __half2 xp = *reinterpret_cast<const __half2*>(
-                qtile + sw128_off((uint32_t)q, pair_unit) + pair_byte);
-            const float x0 = __low2float(xp), x1 = __high2float(xp);
-            const float g0 = odd ? other : mine, g1 = odd ? mine : other;
-            const float w = (float)(i0 + q) - center;
-            acc = fmaf(w, g1 * x0 - g0 * x1, acc);  // rows past n hold g = 0
-          }
-        }
-        torque += (double)acc;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[FB_Q_EMPTY + s]);
-    }
-    // the last reductions complete (and stop reading shared memory) before the CTA exits
-    if (threadIdx.x == kFusedDrainWarp0 * 32) bulk_wait();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar[FB_DRAIN_DONE]);
-    if (dpart != nullptr) {
-      // this CTA's Q-side partial of band c/2: the two lanes of the pair hold the even and
-      // odd query rows; scale as the epilogues do (1 / (sqrt(d) s))
-      const double other = __shfl_xor_sync(0xffffffffu, torque, 1);
-      const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      const int ntile128 = (n + C::BN - 1) / C::BN;
-      float* side = dpart + (size_t)(0 * BH + bh) * ntile64 * (D / 2);
-      if ((c & 1) == 0) {
-        const double scale = (double)rsqrtf((float)D) / (double)ds_scale(stats);
-        side[(size_t)jt * (D / 2) + c / 2] = (float)((torque + other) * scale);
-        // slots past the key tiles (the Q side has one partial per 128 rows here) are zero
-        if (ntile128 + jt < ntile64) side[(size_t)(ntile128 + jt) * (D / 2) + c / 2] = 0.f;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = threadIdx.x % 128;      // key row == TMEM lane
-    const int half = threadIdx.x / 128;   // warpgroup: query columns 32 half .. 32 half + 31
-    const int key = jt * C::BN + t;
-    const uint32_t lane_base = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-    const float scale_log2 = kLog2e / sqrtf((float)D);
-    const float dss = ds_scale(stats);
-    // this thread's 4 16-byte units of the dS^T row in shared memory (128B-swizzled)
-    const uint32_t ds_row = base_s + C::OFF_DS + (uint32_t)t * 128u;
-    bool ok = true;
-    for (int it = 0; it < nq; ++it) {
-      const int s = it % C::NS, b = it & 1;
-      const int i0 = qstart + it * C::BQ;
-      if (!mbar_wait_warp(&bar[FB_Q_FULL + s], (it / C::NS) & 1, abort_flag, err, KID, 6,
-                          wait_ns) ||
-          !mbar_wait_warp(&bar[FB_SDP_FULL + b], (it >> 1) & 1, abort_flag, err, KID, 7,
-                          wait_ns)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t st_base = lane_base + b * 128 + C::COL_ST;
-      const uint32_t dpt_base = lane_base + b * 128 + C::COL_DPT;
-      const float4* lv = reinterpret_cast<const float4*>(base + C::OFF_ST + s * C::STAGE +
-                                                         2 * C::QTILE);
-      const float4* dvv = lv + C::BQ / 4;
-      const bool need_mask = causal && (i0 < jt * C::BN + C::BN);
-      uint32_t sr[32], dr[32];
-      tmem_ld32(st_base + 32 * half, sr);
-      tmem_ld32(dpt_base + 32 * half, dr);
-      tmem_wait_ld(sr);
-      tmem_wait_ld(dr);
-      uint32_t pw[16], dw[16];
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 l4 = lv[8 * half + c4], d4 = dvv[8 * half + c4];
-        const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pv[4], dsv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int cc = 4 * c4 + e;  // column within this warpgroup's half
-          float p = fast_exp2(__uint_as_float(sr[cc]) * scale_log2 - la[e]);
-          if (need_mask && (i0 + 32 * half + cc < key)) p = 0.f;
-          pv[e] = p;
-          dsv[e] = p * (__uint_as_float(dr[cc]) - da[e]) * dss;
-        }
-        pw[2 * c4] = pack_bf16x2(pv[0], pv[1]);
-        pw[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
-        dw[2 * c4] = pack_f16x2_sat(dsv[0], dsv[1]);
-        dw[2 * c4 + 1] = pack_f16x2_sat(dsv[2], dsv[3]);
-      }
-      tmem_st16(st_base + packed_col(32 * half), pw);
-      tmem_st16(dpt_base + packed_col(32 * half), dw);
-      // dS^T row t, query columns 32 half .. + 31 = 16-byte units 4 half .. 4 half + 3, into
-      // shared memory once the previous step's dQ~^T MMA has read it
-      if (it >= 1 && !mbar_wait_warp(&bar[FB_DSM_FREE], (it - 1) & 1, abort_flag, err, KID, 9,
-                                     wait_ns)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        st_shared_v4(ds_row + (((uint32_t)(4 * half + u) ^ ((uint32_t)t & 7u)) << 4),
-                     dw[4 * u], dw[4 * u + 1], dw[4 * u + 2], dw[4 * u + 3]);
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[FB_DS_FULL + b]);
-    }
-    // the ring holds the torque buffer and the table once every MMA (ACC_DONE) and the
-    // drain warps' torque reads of the last Q~ tiles (DRAIN_DONE) are finished
-    if (ok && mbar_wait_warp(&bar[FB_ACC_DONE], 0, abort_flag, err, KID, 10, wait_ns) &&
-        mbar_wait_warp(&bar[FB_DRAIN_DONE], 0, abort_flag, err, KID, 13, wait_ns)) {
-      tc_fence_after();
-      const bool live = key < n;
-      float* red = reinterpret_cast<float*>(base + C::OFF_ST);
-      uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
-      stage_table<D>(table, jt * C::BN, n, tab);
-#pragma unroll
-      for (int cc = 0; cc < D / 32 / kSoftWG; ++cc) {
-        const int c = half * (D / 32 / kSoftWG) + cc;
-        uint32_t r[32];
-        tmem_ld32(lane_base + C::COL_DV + 32 * c, r);
-        tmem_wait_ld(r);
-        if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)bh * n + key) * D + 32 * c);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float* f = reinterpret_cast<const float*>(&r[8 * u]);
-            dst[u] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                                pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-          }
-        }
-      }
-      softmax_group_sync();
-      grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
-                           tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
-                           (float)key - 0.5f * (float)(n - 1), live,
-                           dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
-                           half);
-      softmax_group_sync();
-      const int ntile64 = (n + kDalphaRows - 1) / kDalphaRows;
-      if (dpart != nullptr && threadIdx.x < 128)
-        write_dalpha_partials<D>(red, dpart + ((size_t)(1 * BH + bh) * ntile64) * (D / 2), jt,
-                                 ntile64, t);
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kMmaWarp) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
 template <int D>
 cudaError_t launch_dkdv_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
                           const float* deltap, const float2* table, const uint32_t* stats,
@@ -1257,72 +820,7 @@ cudaError_t launch_dq_d(const ra_problem& p, const Sm100Maps& maps, const float*
   return cudaGetLastError();
 }
 
-cudaError_t launch_fused_d(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
-                           const float* deltap, const float2* table, const uint32_t* stats,
-                           void* dk, void* dv, float* dpart, const DevCtl& ctl,
-                           cudaStream_t s) {
-  using C = FusedCfg<128>;
-  cudaError_t e = cudaFuncSetAttribute(bwd_fused_kernel<128>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  const int BH = (int)(p.B * p.H);
-  const long long ntk = (p.n + C::BN - 1) / C::BN;
-  bwd_fused_kernel<128><<<(unsigned)(ntk * BH), kFusedThreads, C::SMEM, s>>>(
-      maps.kt, maps.v, maps.qt64, maps.dO64, lse2p, deltap, table, stats, (__nv_bfloat16*)dk,
-      (__nv_bfloat16*)dv, maps.dqacc, dpart, (int)p.n, BH, p.causal, ctl.err, ctl.wait_ns);
-  return cudaGetLastError();
-}
-
-// dQ from the fused kernel's fp32 accumulator of dQ~ * sqrt(d) * s: scaled by 1 / (sqrt(d) s)
-// and rotated back by -p theta_hat band by band (R(-phi) (g0, g1) = (c g0 + s g1, c g1 - s g0)),
-// written as bf16.  8 elements (4 bands) per thread; HBM-bound.
-template <int D>
-__global__ void __launch_bounds__(256)
-    dq_finish_kernel(const float4* __restrict__ acc, const float4* __restrict__ table,
-                     const uint32_t* __restrict__ stats, uint4* __restrict__ dq, long long rows,
-                     int n) {
-  constexpr int VPR = D / 8;  // 8-element vectors per row
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * VPR) return;
-  const long long row = idx / VPR;
-  const int v = (int)(idx % VPR);
-  const int pos = (int)(row % n);
-  const float scale = rsqrtf((float)D) / ds_scale(stats);
-  const float4 g01 = acc[2 * idx], g23 = acc[2 * idx + 1];
-  const float4 t01 = table[(size_t)pos * (D / 4) + 2 * v];      // bands 4v, 4v + 1
-  const float4 t23 = table[(size_t)pos * (D / 4) + 2 * v + 1];  // bands 4v + 2, 4v + 3
-  const float g[8] = {g01.x, g01.y, g01.z, g01.w, g23.x, g23.y, g23.z, g23.w};
-  const float cs[8] = {t01.x, t01.y, t01.z, t01.w, t23.x, t23.y, t23.z, t23.w};
-  uint32_t w[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float g0 = g[2 * k] * scale, g1 = g[2 * k + 1] * scale;
-    const float c = cs[2 * k], sn = cs[2 * k + 1];
-    w[k] = pack_bf16x2(c * g0 + sn * g1, c * g1 - sn * g0);
-  }
-  dq[idx] = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 }  // namespace
-
-cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,
-                                   const float* lse2p, const float* deltap, const float2* table,
-                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
-                                   const DevCtl& ctl, cudaStream_t s) {
-  if (p.d != 128) return cudaErrorInvalidValue;
-  return launch_fused_d(p, maps, lse2p, deltap, table, stats, dk, dv, dpart, ctl, s);
-}
-
-cudaError_t launch_dq_finish(const ra_problem& p, const float* dqacc, const float2* table,
-                             const uint32_t* stats, void* dq, cudaStream_t s) {
-  if (p.d != 128) return cudaErrorInvalidValue;
-  const long long rows = p.B * p.H * p.n;
-  const long long total = rows * (p.d / 8);
-  dq_finish_kernel<128><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-      reinterpret_cast<const float4*>(dqacc), reinterpret_cast<const float4*>(table), stats,
-      reinterpret_cast<uint4*>(dq), rows, (int)p.n);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,

@@ -21,10 +21,8 @@ enum KernelId : int {
   K_BWD_DQ_SM100 = 9,
   K_BWD_DKDV_SM100 = 10,
   K_DALPHA = 11,
-  K_BWD_FUSED_SM100 = 12,
-  K_DQ_FINISH = 13,
-  K_PROJ_GEMM = 14,
-  K_COUNT = 15
+  K_PROJ_GEMM = 12,
+  K_COUNT = 13
 };
 
 // Rows per dalpha partial (one partial per band per tile of query or key rows).
@@ -44,16 +42,9 @@ struct WsLayout {
   size_t delta;      // float [B*H][npad]   rowsum(dO o O); 0 on rows >= n
   size_t lse2;       // float [B*H][npad]   lse * log2(e); +inf on rows >= n
   size_t dpart;      // float [2][B*H][ceil(n/kDalphaRows)][M]
-  size_t dqacc;      // float [B*H][n][d]: dQ~ accumulator of the fused backward (bf16, d = 128)
   size_t total;
   size_t fwd_total;  // the regions the forward touches (error word .. K~): a prefix of total
 };
-
-// The one-pass backward (fused dK/dV/dQ kernel, an fp32 dQ~ accumulator in the workspace):
-// bf16 with d = 128 when the caller asks for it (RA_FLAG_FUSED_BWD).
-inline bool uses_fused_bwd(const ra_problem& p) {
-  return p.dtype == RA_BF16 && p.d == 128 && (p.flags & RA_FLAG_FUSED_BWD) != 0;
-}
 
 // Rows of the padded per-row vectors (a whole number of 128-row tiles).
 inline int64_t padded_rows(int64_t n) { return (n + 127) / 128 * 128; }
@@ -80,7 +71,6 @@ inline WsLayout ws_layout(const ra_problem& p) {
   w.delta = take(sizeof(float) * BH * npad);
   w.lse2 = take(sizeof(float) * BH * npad);
   w.dpart = take(sizeof(float) * 2 * BH * ntile * M);
-  w.dqacc = take(uses_fused_bwd(p) ? sizeof(float) * BH * n * d : 0);
   w.total = off;
   return w;
 }

@@ -55,7 +55,6 @@ cudaError_t launch_bwd_dkdv_f32(const ra_problem& p, const float* qt, const floa
 struct Sm100Maps {
   CUtensorMap qt, kt, v, dO;         // boxes of 64 columns x 128 rows
   CUtensorMap qt64, kt64, v64, dO64; // boxes of 64 columns x 64 rows
-  CUtensorMap dqacc;                 // fp32 [BH][n][d], box d x 64 rows, no swizzle (fused)
 };
 cudaError_t launch_fwd_sm100(const ra_problem& p, const Sm100Maps& maps, void* o, float* lse,
                              const DevCtl& ctl, cudaStream_t s);
@@ -70,14 +69,6 @@ cudaError_t launch_bwd_dkdv_sm100(const ra_problem& p, const Sm100Maps& maps,
                                   const float* lse2p, const float* deltap, const float2* table,
                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
                                   const DevCtl& ctl, cudaStream_t s);
-// Fused dK, dV and dQ~ (added into the fp32 accumulator behind maps.dqacc, zeroed by the
-// caller) in one pass (d = 128); dq_finish turns the accumulator into dQ.
-cudaError_t launch_bwd_fused_sm100(const ra_problem& p, const Sm100Maps& maps,
-                                   const float* lse2p, const float* deltap, const float2* table,
-                                   const uint32_t* stats, void* dk, void* dv, float* dpart,
-                                   const DevCtl& ctl, cudaStream_t s);
-cudaError_t launch_dq_finish(const ra_problem& p, const float* dqacc, const float2* table,
-                             const uint32_t* stats, void* dq, cudaStream_t s);
 cudaError_t launch_bwd_dq_sm100(const ra_problem& p, const Sm100Maps& maps, const float* lse2p,
                                 const float* deltap, const float2* table, const uint32_t* stats,
                                 void* dq, float* dpart, const DevCtl& ctl, cudaStream_t s);

@@ -36,10 +36,8 @@ int main(void) {
   bad.d = 3;
   expect(rope_attn_workspace_bytes(&bad) == 0, "odd d has no workspace");
   bad = p;
-  bad.flags = 2;
-  expect(rope_attn_workspace_bytes(&bad) == 0, "unknown flag bits are rejected");
-  bad.flags = RA_FLAG_FUSED_BWD;
-  expect(rope_attn_workspace_bytes(&bad) > 0, "the one-pass backward flag is accepted");
+  bad.reserved = 1;
+  expect(rope_attn_workspace_bytes(&bad) == 0, "reserved must be zero");
 
   expect(strcmp(rope_attn_status_string(RA_OK), "ok") == 0, "status string of RA_OK");
   expect(rope_attn_status_string(RA_ERR_TIMEOUT) != NULL, "status string of RA_ERR_TIMEOUT");

@@ -41,10 +41,6 @@ def test_workspace_bytes():
     # the two rotated 16-bit tensors dominate
     assert 2 * elems * 2 <= nb < 2 * elems * 2 * 1.1
     assert nb % 1024 == 0
-    # the one-pass backward adds the fp32 dQ accumulator
-    p = rb.problem(2, 32, 8192, 128, rb.RA_BF16, True, 1e4, fused=True)
-    nb = rb.rope_attn_workspace_bytes(p)
-    assert 2 * elems * 2 + 4 * elems <= nb < (2 * elems * 2 + 4 * elems) * 1.1
 
 
 @pytest.mark.parametrize("bad", [
@@ -106,25 +102,20 @@ def test_workspace_checks_before_launch():
 
 def test_kernel_names():
     lib = rb.lib()
-    names = {lib.rope_attn_kernel_name(i).decode() for i in range(14)}
+    names = {lib.rope_attn_kernel_name(i).decode() for i in range(13)}
     assert {"fwd_sm100", "bwd_dkdv_sm100", "bwd_dq_sm100", "dalpha_final",
-            "bwd_fused_sm100", "dq_finish"} <= names
+            "proj_gemm"} <= names
 
 
-def test_fixed_bands_and_flags_are_validated():
-    """fixed_bands must lie in 0..d/2 and flags hold only RA_FLAG_FUSED_BWD (checked before
-    any launch); only the one-pass backward needs the dQ accumulator."""
+def test_fixed_bands_and_reserved_are_validated():
+    """fixed_bands must lie in 0..d/2 and reserved must be 0 (checked before any launch)."""
     lib = rb.lib()
     for fb, ok in ((0, True), (64, True), (65, False), (-1, False)):
         p = rb.problem(1, 1, 256, 128, rb.RA_BF16, True, 1e4, fixed_bands=fb)
         assert (rb.rope_attn_workspace_bytes(p) > 0) == ok, fb
     p = rb.problem(1, 1, 256, 128, rb.RA_BF16, True, 1e4)
-    two_pass = lib.rope_attn_workspace_bytes(ctypes.byref(p))
-    p.flags = 2
+    p.reserved = 1
     assert lib.rope_attn_workspace_bytes(ctypes.byref(p)) == 0
-    p.flags = rb.RA_FLAG_FUSED_BWD
-    fused = lib.rope_attn_workspace_bytes(ctypes.byref(p))
-    assert 0 < two_pass and fused - two_pass >= 4 * 256 * 128  # the fp32 dQ accumulator
 
 
 def test_alpha_adam_rejects_bad_arguments():

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("dtype,d,n", [("f32", 16, 96), ("bf16", 64, 96), ("bf16", 128, 300),
-                                       ("f32", 128, 200)])
+                                       ("f32", 128, 200), ("bf16", 128, 1100)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_spectrum_matches_oracle_and_backward(dtype, d, n, causal):
     """Several 64-row blocks (the last one ragged), d up to 128."""

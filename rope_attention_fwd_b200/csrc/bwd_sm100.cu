@@ -361,20 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              sdesc_at(dkm, C::OFF_V), sdesc_at(qs, C::QTILE),
                                              idDPT, 0);
         } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
-            const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-            mma_ss_warp(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K + ka),
-                        sdesc_at(qs, kq), idST, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk / 4) * C::KCH + (kk % 4) * 32;
-            const uint32_t kq = (kk / 4) * C::QCH + (kk % 4) * 32;
-            mma_ss_warp(tmem + b * 128 + C::COL_DPT, sdesc_at(dkm, C::OFF_V + ka),
-                        sdesc_at(qs, C::QTILE + kq), idDPT, kk > 0);
-          }
+          mma4_kmajor<false>(tmem + b * 128 + C::COL_ST, sdesc_at(dkm, C::OFF_K), sdesc_at(qs, 0),
+                             idST, 0);
+          mma4_kmajor<false>(tmem + b * 128 + C::COL_DPT, sdesc_at(dkm, C::OFF_V),
+                             sdesc_at(qs, C::QTILE), idDPT, 0);
         }
         mma_commit_warp(&bar[KB_SDP_FULL + b]);
         return true;
@@ -655,18 +645,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma8_kmajor<true, 0, C::KCH>(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT,
                                        sdesc_at(ks, C::KTILE), idDP, 0);
         } else {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-            mma_ts_warp(tmem + C::COL_S + b * 128, tmem + C::COL_QT + 8 * kk, sdesc_at(ks, kq),
-                        idS, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t kq = (kk / 4) * C::KCH + (kk % 4) * 32;
-            mma_ts_warp(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT + 8 * kk,
-                        sdesc_at(ks, C::KTILE + kq), idDP, kk > 0);
-          }
+          mma4_kmajor<true>(tmem + C::COL_S + b * 128, tmem + C::COL_QT, sdesc_at(ks, 0), idS, 0);
+          mma4_kmajor<true>(tmem + C::COL_DP + b * 128, tmem + C::COL_DOT, sdesc_at(ks, C::KTILE),
+                            idDP, 0);
         }
         mma_commit_warp(&bar[QB_SP_FULL + b]);
         return true;

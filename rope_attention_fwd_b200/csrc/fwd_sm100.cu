@@ -224,12 +224,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma8_kmajor<false, C::CHUNK, C::CHUNK>(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off),
                                                sdesc_at(ks, 0), idS, 0);
       } else {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss_warp(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off + koff), sdesc_at(ks, koff),
-                      idS, kk > 0);
-        }
+        mma4_kmajor<false>(tmem + C::COL_S + x * 128, sdesc_at(dkm, q_off), sdesc_at(ks, 0), idS,
+                           0);
       }
       mma_commit_warp(&bar[B_S_FULL + x]);
     };

@@ -201,10 +201,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
         }
         tc_fence_after();
         const SDesc sa = sdesc_advance(da, s * GSTAGE), sb = sdesc_advance(db, s * GSTAGE);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss_warp(tmem + acc * 256, sdesc_at(sa, kk * astep), sdesc_at(sb, kk * bstep), idesc,
-                      (kc > 0 || kk > 0) ? 1u : 0u);
+        mma4_ss(tmem + acc * 256, sdesc_at(sa, 0), sdesc_at(sb, 0), idesc, kc > 0 ? 1u : 0u,
+                astep >> 4, bstep >> 4);
         mma_commit_warp(&bar[GB_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[GB_ACC_FULL + acc]);

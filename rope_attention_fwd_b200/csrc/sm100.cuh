@@ -291,6 +291,60 @@ __device__ __forceinline__ void mma8_kmajor(uint32_t d_tmem, uint64_t a, uint64_
   }
 }
 
+// mma4_kmajor: 4 K-steps of 16 inside one 64-column chunk (K = 64: the d = 64 forms of the
+// S-type products), K-major B (+32 B per step); A from TMEM (+8 columns per step) or
+// K-major in shared memory (+32 B per step).
+template <bool A_TMEM>
+__device__ __forceinline__ void mma4_kmajor(uint32_t d_tmem, uint64_t a, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t acc) {
+  if constexpr (A_TMEM) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a0, a1, a2, a3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+        "cvt.u32.u64 a0, %1;\n\t"
+        "add.u32 a1, a0, 8;\n\tadd.u32 a2, a0, 16;\n\tadd.u32 a3, a0, 24;\n\t"
+        "add.u64 b1, %2, 2;\n\tadd.u64 b2, %2, 4;\n\tadd.u64 b3, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a0], %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b_desc), "r"(idesc), "r"(acc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+        "add.u64 a1, %1, 2;\n\tadd.u64 a2, %1, 4;\n\tadd.u64 a3, %1, 6;\n\t"
+        "add.u64 b1, %2, 2;\n\tadd.u64 b2, %2, 4;\n\tadd.u64 b3, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b_desc), "r"(idesc), "r"(acc)
+        : "memory");
+  }
+}
+
+// mma4_ss: 4 K-steps of 16, both operands in shared memory, each descriptor advanced by its
+// own step per K-step (in 16-byte units: 2 for K-major, 128 for MN-major 128-byte rows).
+__device__ __forceinline__ void mma4_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc, uint64_t a_step16, uint64_t b_step16) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+      "add.u64 a1, %1, %5;\n\tadd.u64 a2, a1, %5;\n\tadd.u64 a3, a2, %5;\n\t"
+      "add.u64 b1, %2, %6;\n\tadd.u64 b2, b1, %6;\n\tadd.u64 b3, b2, %6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a2, b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a3, b3, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "l"(a_step16), "l"(b_step16)
+      : "memory");
+}
+
 // mma4_ts_mn: 4 K-steps of 16 with the A operand in TMEM at columns a0 + {0, A1, A2, A3}
 // and MN-major B (+2048 B = 16 rows of 128 B per step).
 template <uint32_t A1, uint32_t A2, uint32_t A3>

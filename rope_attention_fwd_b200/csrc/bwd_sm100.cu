@@ -270,11 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * KB_COUNT + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // head-major grid: the CTAs resident at one time share a few heads' Q~ / dO stream in L2;
-  // key tile 0 (the most causal work) first within a head
+  // grid in groups of kHeadGroup heads (grid_item): the resident CTAs share a few heads'
+  // Q~ / dO stream in L2
   const int ntk_grid = (n + C::BN - 1) / C::BN;
-  const int jt = (int)(blockIdx.x % ntk_grid);
-  const int bh = (int)(blockIdx.x / ntk_grid);
+  const GridItem gi = grid_item((int)blockIdx.x, ntk_grid, BH);
+  const int jt = gi.rank;  // key tile 0 (the most causal work) first
+  const int bh = gi.bh;
   const int npad = (int)((n + 127) / 128 * 128);
   const int qstart = causal ? jt * C::BN : 0;
   const int nq = (n - qstart + C::BQ - 1) / C::BQ;
@@ -559,10 +560,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
-  // head-major grid (the resident CTAs share a few heads' K~ / V stream in L2), heaviest
-  // causal tiles first within a head
-  const int qtile = ntq - 1 - (int)(blockIdx.x % ntq);
-  const int bh = (int)(blockIdx.x / ntq);
+  // grid in groups of kHeadGroup heads (grid_item): the resident CTAs share a few heads'
+  // K~ / V stream in L2
+  const GridItem gi = grid_item((int)blockIdx.x, ntq, BH);
+  const int qtile = ntq - 1 - gi.rank;  // heaviest causal query tile first
+  const int bh = gi.bh;
   const int npad = (int)((n + 127) / 128 * 128);
   const int kend = causal ? min(n, (qtile + 1) * C::BM) : n;
   const int nk = (kend + C::BK - 1) / C::BK;

@@ -27,6 +27,24 @@ enum KernelId : int {
 
 // Rows per dalpha partial (one partial per band per tile of query or key rows).
 constexpr int kDalphaRows = 64;
+
+// Grid order of the attention kernels: the CTAs of kHeadGroup (batch, head) pairs are
+// consecutive, heaviest causal tiles of the whole group first.  The CTAs resident at one
+// time share a few heads' streamed tiles in L2, and the last heads' heaviest tiles no
+// longer start at the end of the launch.  Measured on one B200 (2 x 32 x 8192 x 128
+// causal, three alternating runs): groups of 4 heads against 1 took the forward from
+// 1.117 to 1.052 ms and dQ from 1.405 to 1.382 ms, dK/dV from 1.881 to 1.906 ms, the step
+// from 4.728 to 4.674 ms.  Item r of a group is head r % heads, tile rank r / heads.
+struct GridItem {
+  int bh, rank;  // (batch, head) and the tile's rank in the heaviest-first order
+};
+constexpr int kHeadGroup = 4;
+__host__ __device__ inline GridItem grid_item(int block, int tiles_per_head, int BH) {
+  const int per_group = kHeadGroup * tiles_per_head;
+  const int g = block / per_group, r = block - g * per_group;
+  const int heads = BH - g * kHeadGroup < kHeadGroup ? BH - g * kHeadGroup : kHeadGroup;
+  return GridItem{g * kHeadGroup + r % heads, r / heads};
+}
 // Blocks of the first loss stage (fixed so the fp64 sum order never changes).
 constexpr int kLossBlocks = 1024;
 constexpr int kLossThreads = 256;

@@ -125,8 +125,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int ntq = (n + C::BM - 1) / C::BM;
   const int ntp = (ntq + 1) / 2;
-  const int T = ntp - 1 - (int)(blockIdx.x % ntp);
-  const int bh = (int)(blockIdx.x / ntp);
+  const GridItem gi = grid_item((int)blockIdx.x, ntp, BH);
+  const int T = ntp - 1 - gi.rank;  // heaviest causal pair first
+  const int bh = gi.bh;
   const int ntk = (n + C::BN - 1) / C::BN;
   // key tiles of query tile x (0 when the tile lies past the end of the sequence)
   auto nkv_of = [&](int x) -> int {

@@ -74,6 +74,10 @@ __global__ void rotate_kernel(const T* __restrict__ q, const T* __restrict__ k,
 // bf16 inputs: 4 pairs (16 bytes) per thread; the rotated rows are written as fp16, the
 // score-operand type of the tensor-core path (11-bit significand).  An entry beyond the
 // fp16 range is clamped (satfinite) and reported as status 6 (RA_ERR_RANGE) in err[0].
+// Each thread rotates kRotUnroll vectors of 8 elements, blockDim.x apart inside its block's
+// span, with all loads issued before the arithmetic, so that enough bytes are in flight to
+// stream at the HBM rate.
+constexpr int kRotUnroll = 4;
 __global__ void rotate_bf16x8_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k,
                                      uint4* __restrict__ qt, uint4* __restrict__ kt,
                                      const float2* __restrict__ table, long long rows, int n,
@@ -81,29 +85,43 @@ __global__ void rotate_bf16x8_kernel(const uint4* __restrict__ q, const uint4* _
   const uint4* src = blockIdx.y == 0 ? q : k;
   uint4* dst = blockIdx.y == 0 ? qt : kt;
   const int vec_per_row = M / 4;  // d/8 vectors of 8 bf16
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * vec_per_row) return;
-  const long long row = idx / vec_per_row;
-  const int m0 = (int)(idx % vec_per_row) * 4;
-  const int p = (int)(row % n);
-  uint4 in = src[idx];
-  const float4* tab = reinterpret_cast<const float4*>(table + (long long)p * M + m0);
-  const float4 t01 = tab[0], t23 = tab[1];
-  const float c[4] = {t01.x, t01.z, t23.x, t23.z};
-  const float s[4] = {t01.y, t01.w, t23.y, t23.w};
-  uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  const long long total = rows * vec_per_row;
+  const long long base = (long long)blockIdx.x * blockDim.x * kRotUnroll + threadIdx.x;
+  uint4 in[kRotUnroll];
+  float4 t01[kRotUnroll], t23[kRotUnroll];
+#pragma unroll
+  for (int u = 0; u < kRotUnroll; ++u) {
+    const long long idx = base + (long long)u * blockDim.x;
+    if (idx < total) {
+      const long long row = idx / vec_per_row;
+      const int m0 = (int)(idx % vec_per_row) * 4;
+      const int p = (int)(row % n);
+      in[u] = src[idx];
+      const float4* tab = reinterpret_cast<const float4*>(table + (long long)p * M + m0);
+      t01[u] = tab[0];
+      t23[u] = tab[1];
+    }
+  }
   float amax = 0.f;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
-    const float x0 = __low2float(pr), x1 = __high2float(pr);
-    const float y0 = c[j] * x0 - s[j] * x1, y1 = s[j] * x0 + c[j] * x1;
-    amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
-    uint32_t h;
-    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(y1), "f"(y0));
-    w[j] = h;
+  for (int u = 0; u < kRotUnroll; ++u) {
+    const long long idx = base + (long long)u * blockDim.x;
+    if (idx >= total) break;
+    const float c[4] = {t01[u].x, t01[u].z, t23[u].x, t23[u].z};
+    const float s[4] = {t01[u].y, t01[u].w, t23[u].y, t23[u].w};
+    uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162*>(&w[j]);
+      const float x0 = __low2float(pr), x1 = __high2float(pr);
+      const float y0 = c[j] * x0 - s[j] * x1, y1 = s[j] * x0 + c[j] * x1;
+      amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
+      uint32_t h;
+      asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(y1), "f"(y0));
+      w[j] = h;
+    }
+    dst[idx] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  dst[idx] = make_uint4(w[0], w[1], w[2], w[3]);
   if (!(amax <= 65504.f)) atomicCAS(err, 0u, 6u);  // also catches NaN
 }
 
@@ -438,7 +456,8 @@ cudaError_t launch_rotate(const ra_problem& p, const void* q, const void* k, voi
   const int threads = 256;
   if (p.dtype == RA_BF16) {  // d in {64, 128}: M is a multiple of 4
     const long long total = rows * (M / 4);
-    dim3 grid((unsigned)((total + threads - 1) / threads), 2);
+    const long long per_block = (long long)threads * kRotUnroll;
+    dim3 grid((unsigned)((total + per_block - 1) / per_block), 2);
     rotate_bf16x8_kernel<<<grid, threads, 0, s>>>((const uint4*)q, (const uint4*)k,
                                                   (uint4*)qt, (uint4*)kt, table, rows,
                                                   (int)p.n, M, err);

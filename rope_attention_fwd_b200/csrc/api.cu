@@ -164,6 +164,19 @@ uint64_t wait_limit_ns() {
   return (uint64_t)(ms * 1e6);
 }
 
+bool tensor_map_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t chunks,
+                     uint64_t row_bytes, uint32_t box_rows, uint32_t box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)chunks};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, 128};
+  const cuuint32_t box[3] = {64, box_rows, box_chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();

@@ -16,6 +16,13 @@ struct GemmSpec {
   int M, N, K;
   int a_mn, a_seg_k, a_seg_len, a_nseg;
   int b_mn, b_seg_k, b_seg_len, b_nseg;
+  // MN-major B given as 3-D whole-row views (tensor_map_rows: x = 64 columns of a chunk,
+  // y = K row, z = 64-column chunk), each 256-column tile one request; only for segments
+  // along N whose length is a multiple of 256.  0: one 2-D 64 x 64 box per chunk.
+  int b_rowbox = 0;
+  // MN-major A (one segment) given as a tensor_map_rows view, each 128-column tile one
+  // request (the MN extent a multiple of 64).
+  int a_rowbox = 0;
 };
 
 enum GemmOutKind { GEMM_OUT_F32 = 0, GEMM_OUT_HEADS = 1 };
@@ -31,8 +38,9 @@ struct GemmOut {
   int n, H, d;
 };
 
-// bf16 operands on the tensor cores; amaps / bmaps hold one 2-D tensor map per segment
-// (bf16, 128-byte swizzle; boxes: K-major A 64 x 128, every other 64 x 64).
+// bf16 operands on the tensor cores; amaps / bmaps hold one tensor map per segment (bf16,
+// 128-byte swizzle; 2-D boxes: K-major A 64 x 128, every other 64 x 64; with b_rowbox the
+// B maps are tensor_map_rows views).
 cudaError_t launch_gemm_bf16(const GemmSpec& spec, const CUtensorMap* amaps,
                              const CUtensorMap* bmaps, const GemmOut& out, uint32_t* err,
                              uint64_t wait_ns, cudaStream_t s);

@@ -146,6 +146,8 @@ __global__ void __launch_bounds__(GTHREADS, 1)
           if (!spec.a_seg_k) kl = k0;
           if (!spec.a_mn) {
             tma_load_2d(st, &amaps.map[as], &bar[GB_FULL + s], kl, m0);
+          } else if (spec.a_rowbox) {
+            tma_load_3d(st, &amaps.map[as], &bar[GB_FULL + s], 0, kl, m0 / 64);
           } else {
             for (int c = 0; c < 2; ++c)  // two 64-column (M) chunks of 64 K-rows
               tma_load_2d(st + c * 8192, &amaps.map[as], &bar[GB_FULL + s], m0 + 64 * c, kl);
@@ -153,6 +155,12 @@ __global__ void __launch_bounds__(GTHREADS, 1)
           // B: 256 columns (N) in four 64-wide chunks, each inside one N segment (or the K
           // segment of this chunk)
           uint8_t* sb = st + GA_BYTES;
+          if (spec.b_mn && spec.b_rowbox) {
+            // the tile's 64 K rows x 256 columns (one N segment) in one request
+            int nl = n0;
+            const int bs = seg_of(n0, spec.b_seg_len, spec.b_nseg, &nl);
+            tma_load_3d(sb, &bmaps.map[bs], &bar[GB_FULL + s], 0, k0, nl / 64);
+          } else
           for (int c = 0; c < 4; ++c) {
             const int nc = n0 + 64 * c;
             int nl = nc, kbl = k0, bs = 0;

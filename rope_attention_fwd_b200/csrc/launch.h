@@ -12,6 +12,12 @@ uint64_t wait_limit_ns();
 
 // A 2-D row-major tensor map (inner x outer elements, rows row_bytes apart), 128-byte
 // swizzle, box box_inner x box_outer; false if the driver rejects it.
+// bf16 row-major [rows][row_elems] tensor viewed as (x = 64 columns of a chunk, y = row,
+// z = 64-column chunk), the chunk stride (128 B) below the row stride; box {64, box_rows,
+// box_chunks} is box_rows whole row segments of 64 * box_chunks columns in one request,
+// stored chunk-major in shared memory (128-byte swizzle).
+bool tensor_map_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t chunks,
+                     uint64_t row_bytes, uint32_t box_rows, uint32_t box_chunks);
 bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 

@@ -16,13 +16,14 @@ struct GemmSpec {
   int M, N, K;
   int a_mn, a_seg_k, a_seg_len, a_nseg;
   int b_mn, b_seg_k, b_seg_len, b_nseg;
-  // MN-major B given as 3-D whole-row views (tensor_map_rows: x = 64 columns of a chunk,
-  // y = K row, z = 64-column chunk), each 256-column tile one request; only for segments
-  // along N whose length is a multiple of 256.  0: one 2-D 64 x 64 box per chunk.
-  int b_rowbox = 0;
-  // MN-major A (one segment) given as a tensor_map_rows view, each 128-column tile one
-  // request (the MN extent a multiple of 64).
+  // K chunk of one pipeline stage of the tensor-core kernel: 64 (four stages) or 128 (two).
+  int bk = 64;
+  // Operand given as a 3-D whole-row view (tensor_map_rows: x = 64 columns of a chunk, y = row,
+  // z = 64-column chunk), so that one request brings the operand's whole stage: MN-major
+  // y = K row, z = MN chunk (B only for segments along N whose length is a multiple of 256);
+  // K-major y = MN row, z = K chunk (segments along K a multiple of bk long).  0: 2-D maps.
   int a_rowbox = 0;
+  int b_rowbox = 0;
 };
 
 enum GemmOutKind { GEMM_OUT_F32 = 0, GEMM_OUT_HEADS = 1 };
@@ -38,9 +39,14 @@ struct GemmOut {
   int n, H, d;
 };
 
-// bf16 operands on the tensor cores; amaps / bmaps hold one tensor map per segment (bf16,
-// 128-byte swizzle; 2-D boxes: K-major A 64 x 128, every other 64 x 64; with b_rowbox the
-// B maps are tensor_map_rows views).
+// Tensor map of one bf16 operand segment with the box the tensor-core kernel loads under
+// spec (bk, majorness, rowbox flag): ptr is row-major [rows][cols] (cols = K for a K-major
+// operand, MN for an MN-major one), rows 16-byte aligned, cols a multiple of 64 for a rowbox
+// view.  False if the map cannot be encoded.
+bool gemm_operand_map(CUtensorMap* map, const GemmSpec& spec, bool is_b, const void* ptr,
+                      uint64_t rows, uint64_t cols);
+
+// bf16 operands on the tensor cores; amaps / bmaps hold one gemm_operand_map per segment.
 cudaError_t launch_gemm_bf16(const GemmSpec& spec, const CUtensorMap* amaps,
                              const CUtensorMap* bmaps, const GemmOut& out, uint32_t* err,
                              uint64_t wait_ns, cudaStream_t s);

@@ -13,8 +13,9 @@
 // every 64-wide TMA box falls inside one tensor and picks its own tensor map.
 //
 // Tensor-core kernel: persistent, one CTA per SM, 128 x 256 output tiles, K in chunks of 64
-// through a 4-stage TMA ring (48 KB a stage), two 256-column TMEM accumulators so that the
-// epilogue of one tile runs under the main loop of the next.  6 warps:
+// through a 4-stage TMA ring (48 KB a stage) or of 128 through a 2-stage one (96 KB a stage),
+// two 256-column TMEM accumulators so that the epilogue of one tile runs under the main loop
+// of the next.  6 warps:
 //   warp 0      TMA producer;
 //   warp 1      TMEM allocator and MMA issuer (M = 128, N = 256, K = 16 per instruction;
 //               A and B K-major or MN-major straight from the TMA layout);
@@ -28,21 +29,32 @@
 
 #include "common.h"
 #include "gemm.h"
+#include "launch.h"
 #include "sm100.cuh"
 
 namespace ra {
 namespace {
 
-constexpr int GBM = 128, GBN = 256, GBK = 64, GNS = 4;
-constexpr uint32_t GA_BYTES = GBM * GBK * 2;   // 16 KB
-constexpr uint32_t GB_BYTES = GBN * GBK * 2;   // 32 KB
-constexpr uint32_t GSTAGE = GA_BYTES + GB_BYTES;
-constexpr uint32_t GOFF_EPI = GNS * GSTAGE;            // 4 epilogue warps x 32 rows x 144 B
-constexpr uint32_t GEPI_ROW = 144;                     // 32 fp32 + 16 B pad
+constexpr int GBM = 128, GBN = 256;
+constexpr uint32_t GEPI_ROW = 144;  // 32 fp32 + 16 B pad
 constexpr uint32_t GEPI_WARP = 32 * GEPI_ROW;
-constexpr uint32_t GOFF_BAR = GOFF_EPI + 4 * GEPI_WARP;
-constexpr uint32_t GSMEM = GOFF_BAR + 256 + 1024;
 constexpr int GTHREADS = 192;
+
+// Shared-memory plan for a K chunk of BK per pipeline stage: 64 (four 48 KB stages) or 128
+// (two 96 KB stages).  With 128 a K-major row piece of a tile is 256 contiguous bytes, which
+// streams from L2 much faster than 128-byte pieces; 64 keeps more stages in flight.
+template <int BK>
+struct GemmCfg {
+  static constexpr int KH = BK / 64;                      // 64-wide K halves per stage
+  static constexpr int NS = BK == 64 ? 4 : 2;             // stages
+  static constexpr uint32_t A_BYTES = GBM * BK * 2;
+  static constexpr uint32_t B_BYTES = GBN * BK * 2;
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  static constexpr uint32_t MN_CHUNK = BK * 128;          // one 64-wide MN-major chunk
+  static constexpr uint32_t OFF_EPI = NS * STAGE;         // 4 epilogue warps x 32 rows x 144 B
+  static constexpr uint32_t OFF_BAR = OFF_EPI + 4 * GEPI_WARP;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+};
 constexpr int KID_GEMM = K_PROJ_GEMM;
 
 enum GemmBar {
@@ -90,21 +102,24 @@ __device__ __forceinline__ void write_row_chunk(const GemmOut& out, int m, int c
   }
 }
 
+template <int BK>
 __global__ void __launch_bounds__(GTHREADS, 1)
     gemm_bf16_kernel(const __grid_constant__ SegMaps amaps, const __grid_constant__ SegMaps bmaps,
                      GemmSpec spec, GemmOut out, uint32_t* err, uint64_t wait_ns) {
+  using C = GemmCfg<BK>;
+  constexpr int GNS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base_s = (raw_s + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_s - raw_s);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(base + GOFF_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + GOFF_BAR + 8 * GB_COUNT);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + GOFF_BAR + 8 * GB_COUNT + 4);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::OFF_BAR + 8 * GB_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + C::OFF_BAR + 8 * GB_COUNT + 4);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   const int tiles_m = (spec.M + GBM - 1) / GBM, tiles_n = (spec.N + GBN - 1) / GBN;
   const int tiles = tiles_m * tiles_n;
-  const int kchunks = (spec.K + GBK - 1) / GBK;
+  const int kchunks = (spec.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < GB_COUNT; ++i)
@@ -137,39 +152,61 @@ __global__ void __launch_bounds__(GTHREADS, 1)
             ok = false;
             break;
           }
-          uint8_t* st = base + s * GSTAGE;
-          mbar_arrive_expect_tx(&bar[GB_FULL + s], GSTAGE);
-          const int k0 = kc * GBK;
-          // A: 128 rows (M) x 64 K; segmented along K (dX) or not at all
-          int kl = 0;
-          const int as = spec.a_seg_k ? seg_of(k0, spec.a_seg_len, spec.a_nseg, &kl) : 0;
-          if (!spec.a_seg_k) kl = k0;
+          uint8_t* st = base + s * C::STAGE;
+          mbar_arrive_expect_tx(&bar[GB_FULL + s], C::STAGE);
+          const int k0 = kc * BK;
+          uint64_t* fb = &bar[GB_FULL + s];
+          // A: 128 M x BK, as [K half][128 rows][64] (K-major) or [M chunk][BK K rows][64]
+          // (MN-major)
           if (!spec.a_mn) {
-            tma_load_2d(st, &amaps.map[as], &bar[GB_FULL + s], kl, m0);
-          } else if (spec.a_rowbox) {
-            tma_load_3d(st, &amaps.map[as], &bar[GB_FULL + s], 0, kl, m0 / 64);
+            if (spec.a_rowbox) {
+              int kl = k0;
+              const int as = spec.a_seg_k ? seg_of(k0, spec.a_seg_len, spec.a_nseg, &kl) : 0;
+              tma_load_3d(st, &amaps.map[as], fb, 0, m0, kl / 64);
+            } else {
+              for (int h = 0; h < C::KH; ++h) {
+                int kl = k0 + 64 * h;
+                const int as = spec.a_seg_k ? seg_of(kl, spec.a_seg_len, spec.a_nseg, &kl) : 0;
+                tma_load_2d(st + h * 16384, &amaps.map[as], fb, kl, m0);
+              }
+            }
           } else {
-            for (int c = 0; c < 2; ++c)  // two 64-column (M) chunks of 64 K-rows
-              tma_load_2d(st + c * 8192, &amaps.map[as], &bar[GB_FULL + s], m0 + 64 * c, kl);
-          }
-          // B: 256 columns (N) in four 64-wide chunks, each inside one N segment (or the K
-          // segment of this chunk)
-          uint8_t* sb = st + GA_BYTES;
-          if (spec.b_mn && spec.b_rowbox) {
-            // the tile's 64 K rows x 256 columns (one N segment) in one request
-            int nl = n0;
-            const int bs = seg_of(n0, spec.b_seg_len, spec.b_nseg, &nl);
-            tma_load_3d(sb, &bmaps.map[bs], &bar[GB_FULL + s], 0, k0, nl / 64);
-          } else
-          for (int c = 0; c < 4; ++c) {
-            const int nc = n0 + 64 * c;
-            int nl = nc, kbl = k0, bs = 0;
-            if (spec.b_seg_k) bs = seg_of(k0, spec.b_seg_len, spec.b_nseg, &kbl);
-            else bs = seg_of(nc, spec.b_seg_len, spec.b_nseg, &nl);
-            if (!spec.b_mn)
-              tma_load_2d(sb + c * 8192, &bmaps.map[bs], &bar[GB_FULL + s], kbl, nl);
+            int kl = k0;
+            const int as = spec.a_seg_k ? seg_of(k0, spec.a_seg_len, spec.a_nseg, &kl) : 0;
+            if (spec.a_rowbox)
+              tma_load_3d(st, &amaps.map[as], fb, 0, kl, m0 / 64);
             else
-              tma_load_2d(sb + c * 8192, &bmaps.map[bs], &bar[GB_FULL + s], nl, kbl);
+              for (int c = 0; c < 2; ++c)
+                tma_load_2d(st + c * C::MN_CHUNK, &amaps.map[as], fb, m0 + 64 * c, kl);
+          }
+          // B: 256 N x BK, as [K half][256 rows][64] (K-major) or [N chunk][BK K rows][64]
+          // (MN-major), each piece inside one segment
+          uint8_t* sb = st + C::A_BYTES;
+          if (spec.b_rowbox) {
+            int nl = n0, kbl = k0, bs = 0;
+            if (spec.b_seg_k) bs = seg_of(k0, spec.b_seg_len, spec.b_nseg, &kbl);
+            else bs = seg_of(n0, spec.b_seg_len, spec.b_nseg, &nl);
+            if (spec.b_mn)
+              tma_load_3d(sb, &bmaps.map[bs], fb, 0, kbl, nl / 64);
+            else
+              tma_load_3d(sb, &bmaps.map[bs], fb, 0, nl, kbl / 64);
+          } else if (spec.b_mn) {
+            for (int c = 0; c < 4; ++c) {
+              const int nc = n0 + 64 * c;
+              int nl = nc, kbl = k0, bs = 0;
+              if (spec.b_seg_k) bs = seg_of(k0, spec.b_seg_len, spec.b_nseg, &kbl);
+              else bs = seg_of(nc, spec.b_seg_len, spec.b_nseg, &nl);
+              tma_load_2d(sb + c * C::MN_CHUNK, &bmaps.map[bs], fb, nl, kbl);
+            }
+          } else {
+            for (int h = 0; h < C::KH; ++h)
+              for (int c = 0; c < 4; ++c) {
+                const int nc = n0 + 64 * c;
+                int nl = nc, kbl = k0 + 64 * h, bs = 0;
+                if (spec.b_seg_k) bs = seg_of(kbl, spec.b_seg_len, spec.b_nseg, &kbl);
+                else bs = seg_of(nc, spec.b_seg_len, spec.b_nseg, &nl);
+                tma_load_2d(sb + h * 32768 + c * 8192, &bmaps.map[bs], fb, kbl, nl);
+              }
           }
           issued = it;
         }
@@ -183,12 +220,14 @@ __global__ void __launch_bounds__(GTHREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t idesc = idesc_bf16_f32(GBM, GBN, spec.a_mn, spec.b_mn);
-    // K-major: one 128 B row per M / N row, +32 B per K-step; MN-major: 64-wide chunks 8 KB
-    // apart (LBO), +2048 B (16 K-rows) per K-step
-    const SDesc da = spec.a_mn ? sdesc_split(base_s, 8192, 1024) : sdesc_split(base_s, 16, 1024);
-    const SDesc db = spec.b_mn ? sdesc_split(base_s + GA_BYTES, 8192, 1024)
-                               : sdesc_split(base_s + GA_BYTES, 16, 1024);
+    // K-major: one 128 B row per M / N row, +32 B per K-step, a second K half one half-tile
+    // on; MN-major: 64-wide chunks MN_CHUNK apart (LBO), +2048 B (16 K-rows) per K-step
+    const SDesc da =
+        spec.a_mn ? sdesc_split(base_s, C::MN_CHUNK, 1024) : sdesc_split(base_s, 16, 1024);
+    const SDesc db = spec.b_mn ? sdesc_split(base_s + C::A_BYTES, C::MN_CHUNK, 1024)
+                               : sdesc_split(base_s + C::A_BYTES, 16, 1024);
     const uint32_t astep = spec.a_mn ? 2048u : 32u, bstep = spec.b_mn ? 2048u : 32u;
+    const uint32_t ahalf = spec.a_mn ? 8192u : 16384u, bhalf = spec.b_mn ? 8192u : 32768u;
     int it = 0, tl = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tl) {
@@ -208,9 +247,11 @@ __global__ void __launch_bounds__(GTHREADS, 1)
           break;
         }
         tc_fence_after();
-        const SDesc sa = sdesc_advance(da, s * GSTAGE), sb = sdesc_advance(db, s * GSTAGE);
-        mma4_ss(tmem + acc * 256, sdesc_at(sa, 0), sdesc_at(sb, 0), idesc, kc > 0 ? 1u : 0u,
-                astep >> 4, bstep >> 4);
+        const SDesc sa = sdesc_advance(da, s * C::STAGE), sb = sdesc_advance(db, s * C::STAGE);
+#pragma unroll
+        for (int h = 0; h < C::KH; ++h)
+          mma4_ss(tmem + acc * 256, sdesc_at(sa, h * ahalf), sdesc_at(sb, h * bhalf), idesc,
+                  kc > 0 || h > 0 ? 1u : 0u, astep >> 4, bstep >> 4);
         mma_commit_warp(&bar[GB_EMPTY + s]);
       }
       if (ok) mma_commit_warp(&bar[GB_ACC_FULL + acc]);
@@ -222,7 +263,7 @@ __global__ void __launch_bounds__(GTHREADS, 1)
     // ------------------------------------------------------------ epilogue warps 2-5
     const int q = warp % 4;  // TMEM lane quarter == row quarter of the tile
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    uint8_t* stage = base + GOFF_EPI + (warp - 2) * GEPI_WARP;
+    uint8_t* stage = base + C::OFF_EPI + (warp - 2) * GEPI_WARP;
     int tl = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
       const int acc = tl & 1;
@@ -363,11 +404,27 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
+bool gemm_operand_map(CUtensorMap* map, const GemmSpec& spec, bool is_b, const void* ptr,
+                      uint64_t rows, uint64_t cols) {
+  const bool mn = is_b ? spec.b_mn : spec.a_mn, rowbox = is_b ? spec.b_rowbox : spec.a_rowbox;
+  const uint32_t tile_mn = is_b ? GBN : GBM, bk = (uint32_t)spec.bk;
+  if (rowbox) {
+    if (cols % 64 != 0) return false;
+    return mn ? tensor_map_rows(map, ptr, rows, cols / 64, cols * 2, bk, tile_mn / 64)
+              : tensor_map_rows(map, ptr, rows, cols / 64, cols * 2, tile_mn, bk / 64);
+  }
+  // 2-D: MN-major 64 columns x bk K rows; K-major A 64 K x 128 rows, K-major B 64 K x 64 rows
+  return tensor_map_2d(map, ptr, false, cols, rows, cols * 2, 64,
+                       mn ? bk : (is_b ? 64u : 128u));
+}
+
 cudaError_t launch_gemm_bf16(const GemmSpec& spec, const CUtensorMap* amaps,
                              const CUtensorMap* bmaps, const GemmOut& out, uint32_t* err,
                              uint64_t wait_ns, cudaStream_t s) {
-  cudaError_t e =
-      cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GSMEM);
+  if (spec.bk != 64 && spec.bk != 128) return cudaErrorInvalidValue;
+  const auto kernel = spec.bk == 64 ? gemm_bf16_kernel<64> : gemm_bf16_kernel<128>;
+  const uint32_t smem = spec.bk == 64 ? GemmCfg<64>::SMEM : GemmCfg<128>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   SegMaps a{}, b{};
   for (int i = 0; i < spec.a_nseg; ++i) a.map[i] = amaps[i];
@@ -378,7 +435,7 @@ cudaError_t launch_gemm_bf16(const GemmSpec& spec, const CUtensorMap* amaps,
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = (long long)((spec.M + GBM - 1) / GBM) * ((spec.N + GBN - 1) / GBN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  gemm_bf16_kernel<<<grid, GTHREADS, GSMEM, s>>>(a, b, spec, out, err, wait_ns);
+  kernel<<<grid, GTHREADS, smem, s>>>(a, b, spec, out, err, wait_ns);
   return cudaGetLastError();
 }
 

@@ -83,6 +83,7 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
   const int rows = (int)(p->B * p->n), hd = (int)(p->H * p->d), dm = (int)d_model;
   // C[B n][3 H d] = X [W_Q | W_K | W_V]: A = X K-major, B = W MN-major (segmented along N)
   ra::GemmSpec spec{rows, 3 * hd, dm, 0, 0, 0, 1, 1, 0, hd, 3};
+  spec.bk = 64;  // four stages in flight: both operands already stream as whole rows
   spec.b_rowbox = hd % 256 == 0;
   const ra::GemmOut out{{q, k, v}, ra::GEMM_OUT_HEADS, hd, 3, 0, (int)p->n, (int)p->H,
                         (int)p->d};
@@ -90,13 +91,9 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
   cudaError_t e;
   if (p->dtype == RA_BF16) {
     CUtensorMap am[1], bm[3];
-    if (!ra::tensor_map_2d(&am[0], x, false, dm, rows, (uint64_t)dm * 2, 64, 128))
-      return RA_ERR_CUDA;
+    if (!ra::gemm_operand_map(&am[0], spec, false, x, rows, dm)) return RA_ERR_CUDA;
     for (int w = 0; w < 3; ++w)
-      if (!(spec.b_rowbox
-                ? ra::tensor_map_rows(&bm[w], W[w], dm, hd / 64, (uint64_t)hd * 2, 64, 4)
-                : ra::tensor_map_2d(&bm[w], W[w], false, hd, dm, (uint64_t)hd * 2, 64, 64)))
-        return RA_ERR_CUDA;
+      if (!ra::gemm_operand_map(&bm[w], spec, true, W[w], dm, hd)) return RA_ERR_CUDA;
     e = ra::launch_gemm_bf16(spec, am, bm, out, static_cast<uint32_t*>(ws), ra::wait_limit_ns(),
                              s);
   } else {
@@ -133,29 +130,28 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
   // [dW_Q | dW_K | dW_V] (d_model x 3 H d) = X^T [Y_Q | Y_K | Y_V]: A = X MN-major,
   // B = Y MN-major segmented along N; K = B n
   ra::GemmSpec sw{dm, 3 * hd, rows, 1, 0, 0, 1, 1, 0, hd, 3};
-  sw.b_rowbox = hd % 256 == 0;
+  sw.bk = 64;
   sw.a_rowbox = dm % 64 == 0;
+  sw.b_rowbox = hd % 256 == 0;
   const ra::GemmOut ow{{dwq, dwk, dwv}, ra::GEMM_OUT_F32, hd, 3, hd, 0, 0, 0};
   // dX (B n x d_model) = [Y_Q | Y_K | Y_V] [W_Q | W_K | W_V]^T: A = Y K-major segmented along
   // K, B = W K-major ([d_model][H d] rows) segmented along K; K = 3 H d
-  const ra::GemmSpec sx{rows, dm, 3 * hd, 0, 1, hd, 3, 0, 1, hd, 3};
+  ra::GemmSpec sx{rows, dm, 3 * hd, 0, 1, hd, 3, 0, 1, hd, 3};
+  // K-major operands: 128-wide K chunks make every row piece 256 contiguous bytes
+  sx.bk = 128;
+  sx.a_rowbox = sx.b_rowbox = hd % 128 == 0;
   const ra::GemmOut ox{{dx, dx, dx}, ra::GEMM_OUT_F32, dm, 1, dm, 0, 0, 0};
   cudaError_t e;
   if (p->dtype == RA_BF16) {
     uint32_t* err = static_cast<uint32_t*>(ws);
     const uint64_t wait = ra::wait_limit_ns();
     CUtensorMap xa[1], yb[3], ya[3], wb[3];
-    if (!(sw.a_rowbox ? ra::tensor_map_rows(&xa[0], x, rows, dm / 64, (uint64_t)dm * 2, 64, 2)
-                      : ra::tensor_map_2d(&xa[0], x, false, dm, rows, (uint64_t)dm * 2, 64, 64)))
-      return RA_ERR_CUDA;
-    for (int w = 0; w < 3; ++w) {
-      if (!(sw.b_rowbox
-                ? ra::tensor_map_rows(&yb[w], Y[w], rows, hd / 64, (uint64_t)hd * 2, 64, 4)
-                : ra::tensor_map_2d(&yb[w], Y[w], false, hd, rows, (uint64_t)hd * 2, 64, 64)) ||
-          !ra::tensor_map_2d(&ya[w], Y[w], false, hd, rows, (uint64_t)hd * 2, 64, 128) ||
-          !ra::tensor_map_2d(&wb[w], W[w], false, hd, dm, (uint64_t)hd * 2, 64, 64))
+    if (!ra::gemm_operand_map(&xa[0], sw, false, x, rows, dm)) return RA_ERR_CUDA;
+    for (int w = 0; w < 3; ++w)
+      if (!ra::gemm_operand_map(&yb[w], sw, true, Y[w], rows, hd) ||
+          !ra::gemm_operand_map(&ya[w], sx, false, Y[w], rows, hd) ||
+          !ra::gemm_operand_map(&wb[w], sx, true, W[w], dm, hd))
         return RA_ERR_CUDA;
-    }
     e = ra::launch_gemm_bf16(sw, xa, yb, ow, err, wait, s);
     if (e == cudaSuccess) e = ra::launch_gemm_bf16(sx, ya, wb, ox, err, wait, s);
   } else {

@@ -447,35 +447,23 @@ def run_profile(args):
                   for _ in range(4))
     alpha = 0.3 * torch.randn(d // 2, device="cuda", generator=g)
     ws = rb.workspace(rb.problem(B, H, n, d, torch.bfloat16, args.causal, args.base), "cuda")
-    proj_ms = {"proj_fwd": 0.0, "proj_bwd": 0.0}
     if args.d_model > 0:
         x = torch.randn((B, n, args.d_model), device="cuda", generator=g).to(torch.bfloat16)
         w = [(torch.randn((args.d_model, H * d), device="cuda", generator=g)
               * args.d_model ** -0.5).to(torch.bfloat16) for _ in range(3)]
 
-    def timed(name, fn):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        out = fn()
-        e1.record()
-        e1.synchronize()
-        proj_ms[name] += e0.elapsed_time(e1)
-        return out
-
     def step():
-        qq, kk, vv = (q, k, v) if args.d_model <= 0 else timed(
-            "proj_fwd", lambda: rb.rope_attn_proj_fwd(x, *w, H))
+        qq, kk, vv = (q, k, v) if args.d_model <= 0 else rb.rope_attn_proj_fwd(x, *w, H)
         o, lse = rb.rope_attn_fwd(qq, kk, vv, alpha, args.base, args.causal, ws=ws)
         L, dO = rb.rope_attn_loss(o, e, ws=ws)
         grads = rb.rope_attn_bwd_saved(vv, o, lse, dO, alpha, args.base, args.causal, ws)
         if args.d_model > 0:
-            timed("proj_bwd", lambda: rb.rope_attn_proj_bwd(x, *w, *grads[:3]))
+            rb.rope_attn_proj_bwd(x, *w, *grads[:3])
         return grads
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    proj_ms = {k2: 0.0 for k2 in proj_ms}
     rb.rope_attn_timing_read()
     rb.rope_attn_timing_enable(True)
     for _ in range(args.steps):
@@ -484,16 +472,21 @@ def run_profile(args):
     rb.rope_attn_timing_enable(False)
     f = 0.5 if args.causal else 1.0
     alg = {"fwd_sm100": 4.0, "bwd_dkdv_sm100": 8.0, "bwd_dq_sm100": 2.0}
-    for name, (cnt, ms) in rb.rope_attn_timing_read().items():
+    kernels = rb.rope_attn_timing_read()
+    prod = 2.0 * B * n * max(args.d_model, 0) * H * d  # FLOPs of one x W product
+    for name, (cnt, ms) in kernels.items():
         line = f"{name:16s} {cnt:3d} launches {ms / cnt:8.3f} ms"
         if name in alg:
             tf = alg[name] * B * H * n * n * d * f / (ms / cnt * 1e-3) / 1e12
             line += f"  {tf:7.1f} TFLOP/s algorithmic"
+        elif name in ("proj_gemm", "proj_dw_gemm", "proj_dx_gemm"):
+            line += f"  {3 * prod / (ms / cnt * 1e-3) / 1e12:7.1f} TFLOP/s"
         print(line)
     if args.d_model > 0:
-        prod = 2.0 * B * n * args.d_model * H * d  # FLOPs of one x W product
+        parts = {"proj_fwd": ("proj_gemm",),
+                 "proj_bwd": ("merge_heads", "proj_dw_gemm", "proj_dx_gemm")}
         for name, nprod in (("proj_fwd", 3), ("proj_bwd", 6)):
-            ms = proj_ms[name] / args.steps
+            ms = sum(kernels.get(kn, (0, 0.0))[1] for kn in parts[name]) / args.steps
             print(f"{name:16s}   1 launches {ms:8.3f} ms  "
                   f"{nprod * prod / (ms * 1e-3) / 1e12:7.1f} TFLOP/s")
     code, info = rb.rope_attn_device_status(ws)

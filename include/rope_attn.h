@@ -253,7 +253,8 @@ ra_status rope_attn_noalloc_status(void* stream, int32_t info[3]);
 
 /* ---- optional per-kernel timing (instrumentation, off by default) --------
  * While enabled, every kernel launch made by the calls above is bracketed by
- * CUDA events on the caller's stream.  rope_attn_timing_read synchronises
+ * CUDA events on the caller's stream (rope_attn_spectrum: its whole sequence
+ * of launches as one).  rope_attn_timing_read synchronises
  * those events and writes, per kernel id, the number of launches and the sum
  * of their durations in milliseconds; it returns the number of kernel ids
  * (at most max_ids) and clears the record. */

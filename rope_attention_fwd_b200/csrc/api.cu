@@ -38,25 +38,38 @@ cudaEvent_t take_event() {
   return e;
 }
 
+}  // namespace
+
+namespace ra {
+
+cudaEvent_t timing_begin(cudaStream_t s) {
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  if (!g_timing) return nullptr;
+  cudaEvent_t start = take_event();
+  cudaEventRecord(start, s);
+  return start;
+}
+
+void timing_end(cudaEvent_t start, int kid, cudaStream_t s) {
+  if (!start) return;
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  cudaEvent_t stop = take_event();
+  cudaEventRecord(stop, s);
+  g_timed.push_back({kid, start, stop});
+}
+
+}  // namespace ra
+
+namespace {
+
 struct LaunchScope {
   int kid;
   cudaStream_t s;
-  cudaEvent_t start = nullptr;
-  LaunchScope(int k, cudaStream_t st) : kid(k), s(st) {
-    if (g_timing) {
-      std::lock_guard<std::mutex> g(g_timing_mu);
-      start = take_event();
-      cudaEventRecord(start, s);
-    }
-  }
+  cudaEvent_t start;
+  LaunchScope(int k, cudaStream_t st) : kid(k), s(st), start(timing_begin(st)) {}
   void done() {
-    if (start) {
-      std::lock_guard<std::mutex> g(g_timing_mu);
-      cudaEvent_t stop = take_event();
-      cudaEventRecord(stop, s);
-      g_timed.push_back({kid, start, stop});
-      start = nullptr;
-    }
+    timing_end(start, kid, s);
+    start = nullptr;
   }
 };
 
@@ -360,9 +373,9 @@ ra_status rope_attn_alpha_adam(const ra_adam* opt, int64_t count, float* alpha,
   const float bc1 = (float)(1.0 - std::pow((double)opt->beta1, (double)opt->step));
   const float bc2 = (float)(1.0 - std::pow((double)opt->beta2, (double)opt->step));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_alpha_adam(alpha, dalpha, m1, m2, count, opt->lr, opt->beta1, opt->beta2, opt->eps,
-                        opt->clip_norm, bc1, bc2, s) != cudaSuccess)
-    return RA_ERR_CUDA;
+  RA_LAUNCH(K_ALPHA_ADAM, s,
+            launch_alpha_adam(alpha, dalpha, m1, m2, count, opt->lr, opt->beta1, opt->beta2,
+                              opt->eps, opt->clip_norm, bc1, bc2, s));
   return RA_OK;
 }
 
@@ -423,7 +436,8 @@ const char* rope_attn_kernel_name(int id) {
       "rope_table",       "rotate",       "fwd_f32",      "fwd_sm100",
       "loss_partial",     "loss_final",   "bwd_delta",    "bwd_dq_f32",
       "bwd_dkdv_f32",     "bwd_dq_sm100", "bwd_dkdv_sm100", "dalpha_final",
-      "proj_gemm"};
+      "proj_gemm",        "proj_dw_gemm", "proj_dx_gemm", "merge_heads",
+      "spectrum",         "alpha_adam"};
   return (id >= 0 && id < K_COUNT) ? names[id] : "unknown";
 }
 

@@ -21,8 +21,13 @@ enum KernelId : int {
   K_BWD_DQ_SM100 = 9,
   K_BWD_DKDV_SM100 = 10,
   K_DALPHA = 11,
-  K_PROJ_GEMM = 12,
-  K_COUNT = 13
+  K_PROJ_GEMM = 12,  // the q / k / v product (and the GEMM kernel's id in error reports)
+  K_PROJ_DW = 13,
+  K_PROJ_DX = 14,
+  K_MERGE_HEADS = 15,
+  K_SPECTRUM = 16,
+  K_ALPHA_ADAM = 17,
+  K_COUNT = 18
 };
 
 // Rows per dalpha partial (one partial per band per tile of query or key rows).

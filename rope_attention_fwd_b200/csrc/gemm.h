@@ -21,7 +21,8 @@ struct GemmSpec {
   // Operand given as a 3-D whole-row view (tensor_map_rows: x = 64 columns of a chunk, y = row,
   // z = 64-column chunk), so that one request brings the operand's whole stage: MN-major
   // y = K row, z = MN chunk (B only for segments along N whose length is a multiple of 256);
-  // K-major y = MN row, z = K chunk (segments along K a multiple of bk long).  0: 2-D maps.
+  // K-major y = MN row, z = K chunk (bk = 128 only; segments along K a multiple of 128
+  // long).  0: 2-D maps.
   int a_rowbox = 0;
   int b_rowbox = 0;
 };

@@ -21,6 +21,12 @@ bool tensor_map_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t 
 bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, uint64_t outer,
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Per-kernel event timing (rope_attn_timing_enable).  While it is on, timing_begin records a
+// start event on s and timing_end a stop event, the pair filed under kernel id kid; while it
+// is off timing_begin returns nullptr and timing_end does nothing.
+cudaEvent_t timing_begin(cudaStream_t s);
+void timing_end(cudaEvent_t start, int kid, cudaStream_t s);
+
 struct DevCtl {
   uint32_t* err;        // workspace error word
   uint64_t wait_ns;     // bound on every device-side wait

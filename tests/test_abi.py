@@ -102,9 +102,11 @@ def test_workspace_checks_before_launch():
 
 def test_kernel_names():
     lib = rb.lib()
-    names = {lib.rope_attn_kernel_name(i).decode() for i in range(13)}
-    assert {"fwd_sm100", "bwd_dkdv_sm100", "bwd_dq_sm100", "dalpha_final",
-            "proj_gemm"} <= names
+    names = [lib.rope_attn_kernel_name(i).decode() for i in range(18)]
+    assert {"fwd_sm100", "bwd_dkdv_sm100", "bwd_dq_sm100", "dalpha_final", "proj_gemm",
+            "proj_dw_gemm", "proj_dx_gemm", "merge_heads", "spectrum", "alpha_adam"} <= set(names)
+    assert "unknown" not in names and len(set(names)) == 18
+    assert lib.rope_attn_kernel_name(18) == b"unknown"
 
 
 def test_fixed_bands_and_reserved_are_validated():

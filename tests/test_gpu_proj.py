@@ -60,3 +60,24 @@ def test_whole_layer_bf16():
     want = ref.proj_backward(to64(x), *[to64(t) for t in w], r["dq"], r["dk"], r["dv"])
     for a, b in zip(got, want):
         assert rel_frob(to64(a), b) <= TOL["bf16"]["grad"]
+
+
+def test_proj_launches_are_timed_per_product():
+    """With the library's timing on, each projection product is recorded under its own
+    kernel id: one q/k/v GEMM, three head merges, one dW and one dx GEMM per call pair."""
+    g = torch.Generator().manual_seed(5)
+    B, H, n, d, dm = 1, 2, 256, 128, 256
+    x = _rand((B, n, dm), torch.bfloat16, 1.0, g)
+    w = [_rand((dm, H * d), torch.bfloat16, 0.1, g) for _ in range(3)]
+    rb.rope_attn_timing_read()
+    rb.rope_attn_timing_enable(True)
+    try:
+        q, k, v = rb.rope_attn_proj_fwd(x, *w, H)
+        rb.rope_attn_proj_bwd(x, *w, q, k, v)
+        torch.cuda.synchronize()
+    finally:
+        rb.rope_attn_timing_enable(False)
+    rec = rb.rope_attn_timing_read()
+    assert {name: cnt for name, (cnt, _) in rec.items()} == {
+        "proj_gemm": 1, "merge_heads": 3, "proj_dw_gemm": 1, "proj_dx_gemm": 1}
+    assert all(ms > 0 for _, ms in rec.values())

@@ -96,7 +96,7 @@ __device__ __forceinline__ void stage_table(const float2* __restrict__ table, in
                                             uint8_t* dst) {
   using TS = TabStage<D>;
   constexpr int PER = 128 * TS::UNITS / kSoftThreads;  // 16-byte units per thread
-  constexpr int BATCH = PER < 8 ? PER : 8;             // loads in flight before the stores
+  constexpr int BATCH = PER < 16 ? PER : 16;           // loads in flight before the stores
   static_assert(PER * kSoftThreads == 128 * TS::UNITS && PER % BATCH == 0, "even split");
   const uint8_t* src = reinterpret_cast<const uint8_t*>(table);
 #pragma unroll
@@ -119,25 +119,37 @@ __device__ __forceinline__ void stage_table(const float2* __restrict__ table, in
   }
 }
 
-// Epilogue of one gradient row held in TMEM (D fp32 columns from tmem_acc, this
-// thread's lane): g = acc * scale is dX~ of position `pos`; writes R(-pos theta_hat) g as
-// bf16 to out_row (when live) and the band torques w * (g1 x0 - g0 x1) to red_row, where
-// x~ is row t of the 128B-swizzled fp16 tile at x_tile_s (chunk stride x_chunk) and the
-// (cos, sin) pairs of position pos are the staged table row at tab_row.
+// 32-column chunks of a gradient row that one softmax thread finishes (its half of D).
 template <int D>
-__device__ __forceinline__ void grad_row_epilogue(uint32_t tmem_acc, uint32_t x_tile_s,
-                                                  uint32_t x_chunk, int t,
+constexpr int kRowChunks = D / 32 / kSoftWG;
+
+// Issue the TMEM reads of this thread's chunks of a gradient row (D fp32 columns from
+// tmem_acc, this thread's lane); the caller waits (tmem_wait_ld on each chunk) before use.
+template <int D>
+__device__ __forceinline__ void grad_row_load(uint32_t tmem_acc, int half,
+                                              uint32_t (&ra)[kRowChunks<D>][32]) {
+#pragma unroll
+  for (int cc = 0; cc < kRowChunks<D>; ++cc)
+    tmem_ld32(tmem_acc + 32 * (half * kRowChunks<D> + cc), ra[cc]);
+}
+
+// Epilogue of one gradient row, this thread's chunks read by grad_row_load into ra:
+// g = acc * scale is dX~ of position `pos`; writes R(-pos theta_hat) g as bf16 to out_row
+// (when live) and the band torques w * (g1 x0 - g0 x1) to red_row, where x~ is row t of the
+// 128B-swizzled fp16 tile at x_tile_s (chunk stride x_chunk) and the (cos, sin) pairs of
+// position pos are the staged table row at tab_row.
+template <int D>
+__device__ __forceinline__ void grad_row_epilogue(const uint32_t (&ra)[kRowChunks<D>][32],
+                                                  uint32_t x_tile_s, uint32_t x_chunk, int t,
                                                   const uint8_t* tab_row, float scale,
                                                   float w, bool live,
                                                   __nv_bfloat16* __restrict__ out_row,
                                                   float* red_row, int half) {
-  constexpr int NC = D / 32 / kSoftWG;  // 32-column chunks of this thread
+  constexpr int NC = kRowChunks<D>;
 #pragma unroll
   for (int cc = 0; cc < NC; ++cc) {
     const int c = half * NC + cc;
-    uint32_t r[32];
-    tmem_ld32(tmem_acc + 32 * c, r);
-    tmem_wait_ld(r);
+    const uint32_t (&r)[32] = ra[cc];
     const uint32_t ch = x_tile_s + (uint32_t)((32 * c) / 64) * x_chunk;
     const int u0 = ((32 * c) % 64) / 8;
     uint32_t xw[16];
@@ -455,14 +467,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every Q~/dO stage has been consumed: the ring holds the torque buffer and the table
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);
       uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
+      // dV row (this thread's D / kSoftWG columns): its TMEM reads in flight while the
+      // table rows are staged
+      uint32_t rv[kRowChunks<D>][32];
+      grad_row_load<D>(lane_base + C::COL_DV, half, rv);
       stage_table<D>(table, jt * C::BN, n, tab);
-      // dV row (this thread's D / kSoftWG columns)
 #pragma unroll
-      for (int cc = 0; cc < D / 32 / kSoftWG; ++cc) {
-        const int c = half * (D / 32 / kSoftWG) + cc;
-        uint32_t r[32];
-        tmem_ld32(lane_base + C::COL_DV + 32 * c, r);
-        tmem_wait_ld(r);
+      for (int cc = 0; cc < kRowChunks<D>; ++cc) tmem_wait_ld(rv[cc]);
+#pragma unroll
+      for (int cc = 0; cc < kRowChunks<D>; ++cc) {
+        const int c = half * kRowChunks<D> + cc;
+        const uint32_t (&r)[32] = rv[cc];
         if (live) {
           uint4* dst = reinterpret_cast<uint4*>(dv + ((size_t)bh * n + key) * D + 32 * c);
 #pragma unroll
@@ -474,8 +489,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // dK row, its inverse rotation and the K-side torques
+      uint32_t rk[kRowChunks<D>][32];
+      grad_row_load<D>(lane_base + C::COL_DK, half, rk);
       softmax_group_sync();
-      grad_row_epilogue<D>(lane_base + C::COL_DK, base_s + C::OFF_K, C::KCH, t,
+#pragma unroll
+      for (int cc = 0; cc < kRowChunks<D>; ++cc) tmem_wait_ld(rk[cc]);
+      grad_row_epilogue<D>(rk, base_s + C::OFF_K, C::KCH, t,
                            tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
                            (float)key - 0.5f * (float)(n - 1), live,
                            dk + ((size_t)bh * n + (live ? key : 0)) * D, red + t * (D / 2 + 1),
@@ -747,9 +766,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every K~/V stage has been consumed: the ring holds the torque buffer and the table
       float* red = reinterpret_cast<float*>(base + C::OFF_ST);
       uint8_t* tab = base + C::OFF_ST + C::RED_BYTES;
+      // the dQ~ row's TMEM reads in flight while the table rows are staged
+      uint32_t rq[kRowChunks<D>][32];
+      grad_row_load<D>(lane_base + C::COL_DQ, half, rq);
       stage_table<D>(table, qtile * C::BM, n, tab);
       softmax_group_sync();
-      grad_row_epilogue<D>(lane_base + C::COL_DQ, base_s + C::OFF_Q, C::QCH, t,
+#pragma unroll
+      for (int cc = 0; cc < kRowChunks<D>; ++cc) tmem_wait_ld(rq[cc]);
+      grad_row_epilogue<D>(rq, base_s + C::OFF_Q, C::QCH, t,
                            tab + t * TabStage<D>::STRIDE, rsqrtf((float)D) / dss,
                            (float)row - 0.5f * (float)(n - 1), live,
                            dq + ((size_t)bh * n + (live ? row : 0)) * D, red + t * (D / 2 + 1),

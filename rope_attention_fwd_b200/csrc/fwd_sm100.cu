@@ -39,8 +39,8 @@
 // happens only when some row of the warp needs it, which after the first tiles is rare.
 // The final O / l is identical in exact arithmetic to rescaling at every tile.
 //
-// Exponentials: 2^x on the MUFU unit (ex2.approx), except one pair in eight, which goes
-// through the FMA pipe (exp2_poly2: range reduction and a degree-3 polynomial, relative
+// Exponentials: 2^x on the MUFU unit (ex2.approx), except one pair in eight (one in four at
+// d = 64), which goes through the FMA pipe (exp2_poly2: range reduction and a degree-3 polynomial, relative
 // error below 7.6e-5, far inside P's bf16 rounding).  With two softmax warpgroups per tile
 // and two tiles, the MUFU unit is the softmax's busiest; the split relieves it.
 //
@@ -376,11 +376,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const float2 x2 =
               ffma2(make_float2(__uint_as_float(sr[c][2 * i2]), __uint_as_float(sr[c][2 * i2 + 1])),
                     make_float2(scale_log2, scale_log2), make_float2(-m_use, -m_use));
-          // one pair in eight on the FMA pipe, off the MUFU unit that both tiles' softmax
-          // share (measured on 2 x 32 x 8192 x 128 causal: one in eight -3.5 to -5%, one in
-          // four -2 to -4%, one in two -2%)
-          const float2 p2 = (i2 & 7) == 7 ? exp2_poly2(x2)
-                                          : make_float2(fast_exp2(x2.x), fast_exp2(x2.y));
+          // some pairs on the FMA pipe, off the MUFU unit that both tiles' softmax share:
+          // one in eight at d = 128 (2 x 32 x 8192 x 128 causal: one in eight -3.5 to -5%,
+          // one in four -2 to -4%, one in two -2%), one in four at d = 64, where a tile
+          // carries half the tensor work for the same exponentials (4 x 16 x 2048 x 64
+          // causal: -4 to -5%)
+          constexpr int kPolyEvery = D == 64 ? 4 : 8;
+          const float2 p2 = i2 % kPolyEvery == kPolyEvery - 1
+                                ? exp2_poly2(x2)
+                                : make_float2(fast_exp2(x2.x), fast_exp2(x2.y));
           pv[2 * i2] = p2.x;
           pv[2 * i2 + 1] = p2.y;
         }

@@ -27,6 +27,17 @@ bool tensor_map_2d(CUtensorMap* map, const void* ptr, bool f32, uint64_t inner, 
 cudaEvent_t timing_begin(cudaStream_t s);
 void timing_end(cudaEvent_t start, int kid, cudaStream_t s);
 
+// timing_begin at construction, timing_end when the scope is left (early returns included).
+struct TimingScope {
+  cudaEvent_t start;
+  int kid;
+  cudaStream_t s;
+  TimingScope(int k, cudaStream_t st) : start(timing_begin(st)), kid(k), s(st) {}
+  ~TimingScope() { timing_end(start, kid, s); }
+  TimingScope(const TimingScope&) = delete;
+  TimingScope& operator=(const TimingScope&) = delete;
+};
+
 struct DevCtl {
   uint32_t* err;        // workspace error word
   uint64_t wait_ns;     // bound on every device-side wait

@@ -94,15 +94,13 @@ ra_status rope_attn_proj_fwd(const ra_problem* p, int64_t d_model, const void* x
     if (!ra::gemm_operand_map(&am[0], spec, false, x, rows, dm)) return RA_ERR_CUDA;
     for (int w = 0; w < 3; ++w)
       if (!ra::gemm_operand_map(&bm[w], spec, true, W[w], dm, hd)) return RA_ERR_CUDA;
-    const cudaEvent_t t0 = ra::timing_begin(s);
+    const ra::TimingScope timed(ra::K_PROJ_GEMM, s);
     e = ra::launch_gemm_bf16(spec, am, bm, out, static_cast<uint32_t*>(ws), ra::wait_limit_ns(),
                              s);
-    ra::timing_end(t0, ra::K_PROJ_GEMM, s);
   } else {
     const void* a[1] = {x};
-    const cudaEvent_t t0 = ra::timing_begin(s);
+    const ra::TimingScope timed(ra::K_PROJ_GEMM, s);
     e = ra::launch_gemm_f32(spec, a, dm, 0, W, hd, 0, out, s);
-    ra::timing_end(t0, ra::K_PROJ_GEMM, s);
   }
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
@@ -129,9 +127,11 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
   for (int w = 0; w < 3; ++w) {
     Y[w] = merged_at(ws, p, w);
     // Y_w = the gradient merged to [B n, H d] rows (row (b, i) holds every head of position i)
-    const cudaEvent_t t0 = ra::timing_begin(s);
-    const cudaError_t em = ra::launch_merge_heads(*p, G[w], Y[w], s);
-    ra::timing_end(t0, ra::K_MERGE_HEADS, s);
+    cudaError_t em;
+    {
+      const ra::TimingScope timed(ra::K_MERGE_HEADS, s);
+      em = ra::launch_merge_heads(*p, G[w], Y[w], s);
+    }
     if (em != cudaSuccess) return RA_ERR_CUDA;
   }
   // [dW_Q | dW_K | dW_V] (d_model x 3 H d) = X^T [Y_Q | Y_K | Y_V]: A = X MN-major,
@@ -159,24 +159,24 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
           !ra::gemm_operand_map(&ya[w], sx, false, Y[w], rows, hd) ||
           !ra::gemm_operand_map(&wb[w], sx, true, W[w], dm, hd))
         return RA_ERR_CUDA;
-    cudaEvent_t t0 = ra::timing_begin(s);
-    e = ra::launch_gemm_bf16(sw, xa, yb, ow, err, wait, s);
-    ra::timing_end(t0, ra::K_PROJ_DW, s);
+    {
+      const ra::TimingScope timed(ra::K_PROJ_DW, s);
+      e = ra::launch_gemm_bf16(sw, xa, yb, ow, err, wait, s);
+    }
     if (e == cudaSuccess) {
-      t0 = ra::timing_begin(s);
+      const ra::TimingScope timed(ra::K_PROJ_DX, s);
       e = ra::launch_gemm_bf16(sx, ya, wb, ox, err, wait, s);
-      ra::timing_end(t0, ra::K_PROJ_DX, s);
     }
   } else {
     const void* xs[1] = {x};
     const void* ys[3] = {Y[0], Y[1], Y[2]};
-    cudaEvent_t t0 = ra::timing_begin(s);
-    e = ra::launch_gemm_f32(sw, xs, dm, 0, ys, hd, 0, ow, s);
-    ra::timing_end(t0, ra::K_PROJ_DW, s);
+    {
+      const ra::TimingScope timed(ra::K_PROJ_DW, s);
+      e = ra::launch_gemm_f32(sw, xs, dm, 0, ys, hd, 0, ow, s);
+    }
     if (e == cudaSuccess) {
-      t0 = ra::timing_begin(s);
+      const ra::TimingScope timed(ra::K_PROJ_DX, s);
       e = ra::launch_gemm_f32(sx, ys, hd, 0, W, hd, 0, ox, s);
-      ra::timing_end(t0, ra::K_PROJ_DX, s);
     }
   }
   return e == cudaSuccess ? RA_OK : RA_ERR_CUDA;

@@ -208,7 +208,7 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
   const GemmOut os{{S, S, S}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
   const GemmOut op{{dP, dP, dP}, GEMM_OUT_F32, n, 1, n, 0, 0, 0};
   // timed as one unit: its launches run per head and per block of query rows
-  const cudaEvent_t t0 = timing_begin(s);
+  const TimingScope timed(K_SPECTRUM, s);
   if (launch_table(*p, alpha, table, s) != cudaSuccess) return RA_ERR_CUDA;
   if (cudaMemsetAsync(g64, 0, (size_t)M * (2 * n - 1) * sizeof(double2), s) != cudaSuccess)
     return RA_ERR_CUDA;
@@ -242,7 +242,6 @@ ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, 
   }
   spectrum_final_kernel<<<M, 256, 0, s>>>(g64, alpha, g, dalpha, n, d, p->base,
                                           M - p->fixed_bands);
-  timing_end(t0, K_SPECTRUM, s);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 

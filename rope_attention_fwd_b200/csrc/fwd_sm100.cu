@@ -40,9 +40,12 @@
 // The final O / l is identical in exact arithmetic to rescaling at every tile.
 //
 // Exponentials: 2^x on the MUFU unit (ex2.approx), except one pair in eight (one in four at
-// d = 64), which goes through the FMA pipe (exp2_poly2: range reduction and a degree-3 polynomial, relative
-// error below 7.6e-5, far inside P's bf16 rounding).  With two softmax warpgroups per tile
-// and two tiles, the MUFU unit is the softmax's busiest; the split relieves it.
+// d = 64), which goes through the FMA pipe (exp2_poly2: range reduction and a degree-3
+// polynomial, relative error below 7.6e-5, far inside P's bf16 rounding).  With two softmax
+// warpgroups per tile and two tiles, the MUFU unit is the softmax's busiest; the split
+// relieves it.  P is written while the two warpgroups of a tile exchange their partial row
+// maxima (the exchange only decides whether to rescale), and scaled in TMEM in the rare
+// case that the exchange moves the reference max.
 //
 // Every wait is bounded; an expired wait records RA_ERR_TIMEOUT in the workspace error
 // word and the CTA drains its copies and MMAs and exits.
@@ -336,46 +339,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int i = 8; i < 64; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
       float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                        fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      // the row max over both halves, through TMEM columns and the tile's exchange barrier
-      // (phase j; a bounded wait, like every other)
-      {
-        uint32_t w1[1] = {__float_as_uint(mh)};
-        tmem_st1(x_mine, w1);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_XCH + x]);
-        if (!mbar_wait_warp(&bar[B_XCH + x], j & 1, abort_flag, err, KID, 12, wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t o1 = tmem_ld1(x_other);
-        mh = fmaxf(mh, __uint_as_float(o1));
-      }
-      const float mt = mh * scale_log2;
-      // lazy rescale: move the reference max only when some row of the warp needs it (both
-      // warpgroups of a tile see the same row maxima, so they decide alike)
-      const bool need = mt > m + kRescaleTau;
-      const bool warp_rescale = __any_sync(0xffffffffu, need);
-      float corr = 1.f;
-      if (warp_rescale) {
-        const float m_new = fmaxf(m, mt);
-        corr = fast_exp2(m - m_new);  // 0 on the first tile (m = -inf)
-        m = m_new;
-      }
-      const float m_use = m == -CUDART_INF_F ? 0.f : m;
-      // P = 2^(s scale - m), summed and written as bf16 pairs: columns 64h + 32c .. + 31 land
-      // in S columns 64h + 16c .. + 15 (masked entries give 2^-inf = 0)
-      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      // P = 2^(s scale - mu) for the 32 columns 64h + 32c .. + 31, summed into sp and written
+      // as bf16 pairs into S columns 64h + 16c .. + 15 (masked entries give 0)
+      auto write_p = [&](int c, float mu, float (&sp)[8]) {
         float pv[32];
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) {
           const float2 x2 =
               ffma2(make_float2(__uint_as_float(sr[c][2 * i2]), __uint_as_float(sr[c][2 * i2 + 1])),
-                    make_float2(scale_log2, scale_log2), make_float2(-m_use, -m_use));
+                    make_float2(scale_log2, scale_log2), make_float2(-mu, -mu));
           // some pairs on the FMA pipe, off the MUFU unit that both tiles' softmax share:
           // one in eight at d = 128 (2 x 32 x 8192 x 128 causal: one in eight -3.5 to -5%,
           // one in four -2 to -4%, one in two -2%), one in four at d = 64, where a tile
@@ -399,8 +371,83 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) w[i2] = pack_bf16x2(pv[2 * i2], pv[2 * i2 + 1]);
         tmem_st16(s_base + 64 * h + 16 * c, w);
+      };
+      // P depends on the row max only through the rescale decision: unless this half
+      // already sees a rescale coming (or there is no reference max yet), P is written
+      // against the current reference max while the partial maxima are exchanged.  If the
+      // exchange then moves the reference max (the other half's maximum ran ahead by more
+      // than kRescaleTau, which is rare after the first tiles), the P already in TMEM is
+      // scaled by corr = 2^(m_old - m_new) <= 1: exact up to one more bf16 rounding, and
+      // this half's entries are at most 2^kRescaleTau before it.  The two forms sit in
+      // separate branches so that the early one keeps no score register alive across the
+      // exchange.
+      const bool early =
+          __all_sync(0xffffffffu, m != -CUDART_INF_F && !(mh * scale_log2 > m + kRescaleTau));
+      // the row max over both halves, through TMEM columns and the tile's exchange barrier
+      // (phase j; a bounded wait, like every other): posted here, read by take_max
+      {
+        uint32_t w1[1] = {__float_as_uint(mh)};
+        tmem_st1(x_mine, w1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_XCH + x]);
       }
-      l = l * corr + (((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7])));
+      // the other half's max in; then the lazy rescale: move the reference max only when
+      // some row of the warp needs it (both warpgroups of a tile see the same row maxima, so
+      // they decide alike); corr = 2^(m_old - m_new), 0 on the first tile (m = -inf)
+      float corr = 1.f;
+      bool warp_rescale = false;
+      auto take_max = [&]() -> bool {
+        if (!mbar_wait_warp(&bar[B_XCH + x], j & 1, abort_flag, err, KID, 12, wait_ns))
+          return false;
+        tc_fence_after();
+        mh = fmaxf(mh, __uint_as_float(tmem_ld1(x_other)));
+        const float mt = mh * scale_log2;
+        warp_rescale = __any_sync(0xffffffffu, mt > m + kRescaleTau);
+        if (warp_rescale) {
+          const float m_new = fmaxf(m, mt);
+          corr = fast_exp2(m - m_new);
+          m = m_new;
+        }
+        return true;
+      };
+      float psum;
+      {
+        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (early) {
+          write_p(0, m, sp);
+          write_p(1, m, sp);
+          psum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+          if (!take_max()) {
+            ok = false;
+            break;
+          }
+          if (warp_rescale) {
+            // this half's 64 P values, two per column in S columns 64h .. 64h + 31
+            uint32_t pw[32];
+            tmem_wait_st();
+            tmem_ld32(s_base + 64 * h, pw);
+            tmem_wait_ld(pw);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              pw[i] = pack_bf16x2(__uint_as_float(pw[i] << 16) * corr,
+                                  __uint_as_float(pw[i] & 0xffff0000u) * corr);
+            tmem_st32(s_base + 64 * h, pw);
+            psum *= corr;
+          }
+        } else {
+          if (!take_max()) {
+            ok = false;
+            break;
+          }
+          const float m_use = m == -CUDART_INF_F ? 0.f : m;
+          write_p(0, m_use, sp);
+          write_p(1, m_use, sp);
+          psum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        }
+      }
+      l = l * corr + psum;
       tmem_wait_st();
       if (warp_rescale && j > 0) {
         // O_x must hold every P_x(j') V_j' with j' < j: wait for the PV MMA of step j-1;

@@ -20,6 +20,8 @@ every rank -- is an NCCL all-reduce of d/2 floats per step.
 method; the pages ship no code) on a bounded sample of the same workload.
 """
 import argparse
+import atexit
+import datetime
 import json
 import os
 import statistics
@@ -59,14 +61,18 @@ def config_dict(wl, cfg, world):
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 50 ms, timestamped) from before the warm-up to the end of
+    the timed passes; summary() keeps the samples inside the windows mark() recorded."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.windows = []
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -74,34 +80,62 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader", "-lms", "200"],
+                 "--format=csv,noheader", "-lms", str(self.PERIOD_MS)],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+        atexit.register(self.stop)   # never left running if the bench fails in between
         return self
 
-    def __exit__(self, *a):
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+            self.proc = None
+
+    def __exit__(self, *a):
+        self.stop()
+
+    def window(self):
+        """Context manager marking a timed region (wall clock, as nvidia-smi stamps it)."""
+        sampler = self
+
+        class _Window:
+            def __enter__(self):
+                self.t0 = datetime.datetime.now()
+                return self
+
+            def __exit__(self, *a):
+                sampler.windows.append((self.t0, datetime.datetime.now()))
+        return _Window()
+
+    @staticmethod
+    def parse(lines, windows):
+        """(sm MHz, max MHz, [hw_slowdown, hw_thermal, sw_thermal, sw_power_cap]) of the
+        samples stamped inside any window."""
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                sm = float(parts[2].split()[0])
+                mx = float(parts[3].split()[0])
+            except ValueError:
+                continue
+            if any(a <= ts <= b for a, b in windows):
+                rows.append((sm, mx, parts[6:10]))
+        return rows
 
     def summary(self):
         rows = []
         if self.path and os.path.exists(self.path):
-            for line in open(self.path):
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm = float(parts[1].split()[0])
-                    mx = float(parts[2].split()[0])
-                except ValueError:
-                    continue
-                rows.append((sm, mx, parts[5:9]))
+            with open(self.path) as f:
+                rows = self.parse(f, self.windows)
             os.remove(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
@@ -229,6 +263,7 @@ def run_ours(args):
 
     stream = torch.cuda.current_stream(dev)
     # ---------------- device-resident timing
+    clk = ClockSampler(local).__enter__()   # running before the timed passes begin
     for _ in range(args.warmup):
         step(dv_in, out0)
     barrier()
@@ -238,8 +273,8 @@ def run_ours(args):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # the headline: whole steps, no per-kernel events between the launches (those would
     # serialise the dQ kernel behind the dK/dV kernel, which it may otherwise overlap)
-    with ClockSampler(local) as clk:
-        barrier()
+    barrier()
+    with clk.window():
         ev0.record(stream)
         for _ in range(args.steps):
             step(dv_in, out0)
@@ -247,17 +282,20 @@ def run_ours(args):
         barrier()
     ms = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(ms)
-    clocks = clk.summary()
     value = world * flops / (ms * 1e-3) / 1e12
     # the per-kernel breakdown (and the roofline's kernel durations): the same steps again,
     # each launch bracketed by the library's own events on the launching stream
     rb.rope_attn_timing_read()
     rb.rope_attn_timing_enable(True)
     barrier()
-    for _ in range(args.steps):
-        step(dv_in, out0)
-    barrier()
+    with clk.window():
+        for _ in range(args.steps):
+            step(dv_in, out0)
+        barrier()
     rb.rope_attn_timing_enable(False)
+    # clocks: the samples taken inside the two timed passes of the same steps
+    clk.stop()
+    clocks = clk.summary()
     kernels = rb.rope_attn_timing_read()
     launches = sum(c for c, _ in kernels.values())
 

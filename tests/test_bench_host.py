@@ -1,5 +1,6 @@
 """Host logic of bench.py that needs no GPU: the DRAM-traffic record is reported only while
-the kernel's code (comments aside, optionally a span of its file) is the captured one."""
+the kernel's code (comments aside, optionally a span of its file) is the captured one, and
+the clock summary keeps only the nvidia-smi samples taken inside the timed windows."""
 import hashlib
 import json
 import os
@@ -50,3 +51,22 @@ def test_traffic_tracks_code_not_comments(tmp_path, monkeypatch):
     src.write_text(SRC.replace("y = 2", "y = 3"))
     assert (bench.traffic_for("a"), bench.traffic_for("b"), bench.traffic_for("whole")) == \
         (10, None, None)
+
+
+def test_clock_samples_inside_windows_only():
+    import datetime
+    rows = [
+        "2026/12/03 10:39:12.900, 0, 1200 MHz, 1965 MHz, 90.0 W, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 10:39:13.100, 0, 1965 MHz, 1965 MHz, 700.0 W, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 10:39:13.150, 0, 1950 MHz, 1965 MHz, 710.0 W, 0x4, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 10:39:14.000, 0, 1100 MHz, 1965 MHz, 500.0 W, 0x8, Active, Not Active, Not Active, Not Active",
+        "2026/12/03 10:39:15.050, 0, 1965 MHz, 1965 MHz, 650.0 W, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "not a sample",
+    ]
+    t = lambda s, us: datetime.datetime(2026, 12, 3, 10, 39, s, us)
+    windows = [(t(13, 0), t(13, 500000)), (t(15, 0), t(15, 100000))]
+    got = bench.ClockSampler.parse(rows, windows)
+    assert [r[0] for r in got] == [1965.0, 1950.0, 1965.0]
+    assert [r[2][3] for r in got] == ["Active", "Active", "Not Active"]
+    # the idle sample before and the slowed one between the windows are left out
+    assert bench.ClockSampler.parse(rows, []) == []

@@ -439,15 +439,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
           const float4 l4 = lv[8 * h + c4], d4 = dvv[8 * h + c4];
-          const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
           float pv[4], dsv[4];
+          // columns in pairs, in packed f32x2 arithmetic (each lane rounded as the scalar
+          // instruction): x = s log2e/sqrt(d) - lse2, P = 2^x, and dS s = P fma(dP, s, -Delta s),
+          // which rounds exactly like P (dP - Delta) s because s is a power of two
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;  // column within this half
-            float p = fast_exp2(__uint_as_float(sr[c]) * scale_log2 - la[e]);
-            if (need_mask && (i0 + 32 * h + c < key)) p = 0.f;
-            pv[e] = p;
-            dsv[e] = p * (__uint_as_float(dr[c]) - da[e]) * dss;
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = 4 * c4 + 2 * e2;  // column within this half
+            const float2 la2 = e2 == 0 ? make_float2(l4.x, l4.y) : make_float2(l4.z, l4.w);
+            const float2 da2 = e2 == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
+            const float2 x2 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])),
+                                    make_float2(scale_log2, scale_log2), make_float2(-la2.x, -la2.y));
+            float2 p2 = make_float2(fast_exp2(x2.x), fast_exp2(x2.y));
+            if (need_mask) {
+              if (i0 + 32 * h + c < key) p2.x = 0.f;
+              if (i0 + 32 * h + c + 1 < key) p2.y = 0.f;
+            }
+            const float2 nd2 = fmul2(da2, make_float2(-dss, -dss));
+            const float2 ds2 = fmul2(
+                p2, ffma2(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                          make_float2(dss, dss), nd2));
+            pv[2 * e2] = p2.x;
+            pv[2 * e2 + 1] = p2.y;
+            dsv[2 * e2] = ds2.x;
+            dsv[2 * e2 + 1] = ds2.y;
           }
           pw[2 * c4] = pack_bf16x2(pv[0], pv[1]);
           pw[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);

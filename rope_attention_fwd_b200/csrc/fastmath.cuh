@@ -44,6 +44,13 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return d;
 }
 
+// max(a, b, c) in one instruction (sm_100); for non-NaN inputs exactly max(max(a, b), c).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x for a pair on the FMA pipe instead of the MUFU unit.  Cody-Waite range reduction:
 // x = j + f with j the nearest integer (adding and subtracting 1.5 * 2^23 rounds x to an
 // integer, which also sits in the low bits of the sum) and |f| <= 1/2; 2^f from a degree-3

@@ -332,13 +332,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= nvalid) sr[c][i] = __float_as_uint(-CUDART_INF_F);
       }
+      // the row max of this half: 8 independent chains of three-input maxima
+      auto sv = [&](int i) { return __uint_as_float(sr[i / 32][i % 32]); };
       float mp[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mp[a] = __uint_as_float(sr[0][a]);
-#pragma unroll
-      for (int i = 8; i < 64; ++i) mp[i & 7] = fmaxf(mp[i & 7], __uint_as_float(sr[i / 32][i % 32]));
-      float mh = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      for (int a = 0; a < 8; ++a) {
+        float t = fmax3(sv(a), sv(a + 8), sv(a + 16));
+        t = fmax3(t, sv(a + 24), sv(a + 32));
+        t = fmax3(t, sv(a + 40), sv(a + 48));
+        mp[a] = fmaxf(t, sv(a + 56));
+      }
+      float mh = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]),
+                       fmaxf(mp[6], mp[7]));
       // P = 2^(s scale - mu) for the 32 columns 64h + 32c .. + 31, summed into sp and written
       // as bf16 pairs into S columns 64h + 16c .. + 15 (masked entries give 0)
       auto write_p = [&](int c, float mu, float (&sp)[8]) {

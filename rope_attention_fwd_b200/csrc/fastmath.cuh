@@ -53,10 +53,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // 2^x for a pair on the FMA pipe instead of the MUFU unit.  Cody-Waite range reduction:
 // x = j + f with j the nearest integer (adding and subtracting 1.5 * 2^23 rounds x to an
-// integer, which also sits in the low bits of the sum) and |f| <= 1/2; 2^f from a degree-3
-// polynomial whose coefficients were fitted for this library by least squares in relative
-// error on Chebyshev nodes of [-1/2, 1/2] (maximum relative error 7.5e-5); j goes into the
-// exponent field with one integer add.  x is clamped below at -126, so the result is then
+// integer, which also sits in the low bits of the sum) and |f| <= 1/2; 2^f from the degree-3
+// minimax polynomial in relative error on [-1/2, 1/2], computed for this library with the
+// Remez exchange algorithm (maximum relative error 7.48e-5; tests/test_fastmath.py
+// re-derives the coefficients); j goes into the exponent field with one integer add.  x is clamped below at -126, so the result is then
 // at most 2^-126 rather than 0; callers pass x <= 2^7.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23

@@ -54,7 +54,7 @@ def test_packed_pairs_round_like_scalars(probe):
 
 
 # ---------------------------------------------------------------- exp2_poly2
-EXP2_REL_ERR = 7.6e-5   # the fitted polynomial's bound (7.5e-5) plus float32 rounding
+EXP2_REL_ERR = 7.6e-5   # the minimax cubic's bound (7.48e-5) plus float32 rounding
 
 
 def _poly_coefficients():
@@ -90,6 +90,48 @@ def test_exp2_poly_relative_error_cpu():
     y = _exp2_poly_cpu(x).astype(np.float64)
     rel = np.abs(y / np.exp2(x.astype(np.float64)) - 1.0)
     assert rel.max() <= EXP2_REL_ERR, rel.max()
+
+
+def _remez_relative(deg, a, b, grid_points=200_001, iters=30):
+    """Best uniform (minimax) polynomial approximation of 2^x on [a, b] in relative error,
+    by the Remez exchange algorithm: solve p(x_i) - 2^x_i = (-1)^i E 2^x_i on deg + 2
+    reference points, move each point to the extremum of the error on its sign-alternating
+    segment, repeat.  Returns the coefficients (constant first) and the maximum error."""
+    import numpy as np
+    n = deg + 2
+    k = np.arange(n)
+    xs = (a + b) / 2 + (b - a) / 2 * np.cos(np.pi * k[::-1] / (n - 1))
+    grid = np.linspace(a, b, grid_points)
+    fg = np.exp2(grid)
+    for _ in range(iters):
+        f = np.exp2(xs)
+        m = np.hstack([np.stack([xs ** j for j in range(deg + 1)], 1),
+                       ((-1.0) ** k * f)[:, None]])
+        c = np.linalg.solve(m, f)[:-1]
+        e = np.polyval(c[::-1], grid) / fg - 1.0
+        sign = np.sign(e)
+        cuts = np.flatnonzero(sign[1:] != sign[:-1]) + 1
+        idx = np.array([s0 + np.argmax(np.abs(e[s0:s1]))
+                        for s0, s1 in zip(np.r_[0, cuts], np.r_[cuts, len(e)])])
+        while len(idx) > n:
+            idx = idx[1:] if abs(e[idx[0]]) < abs(e[idx[-1]]) else idx[:-1]
+        if len(idx) < n:
+            break
+        xs = grid[idx]
+    return c, np.abs(e).max()
+
+
+def test_exp2_poly_coefficients_are_the_minimax_cubic():
+    """The constants of exp2_poly2 are the degree-3 minimax approximation of 2^f in relative
+    error on [-1/2, 1/2] (the range the round-to-nearest split leaves), re-derived here from
+    the definition; their own error is that minimax error."""
+    import numpy as np
+    c, err = _remez_relative(3, -0.5, 0.5)
+    got = np.array(_poly_coefficients())
+    assert np.abs(got - c).max() <= 1e-6, (got, c)
+    x = np.linspace(-0.5, 0.5, 200_001)
+    own = np.abs(np.polyval(got[::-1], x) / np.exp2(x) - 1.0).max()
+    assert own <= err * 1.001 and err <= 7.5e-5, (own, err)
 
 
 def test_exp2_poly_clamp_cpu():

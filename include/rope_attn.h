@@ -73,7 +73,8 @@ typedef enum {
 
 typedef enum { RA_F32 = 0, RA_BF16 = 1 } ra_dtype;
 
-/* Problem description, passed by pointer to every call. */
+/* Problem description, passed by pointer to every call.  Limits (RA_ERR_UNSUPPORTED
+ * beyond them): B, H, n <= 2^30; B*H <= 2^30 (fp32: <= 65535); B*H*n*d <= 2^38. */
 typedef struct {
     int64_t B, H, n, d;  /* batch, heads, sequence length, head dimension      */
     int32_t dtype;       /* ra_dtype of Q, K, V, O, E, dO, dQ, dK, dV          */

@@ -90,7 +90,16 @@ ra_status check_problem(const ra_problem* p) {
   if (p->dtype != RA_F32 && p->dtype != RA_BF16) return RA_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return RA_ERR_INVALID_ARG;
   if (!(p->base > 0.0) || !std::isfinite(p->base)) return RA_ERR_INVALID_ARG;
-  if (p->n > (int64_t(1) << 30) || p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
+  // Size limits, each tested before a product that could overflow: every byte count and
+  // grid size the launchers form from B, H, n and d then fits its type (B H n d <= 2^38
+  // elements is 512 GiB per bf16 tensor, beyond any one device).
+  if (p->B > (int64_t(1) << 30) || p->H > (int64_t(1) << 30) || p->n > (int64_t(1) << 30))
+    return RA_ERR_UNSUPPORTED;
+  if (p->B * p->H > (int64_t(1) << 30)) return RA_ERR_UNSUPPORTED;
+  if (p->d > 128) return RA_ERR_UNSUPPORTED;
+  if (p->B * p->H * p->n > (int64_t(1) << 38) / p->d) return RA_ERR_UNSUPPORTED;
+  // the fp32 kernels put (batch, head) on the grid's y dimension
+  if (p->dtype == RA_F32 && p->B * p->H > 65535) return RA_ERR_UNSUPPORTED;
   if (p->fixed_bands < 0 || p->fixed_bands > p->d / 2 || p->reserved != 0)
     return RA_ERR_INVALID_ARG;
   if (p->d > 128) return RA_ERR_UNSUPPORTED;

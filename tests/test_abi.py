@@ -34,6 +34,17 @@ def test_status_strings():
     assert lib.rope_attn_status_string(0) == b"ok"
 
 
+def test_size_limits_are_inclusive():
+    """The largest problems inside the limits still get a workspace size, computed without
+    overflow (it exceeds the bytes of the rotated Q~ and K~ alone)."""
+    for B, H, n, d, dt in [(1 << 8, 1 << 8, 1 << 16, 64, rb.RA_BF16),
+                           (1, 1, 1 << 30, 128, rb.RA_BF16), (1, 65535, 1 << 16, 64, rb.RA_F32)]:
+        p = rb.problem(B, H, n, d, dt, True, 1e4)
+        elems = B * H * n * d
+        assert elems <= 1 << 38
+        assert rb.rope_attn_workspace_bytes(p) > 2 * elems * (2 if dt == rb.RA_BF16 else 4)
+
+
 def test_workspace_bytes():
     elems = 2 * 32 * 8192 * 128
     p = rb.problem(2, 32, 8192, 128, rb.RA_BF16, True, 1e4)
@@ -57,12 +68,17 @@ def test_invalid_problem_has_no_workspace(bad):
 
 @pytest.mark.parametrize("bad, code", [
     (dict(d=96, dtype=rb.RA_BF16), 2), (dict(d=256), 2), (dict(d=32, dtype=rb.RA_BF16), 2),
+    # sizes whose products would overflow, or that no device holds
+    (dict(B=1 << 32, H=1 << 32), 2), (dict(B=1 << 31), 2), (dict(n=(1 << 30) + 1), 2),
+    (dict(B=1 << 15, H=1 << 15, n=1 << 30), 2), (dict(B=1 << 20, H=1 << 10, n=1 << 12), 2),
+    (dict(H=65536, n=64), 2),
 ])
 def test_unsupported_problem(bad, code):
     args = dict(B=1, H=1, n=16, d=64, dtype=rb.RA_F32, causal=0, base=1e4)
     args.update(bad)
     p = rb.RaProblem(args["B"], args["H"], args["n"], args["d"], args["dtype"], args["causal"],
                      args["base"])
+    assert rb.rope_attn_workspace_bytes(p) == 0
     lib = rb.lib()
     null = ctypes.c_void_p(0)
     r = lib.rope_attn_fwd(ctypes.byref(p), null, null, null, null, null, null, null, 0, null)

@@ -144,7 +144,8 @@ ra_status rope_attn_bwd_saved(const ra_problem* p, const void* v, const void* o,
  * fp32.  The library's own GEMMs: bf16 on the tcgen05 tensor cores (d in {64, 128},
  * d_model a multiple of 8, else RA_ERR_UNSUPPORTED), fp32 on CUDA cores (exact fp32
  * products); fp32 accumulation in a fixed order (deterministic).  Pointers 16-byte
- * aligned; d_model in 1..2^20.  Only p's B, H, n, d and dtype are used.
+ * aligned; d_model in 1..2^20.  Only p's B, H, n, d and dtype are used; B, H, n, d <= 2^30,
+ * B*n and 3*H*d <= 2^30, B*H*n*d <= 2^38 (RA_ERR_UNSUPPORTED beyond).
  * ws / ws_bytes (both calls): caller workspace, 256-byte aligned, of at least
  * rope_attn_proj_workspace_bytes(p) bytes for rope_attn_proj_bwd and at least 1024 bytes
  * for rope_attn_proj_fwd (RA_ERR_WORKSPACE otherwise).  Its first 64 bytes are the device
@@ -180,8 +181,8 @@ ra_status rope_attn_proj_bwd(const ra_problem* p, int64_t d_model, const void* x
  * Outputs: g [d/2][2n-1][2] fp32 (re, im; offset D at index D + n - 1; causal: D < 0 is 0)
  * and dalpha [d/2] fp32.  A diagnostic: one (batch, head) and one block of 64 query rows at
  * a time, with 64 x n fp32 scratch for the block's score matrices (fp32 CUDA-core GEMMs;
- * workspace from rope_attn_spectrum_workspace_bytes, O(n d); n <= 32768); sums in a fixed
- * order (deterministic). */
+ * workspace from rope_attn_spectrum_workspace_bytes, O(n d); n <= 32768; B, H <= 2^30,
+ * B*H <= 2^30, B*H*n*d <= 2^38); sums in a fixed order (deterministic). */
 size_t rope_attn_spectrum_workspace_bytes(const ra_problem* p);
 ra_status rope_attn_spectrum(const ra_problem* p, const void* q, const void* k, const void* v,
                              const void* o, const float* lse, const void* dO,

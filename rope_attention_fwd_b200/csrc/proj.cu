@@ -32,9 +32,14 @@ ra_status check(const ra_problem* p, int64_t d_model) {
     return RA_ERR_INVALID_ARG;
   if (p->dtype != RA_F32 && p->dtype != RA_BF16) return RA_ERR_INVALID_ARG;
   if (d_model < 1 || d_model > (int64_t(1) << 20)) return RA_ERR_INVALID_ARG;
-  // 32-bit GEMM sizes
+  // 32-bit GEMM sizes; each factor is bounded before a product is formed, so no product
+  // overflows and every byte count fits a size_t
+  if (p->B > (int64_t(1) << 30) || p->n > (int64_t(1) << 30) || p->H > (int64_t(1) << 30) ||
+      p->d > (int64_t(1) << 30))
+    return RA_ERR_UNSUPPORTED;
   if (p->B * p->n > (int64_t(1) << 30) || 3 * p->H * p->d > (int64_t(1) << 30))
     return RA_ERR_UNSUPPORTED;
+  if (p->B * p->n * p->H * p->d > (int64_t(1) << 38)) return RA_ERR_UNSUPPORTED;
   // the tensor-core GEMM: every 64-wide box inside one head and one weight (d in {64, 128}),
   // 16-byte rows for the tensor maps (d_model a multiple of 8)
   if (p->dtype == RA_BF16 && ((p->d != 64 && p->d != 128) || d_model % 8 != 0))

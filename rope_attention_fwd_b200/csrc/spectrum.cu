@@ -160,10 +160,14 @@ SpecLayout spec_layout(const ra_problem& p) {
 }
 
 bool spec_ok(const ra_problem* p) {
-  return p && p->B >= 1 && p->H >= 1 && p->n >= 1 && p->n <= 32768 && p->d >= 2 &&
-         p->d <= 128 && (p->d % 2) == 0 && (p->dtype == RA_F32 || p->dtype == RA_BF16) &&
-         (p->causal == 0 || p->causal == 1) && p->base > 0.0 && std::isfinite(p->base) &&
-         p->fixed_bands >= 0 && p->fixed_bands <= p->d / 2 && p->reserved == 0;
+  // B and H bounded before their product, and B H n d within the attention calls' limit
+  return p && p->B >= 1 && p->H >= 1 && p->B <= (int64_t(1) << 30) &&
+         p->H <= (int64_t(1) << 30) && p->B * p->H <= (int64_t(1) << 30) && p->n >= 1 &&
+         p->n <= 32768 && p->d >= 2 && p->d <= 128 && (p->d % 2) == 0 &&
+         p->B * p->H * p->n * p->d <= (int64_t(1) << 38) &&
+         (p->dtype == RA_F32 || p->dtype == RA_BF16) && (p->causal == 0 || p->causal == 1) &&
+         p->base > 0.0 && std::isfinite(p->base) && p->fixed_bands >= 0 &&
+         p->fixed_bands <= p->d / 2 && p->reserved == 0;
 }
 
 bool al16(const void* x) { return x && (reinterpret_cast<uintptr_t>(x) % 16) == 0; }

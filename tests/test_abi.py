@@ -176,6 +176,13 @@ def test_projection_validation_before_any_call():
     p2 = rb.problem(1, 1, 8, 2, rb.RA_F32, False, 1e4)
     need2 = rb.rope_attn_proj_workspace_bytes(p2)
     assert lib.rope_attn_proj_bwd(ctypes.byref(p2), 16, *[fake] * 11, fake, need2, None) == 2
+    # sizes whose products would overflow get no workspace and are refused
+    for B, H, n in [(1 << 40, 1, 1 << 30), (1, 1 << 40, 64), (1 << 20, 1 << 10, 1 << 10),
+                    (1 << 15, 1 << 14, 1 << 15)]:
+        big = rb.problem(B, H, n, 64, rb.RA_BF16, False, 1e4)
+        assert rb.rope_attn_proj_workspace_bytes(big) == 0
+        assert lib.rope_attn_proj_fwd(ctypes.byref(big), 256, *[fake] * 7, fake, 1 << 40,
+                                      None) == 2
 
 
 def test_spectrum_validation_before_any_call():
@@ -198,6 +205,11 @@ def test_spectrum_validation_before_any_call():
     assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, fake, need - 1, None) == 3
     assert lib.rope_attn_spectrum(ctypes.byref(p), *[fake] * 9, ctypes.c_void_p(4096 + 16),
                                   need, None) == 3
+    # B and H large enough to overflow their product are refused
+    for B, H in [(1 << 32, 1 << 32), (1 << 31, 1), (1 << 16, 1 << 16)]:
+        big = rb.problem(B, H, 96, 64, rb.RA_BF16, True, 1e4)
+        assert rb.rope_attn_spectrum_workspace_bytes(big) == 0
+        assert lib.rope_attn_spectrum(ctypes.byref(big), *[fake] * 9, fake, 1 << 40, None) == 1
 
 
 def test_header_is_plain_c_and_links(tmp_path):

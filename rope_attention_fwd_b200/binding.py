@@ -119,6 +119,21 @@ def _check(fn, code):
         raise RopeAttnError(fn, code)
 
 
+def _expect(fn, device, *args):
+    """The C ABI takes raw pointers to dense row-major buffers on one device: every tensor
+    argument (name, tensor, element count or None) must be contiguous, on `device` and,
+    where a count is given, hold exactly that many elements."""
+    for name, t, count in args:
+        if t is None:
+            continue
+        if t.device != device:
+            raise ValueError(f"{fn}: {name} is on {t.device}, expected {device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{fn}: {name} is not contiguous")
+        if count is not None and t.numel() != count:
+            raise ValueError(f"{fn}: {name} has {t.numel()} elements, expected {count}")
+
+
 def rope_attn_workspace_bytes(prob):
     return int(lib().rope_attn_workspace_bytes(ctypes.byref(prob)))
 
@@ -147,6 +162,9 @@ def rope_attn_fwd(q, k, v, alpha, base, causal, ws=None, o=None, lse=None, fixed
         ws = workspace(prob, q.device)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
+    N = q.numel()
+    _expect("rope_attn_fwd", q.device, ("q", q, None), ("k", k, N), ("v", v, N),
+            ("alpha", alpha, d // 2), ("o", o, N), ("lse", lse, B * H * n), ("ws", ws, None))
     _check("rope_attn_fwd", lib().rope_attn_fwd(
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(o), _ptr(lse),
         _ptr(ws), ws.numel(), _stream(q.device)))
@@ -160,6 +178,9 @@ def rope_attn_fwd_noalloc(q, k, v, alpha, base, causal, o=None, lse=None, fixed_
     B, H, n, d = q.shape
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device) if lse is None else lse
+    N = q.numel()
+    _expect("rope_attn_fwd_noalloc", q.device, ("q", q, None), ("k", k, N), ("v", v, N),
+            ("alpha", alpha, d // 2), ("o", o, N), ("lse", lse, B * H * n))
     # the library uses the static array of the CURRENT device: make it q's
     with torch.cuda.device(q.device):
         _check("rope_attn_fwd_noalloc", lib().rope_attn_fwd_noalloc(
@@ -185,6 +206,9 @@ def rope_attn_loss(o, e, ws=None, L=None, dO=None, causal=False, base=10000.0):
         ws = workspace(prob, o.device)
     L = torch.empty((), dtype=torch.float32, device=o.device) if L is None else L
     dO = torch.empty_like(o) if dO is None else dO
+    N = o.numel()
+    _expect("rope_attn_loss", o.device, ("o", o, None), ("e", e, N), ("L", L, 1), ("dO", dO, N),
+            ("ws", ws, None))
     _check("rope_attn_loss", lib().rope_attn_loss(
         ctypes.byref(prob), _ptr(o), _ptr(e), _ptr(L), _ptr(dO), _ptr(ws), ws.numel(),
         _stream(o.device)))
@@ -205,6 +229,11 @@ def rope_attn_bwd(q, k, v, o, lse, dO, alpha, base, causal, ws=None, dq=None, dk
         dalpha = None
     elif dalpha is None:
         dalpha = torch.empty_like(alpha)
+    B, H, n, d = q.shape
+    N = q.numel()
+    _expect("rope_attn_bwd", q.device, ("q", q, None), ("k", k, N), ("v", v, N), ("o", o, N),
+            ("lse", lse, B * H * n), ("dO", dO, N), ("alpha", alpha, d // 2), ("dq", dq, N),
+            ("dk", dk, N), ("dv", dv, N), ("dalpha", dalpha, d // 2), ("ws", ws, None))
     _check("rope_attn_bwd", lib().rope_attn_bwd(
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
         _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(),
@@ -224,6 +253,11 @@ def rope_attn_bwd_saved(v, o, lse, dO, alpha, base, causal, ws, dq=None, dk=None
         dalpha = None
     elif dalpha is None:
         dalpha = torch.empty_like(alpha)
+    B, H, n, d = v.shape
+    N = v.numel()
+    _expect("rope_attn_bwd_saved", v.device, ("v", v, None), ("o", o, N), ("lse", lse, B * H * n),
+            ("dO", dO, N), ("alpha", alpha, d // 2), ("dq", dq, N), ("dk", dk, N), ("dv", dv, N),
+            ("dalpha", dalpha, d // 2), ("ws", ws, None))
     _check("rope_attn_bwd_saved", lib().rope_attn_bwd_saved(
         ctypes.byref(prob), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha), _ptr(dq),
         _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(v.device)))
@@ -240,6 +274,9 @@ def rope_attn_proj_fwd(x, wq, wk, wv, H, q=None, k=None, v=None, ws=None):
            for t in (q, k, v)]
     if ws is None:
         ws = torch.empty(1024, dtype=torch.uint8, device=x.device)
+    W, Y = dm * H * d, B * H * n * d
+    _expect("rope_attn_proj_fwd", x.device, ("x", x, None), ("wq", wq, W), ("wk", wk, W),
+            ("wv", wv, W), ("q", out[0], Y), ("k", out[1], Y), ("v", out[2], Y), ("ws", ws, None))
     _check("rope_attn_proj_fwd", lib().rope_attn_proj_fwd(
         ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), *[_ptr(t) for t in out],
         _ptr(ws), ws.numel(), _stream(x.device)))
@@ -257,6 +294,9 @@ def rope_attn_proj_bwd(x, wq, wk, wv, dq, dk, dv):
     dx = torch.empty((B, n, dm), **f32)
     ws = torch.empty(int(lib().rope_attn_proj_workspace_bytes(ctypes.byref(prob))),
                      dtype=torch.uint8, device=x.device)
+    W, Y = dm * H * d, dq.numel()
+    _expect("rope_attn_proj_bwd", x.device, ("x", x, B * n * dm), ("wq", wq, W), ("wk", wk, W),
+            ("wv", wv, W), ("dq", dq, None), ("dk", dk, Y), ("dv", dv, Y))
     _check("rope_attn_proj_bwd", lib().rope_attn_proj_bwd(
         ctypes.byref(prob), dm, _ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk),
         _ptr(dv), *[_ptr(t) for t in dws], _ptr(dx), _ptr(ws), ws.numel(), _stream(x.device)))
@@ -272,6 +312,9 @@ def rope_attn_spectrum(q, k, v, o, lse, dO, alpha, base, causal, fixed_bands=0):
                      dtype=torch.uint8, device=q.device)
     g = torch.empty((d // 2, 2 * n - 1, 2), dtype=torch.float32, device=q.device)
     dalpha = torch.empty(d // 2, dtype=torch.float32, device=q.device)
+    N = q.numel()
+    _expect("rope_attn_spectrum", q.device, ("q", q, None), ("k", k, N), ("v", v, N), ("o", o, N),
+            ("lse", lse, B * H * n), ("dO", dO, N), ("alpha", alpha, d // 2))
     _check("rope_attn_spectrum", lib().rope_attn_spectrum(
         ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(alpha),
         _ptr(g), _ptr(dalpha), _ptr(ws), ws.numel(), _stream(q.device)))
@@ -283,6 +326,9 @@ def rope_attn_alpha_adam(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999
     """One in-place Adam step (weight decay 0) of the fp32 device tensors alpha, m1, m2 from
     dalpha clipped to L2 norm clip_norm (clip_norm <= 0: no clipping); step is 1-based."""
     opt = RaAdam(float(lr), float(beta1), float(beta2), float(eps), float(clip_norm), int(step))
+    M = alpha.numel()
+    _expect("rope_attn_alpha_adam", alpha.device, ("alpha", alpha, None), ("dalpha", dalpha, M),
+            ("m1", m1, M), ("m2", m2, M))
     _check("rope_attn_alpha_adam", lib().rope_attn_alpha_adam(
         ctypes.byref(opt), alpha.numel(), _ptr(alpha), _ptr(dalpha), _ptr(m1), _ptr(m2),
         _stream(alpha.device)))
@@ -291,6 +337,7 @@ def rope_attn_alpha_adam(alpha, dalpha, m1, m2, step, lr, beta1=0.9, beta2=0.999
 
 def rope_attn_device_status(ws):
     """Synchronise the current stream and return (status code, [kernel, site, block])."""
+    _expect("rope_attn_device_status", ws.device, ("ws", ws, None))
     info = (ctypes.c_int32 * 3)()
     code = lib().rope_attn_device_status(_ptr(ws), ws.numel(), _stream(ws.device), info)
     return code, list(info)
